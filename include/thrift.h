@@ -1,0 +1,158 @@
+/*
+ * thrift.h -- C ABI of libthrift: selective mixed-precision (NVFP4 + FP16) attention
+ * forward on NVIDIA B200 (sm_100a).
+ *
+ * The method (ThriftAttention technical summary, gist.science 2605.23081, section
+ * "Methodologie"; the same text in the French version, "Methodologie : ThriftAttention"):
+ *   1. Q, K and V are split into blocks; every (query block i, key block j) pair gets the
+ *      importance score S^_ij = qbar_i . kbar_j, the dot product of the blocks' token means.
+ *   2. The k highest-scoring pairs (per batch and query head here) run in FP16; all other
+ *      pairs run in NVFP4 (E2M1 values, one E4M3 scale per 16 elements, one FP32 tensor
+ *      scale).
+ *   3. Both paths merge through one online softmax; the FP4 path quantises its probability
+ *      blocks with a two-level scheme (a per-row scale per key block, then the 16-element
+ *      E4M3 micro-scale).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named "device" point to GPU memory; all such memory is owned by the caller.
+ *     The library never allocates, never frees and never synchronises the device, except
+ *     thrift_get_device_status, which copies one word to the host and waits for it.
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default stream.  All
+ *     work is enqueued on it, in call order.
+ *   - Argument errors are detected on the host, return a status and launch nothing.
+ *     Errors that only the device can see (a bounded wait that ran out) are recorded in a
+ *     status word inside the workspace and read with thrift_get_device_status.
+ *   - Tensors are dense and row-major.  FP16 means IEEE binary16.
+ */
+#ifndef THRIFT_H
+#define THRIFT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  THRIFT_OK = 0,
+  THRIFT_ERR_INVALID_ARG = 1,  /* null pointer, bad size or inconsistent configuration */
+  THRIFT_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels implement */
+  THRIFT_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
+  THRIFT_ERR_TIMEOUT = 4,      /* device status only: a bounded wait inside a kernel ran out */
+  THRIFT_ERR_WORKSPACE = 5     /* workspace pointer null, misaligned or too small */
+} thrift_status;
+
+/* Problem description, passed by value-pointer; the library keeps no copy. */
+typedef struct {
+  int32_t B, Hq, Hkv, N, d;  /* batch, query heads, key/value heads (Hq % Hkv == 0),
+                                sequence length (queries = keys), head dim (64 or 128) */
+  int32_t causal;            /* 0 or 1: key t is visible to query r when t <= r */
+  int32_t block_q, block_k;  /* selection block sizes: block_q in {64,128}, block_k in {64,128};
+                                N must be a multiple of 128 and of block_k */
+  int32_t topk_abs;          /* >= 0: number of FP16 pairs per (batch, query head);
+                                -1: use topk_bp */
+  int32_t topk_bp;           /* budget in basis points of the valid pairs: k = ceil(bp*V/10000)
+                                (0 = uniform NVFP4 attention, 10000 = all pairs in FP16) */
+  float softmax_scale;       /* tau; 0 selects 1/sqrt(d) rounded to FP32 */
+} thrift_cfg;
+
+/* NVFP4 tensor view.  All pointers are device pointers owned by the caller.
+ * For an FP16 tensor viewed as [outer, N, d]:
+ *   group_axis 0 (Q, K): 16-element groups along d.
+ *       codes  [outer*N, d/2]   E2M1 nibbles, element 2t in the low nibble of byte t
+ *       scales [outer*N, d/16]  E4M3 bytes, one per group (canonical layout)
+ *   group_axis 1 (V):    16-element groups along N (tokens), stored transposed.
+ *       codes  [outer*d, N/2], scales [outer*d, N/16]
+ *   scales_mma: the same scale bytes in the layout the tensor cores read (rows in blocks of
+ *       128, groups in blocks of 4 = 64 elements; each 128x4 block is 512 contiguous bytes,
+ *       row r, group g at (r%32)*16 + ((r%128)/32)*4 + g%4; blocks ordered row-block major).
+ *       Size: thrift_nvfp4_scales_mma_bytes().
+ *   tensor_scale: one device float = amax|X| / 2688 (1 for an all-zero tensor). */
+typedef struct {
+  uint8_t* codes;
+  uint8_t* scales;
+  uint8_t* scales_mma;
+  float* tensor_scale;
+  int32_t group_axis;
+} thrift_nvfp4;
+
+/* Bytes of the scales_mma buffer of a tensor viewed as [outer, N, d] with this group axis. */
+size_t thrift_nvfp4_scales_mma_bytes(int64_t outer, int32_t N, int32_t d, int32_t group_axis);
+
+/* Workspace bytes the calls below need for this configuration (the maximum over
+ * thrift_quantize_nvfp4, thrift_block_select, thrift_attn_fwd).  thrift_attn_fwd_auto needs
+ * thrift_auto_workspace_bytes() instead.  The workspace must be 256-byte aligned device
+ * memory; its first 256 bytes hold the device status word and must be zeroed once before
+ * first use (thrift_reset_device_status does that). */
+size_t thrift_workspace_bytes(const thrift_cfg* cfg);
+
+/* NVFP4 quantisation (ThriftAttention "FP4-pad": the NVFP4 microscaling format).
+ * x: device FP16 [outer, N, d].  Writes codes, scales, scales_mma and tensor_scale of *out
+ * (group_axis taken from out->group_axis).  Per 16-element group: s_b = E4M3(amax16/6/s_t),
+ * codes = E2M1(x / (s_b * s_t)), all roundings to nearest even with saturation.
+ * Requirements: d in {64,128}; N % 128 == 0; outer >= 1.  Two kernels: a grid amax
+ * reduction into the workspace, then the encode pass. */
+thrift_status thrift_quantize_nvfp4(const void* x, int64_t outer, int32_t N, int32_t d,
+                                    const thrift_nvfp4* out, void* ws, size_t ws_bytes,
+                                    void* stream);
+
+/* Block selection (ThriftAttention "Heuristische Blokkenselectie").
+ * q: device FP16 [B,Hq,N,d]; k: device FP16 [B,Hkv,N,d].
+ * Outputs (device):
+ *   mask   [B,Hq,nQb,ceil(nKb/32)] u32: bit j%32 of word j/32 set when pair (i,j) is FP16
+ *   counts [B,Hq,nQb] i32: selected pairs in query block i
+ *   lists  [B,Hq,nQb,nKb] i16: the selected key blocks of query block i in ascending order
+ *          (entries past counts[i] are -1)
+ *   scores [B,Hq,nQb,nKb] float64 (may be NULL): S^_ij, -inf for causal-invalid pairs.
+ * nQb = N/block_q, nKb = N/block_k.  The means are exact FP16 sums in float64 divided by the
+ * block size; S^ has no softmax scale; ties in S^ go to the smaller index i*nKb + j. */
+thrift_status thrift_block_select(const void* q, const void* k, const thrift_cfg* cfg,
+                                  uint32_t* mask, int32_t* counts, int16_t* lists,
+                                  double* scores, void* ws, size_t ws_bytes, void* stream);
+
+/* Attention forward (ThriftAttention "Gemengd-Precisie Berekening & Samenvoeging").
+ * q, k, v: device FP16 [B,Hq,N,d], [B,Hkv,N,d], [B,Hkv,N,d] (used for the FP16 pairs);
+ * q4, k4 (group_axis 0) and v4 (group_axis 1): NVFP4 copies (used for the other pairs);
+ * mask/counts/lists: the selection of thrift_block_select.
+ * out: device FP16 [B,Hq,N,d]; lse: device float [B,Hq,N] (natural log of the softmax
+ * denominator of the tau-scaled scores; may be NULL).
+ * topk_bp == 0 (or topk_abs == 0): uniform NVFP4; q, k, v, mask, counts, lists may be NULL.
+ * topk_bp == 10000: every valid pair in FP16; q4, k4, v4 may be NULL.
+ * One persistent kernel: tcgen05 block-scaled FP4 and FP16 MMAs with TMEM accumulators,
+ * TMA-staged tiles, the probability blocks re-quantised per row and key block. */
+thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v,
+                              const thrift_nvfp4* q4, const thrift_nvfp4* k4,
+                              const thrift_nvfp4* v4, const uint32_t* mask,
+                              const int32_t* counts, const int16_t* lists, void* out,
+                              float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/* Workspace bytes of thrift_attn_fwd_auto (it also holds the NVFP4 copies and the selection). */
+size_t thrift_auto_workspace_bytes(const thrift_cfg* cfg);
+
+/* The whole path in one call: quantise Q, K, V, select, attend. */
+thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, void* out,
+                                   float* lse, const thrift_cfg* cfg, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* Zero the device status word at the start of the workspace (enqueued on stream). */
+thrift_status thrift_reset_device_status(void* ws, void* stream);
+
+/* Copy the device status word to *status_out (0 = no device-side error, otherwise a
+ * thrift_status).  Synchronises `stream`. */
+thrift_status thrift_get_device_status(const void* ws, void* stream, int32_t* status_out);
+
+/* Launch a kernel whose mbarrier wait can never complete; its bounded wait gives up after
+ * about `limit_cycles` SM clock cycles and records THRIFT_ERR_TIMEOUT in the status word.
+ * Exists so that tests can check the timeout path without hanging a GPU. */
+thrift_status thrift_debug_wait_timeout(void* ws, int64_t limit_cycles, void* stream);
+
+/* Static string for a status code. */
+const char* thrift_status_str(thrift_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* THRIFT_H */

@@ -1,0 +1,252 @@
+"""B200-native selective mixed-precision attention forward (NVFP4 + FP16).
+
+The method is the one the ThriftAttention technical summary describes ("Methodologie"):
+block-mean importance scores S^_ij = qbar_i . kbar_j, the top-k block pairs per head in FP16,
+every other pair in NVFP4, one online softmax over both.  All arithmetic runs in libthrift's
+sm_100a kernels; this module only allocates device memory with PyTorch, picks the current
+CUDA stream and passes pointers through the C ABI.
+
+    cfg = Config(B=1, Hq=32, Hkv=8, N=32768, d=128, causal=True, block_q=128, block_k=64,
+                 topk_bp=500)
+    out, lse = attn_fwd_auto(q, k, v, cfg)          # quantise + select + attend
+"""
+
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import ThriftError, check, load
+
+__all__ = ["Config", "NVFP4Tensor", "Selection", "Workspace", "quantize_nvfp4", "quantize_qkv",
+           "block_select", "attn_fwd", "attn_fwd_auto", "device_status", "reset_device_status",
+           "ThriftError", "load"]
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+@dataclasses.dataclass
+class Config:
+    """Problem description (thrift_cfg)."""
+
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    d: int
+    causal: bool
+    block_q: int = 128
+    block_k: int = 64
+    topk_abs: int = -1
+    topk_bp: int = 500
+    softmax_scale: float = 0.0
+
+    @classmethod
+    def from_workload(cls, w) -> "Config":
+        return cls(w.B, w.Hq, w.Hkv, w.N, w.d, bool(w.causal), w.block_q, w.block_k, w.topk_abs,
+                   w.topk_bp)
+
+    def c(self) -> _lib.CCfg:
+        return _lib.CCfg(self.B, self.Hq, self.Hkv, self.N, self.d, int(self.causal), self.block_q,
+                         self.block_k, self.topk_abs, self.topk_bp, self.softmax_scale)
+
+    @property
+    def n_qb(self) -> int:
+        return self.N // self.block_q
+
+    @property
+    def n_kb(self) -> int:
+        return self.N // self.block_k
+
+    @property
+    def mask_words(self) -> int:
+        return (self.n_kb + 31) // 32
+
+
+@dataclasses.dataclass
+class NVFP4Tensor:
+    """Device NVFP4 tensor (thrift_nvfp4): E2M1 codes, E4M3 scales (canonical and MMA layout),
+    FP32 tensor scale."""
+
+    codes: torch.Tensor
+    scales: torch.Tensor
+    scales_mma: torch.Tensor
+    tensor_scale: torch.Tensor
+    group_axis: int
+
+    @classmethod
+    def empty(cls, outer: int, N: int, d: int, group_axis: int, device) -> "NVFP4Tensor":
+        L = load()
+        if group_axis == 0:
+            cshape, sshape = (outer, N, d // 2), (outer, N, d // 16)
+        else:
+            cshape, sshape = (outer, d, N // 2), (outer, d, N // 16)
+        mma = int(L.thrift_nvfp4_scales_mma_bytes(outer, N, d, group_axis))
+        u8 = dict(dtype=torch.uint8, device=device)
+        return cls(torch.empty(cshape, **u8), torch.empty(sshape, **u8), torch.empty(mma, **u8),
+                   torch.empty(1, dtype=torch.float32, device=device), group_axis)
+
+    def c(self) -> _lib.CNVFP4:
+        return _lib.CNVFP4(self.codes.data_ptr(), self.scales.data_ptr(), self.scales_mma.data_ptr(),
+                           self.tensor_scale.data_ptr(), self.group_axis)
+
+
+@dataclasses.dataclass
+class Selection:
+    """Output of block_select: FP16-pair bitmask, per-row counts and sorted lists, scores."""
+
+    mask: torch.Tensor
+    counts: torch.Tensor
+    lists: torch.Tensor
+    scores: Optional[torch.Tensor]
+
+
+class Workspace:
+    """Caller-owned device scratch (256-byte aligned).  The first 256 bytes hold the device
+    status word, zeroed on creation."""
+
+    def __init__(self, nbytes: int, device):
+        self.buf = torch.zeros(max(int(nbytes), 256) + 256, dtype=torch.uint8, device=device)
+        off = (-self.buf.data_ptr()) % 256
+        self.view = self.buf[off:off + max(int(nbytes), 256)]
+        self.nbytes = self.view.numel()
+
+    @property
+    def ptr(self):
+        return ctypes.c_void_p(self.view.data_ptr())
+
+    @classmethod
+    def for_config(cls, cfg: Config, device, auto: bool = False) -> "Workspace":
+        L = load()
+        c = cfg.c()
+        n = L.thrift_auto_workspace_bytes(ctypes.byref(c)) if auto else L.thrift_workspace_bytes(ctypes.byref(c))
+        if n == 0:
+            raise ThriftError(_lib.THRIFT_ERR_UNSUPPORTED, "workspace size")
+        return cls(n, device)
+
+
+def quantize_nvfp4(x: torch.Tensor, group_axis: int, out: Optional[NVFP4Tensor] = None,
+                   ws: Optional[Workspace] = None) -> NVFP4Tensor:
+    """NVFP4 quantisation of a contiguous FP16 [.., N, d] CUDA tensor (thrift_quantize_nvfp4)."""
+    assert x.is_cuda and x.dtype == torch.float16 and x.is_contiguous()
+    *lead, N, d = x.shape
+    outer = 1
+    for s in lead:
+        outer *= s
+    if out is None:
+        out = NVFP4Tensor.empty(outer, N, d, group_axis, x.device)
+    if ws is None:
+        ws = Workspace(256, x.device)
+    c = out.c()
+    check(load().thrift_quantize_nvfp4(_ptr(x), outer, N, d, ctypes.byref(c), ws.ptr, ws.nbytes, _stream()),
+          "thrift_quantize_nvfp4")
+    return out
+
+
+def quantize_qkv(q, k, v, ws: Optional[Workspace] = None):
+    """Q, K grouped along d; V grouped along tokens."""
+    return quantize_nvfp4(q, 0, ws=ws), quantize_nvfp4(k, 0, ws=ws), quantize_nvfp4(v, 1, ws=ws)
+
+
+def block_select(q: torch.Tensor, k: torch.Tensor, cfg: Config, ws: Optional[Workspace] = None,
+                 want_scores: bool = False, out: Optional[Selection] = None) -> Selection:
+    """Block-mean scores and per-head top-k FP16 pairs (thrift_block_select)."""
+    dev = q.device
+    rows = cfg.B * cfg.Hq * cfg.n_qb
+    if out is None:
+        out = Selection(
+            torch.empty((cfg.B, cfg.Hq, cfg.n_qb, cfg.mask_words), dtype=torch.int32, device=dev),
+            torch.empty((cfg.B, cfg.Hq, cfg.n_qb), dtype=torch.int32, device=dev),
+            torch.empty((cfg.B, cfg.Hq, cfg.n_qb, cfg.n_kb), dtype=torch.int16, device=dev),
+            torch.empty((cfg.B, cfg.Hq, cfg.n_qb, cfg.n_kb), dtype=torch.float64, device=dev)
+            if want_scores else None)
+    assert out.counts.numel() == rows
+    if ws is None:
+        ws = Workspace.for_config(cfg, dev)
+    c = cfg.c()
+    check(load().thrift_block_select(_ptr(q), _ptr(k), ctypes.byref(c), _ptr(out.mask), _ptr(out.counts),
+                                     _ptr(out.lists), _ptr(out.scores), ws.ptr, ws.nbytes, _stream()),
+          "thrift_block_select")
+    return out
+
+
+def attn_fwd(q, k, v, q4: Optional[NVFP4Tensor], k4: Optional[NVFP4Tensor], v4: Optional[NVFP4Tensor],
+             sel: Optional[Selection], cfg: Config, out: Optional[torch.Tensor] = None,
+             lse: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None, want_lse: bool = True):
+    """Selective mixed-precision attention forward (thrift_attn_fwd).  Returns (out, lse)."""
+    ref = q if q is not None else q4.codes
+    dev = ref.device
+    if out is None:
+        out = torch.empty((cfg.B, cfg.Hq, cfg.N, cfg.d), dtype=torch.float16, device=dev)
+    if lse is None and want_lse:
+        lse = torch.empty((cfg.B, cfg.Hq, cfg.N), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = Workspace(256, dev)
+    c = cfg.c()
+    n4 = [None if t is None else t.c() for t in (q4, k4, v4)]
+    refs = [None if t is None else ctypes.byref(t) for t in n4]
+    check(load().thrift_attn_fwd(_ptr(q), _ptr(k), _ptr(v), refs[0], refs[1], refs[2],
+                                 None if sel is None else _ptr(sel.mask),
+                                 None if sel is None else _ptr(sel.counts),
+                                 None if sel is None else _ptr(sel.lists),
+                                 _ptr(out), _ptr(lse), ctypes.byref(c), ws.ptr, ws.nbytes, _stream()),
+          "thrift_attn_fwd")
+    return out, lse
+
+
+def attn_fwd_auto(q, k, v, cfg: Config, out=None, lse=None, ws: Optional[Workspace] = None,
+                  want_lse: bool = True):
+    """Quantise, select and attend in one call (thrift_attn_fwd_auto).  Returns (out, lse)."""
+    dev = q.device
+    if out is None:
+        out = torch.empty((cfg.B, cfg.Hq, cfg.N, cfg.d), dtype=torch.float16, device=dev)
+    if lse is None and want_lse:
+        lse = torch.empty((cfg.B, cfg.Hq, cfg.N), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = Workspace.for_config(cfg, dev, auto=True)
+    c = cfg.c()
+    check(load().thrift_attn_fwd_auto(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), ctypes.byref(c),
+                                      ws.ptr, ws.nbytes, _stream()), "thrift_attn_fwd_auto")
+    return out, lse
+
+
+def attn_debug_dump(q, k, v, q4, k4, v4, sel, cfg: Config, entry: int, ws: Optional[Workspace] = None):
+    """thrift_debug_attn_dump: (out, lse, dbg) with the raw S, PV operand row bytes and PV of one
+    entry of the first unit of CTA 0."""
+    ref = q if q is not None else q4.codes
+    dev = ref.device
+    out = torch.empty((cfg.B, cfg.Hq, cfg.N, cfg.d), dtype=torch.float16, device=dev)
+    lse = torch.empty((cfg.B, cfg.Hq, cfg.N), dtype=torch.float32, device=dev)
+    dbg = torch.full((128 * cfg.block_k + 64 * cfg.block_k + 128 * cfg.d,), float("nan"),
+                     dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = Workspace(256, dev)
+    c = cfg.c()
+    n4 = [None if t is None else t.c() for t in (q4, k4, v4)]
+    refs = [None if t is None else ctypes.byref(t) for t in n4]
+    check(load().thrift_debug_attn_dump(_ptr(q), _ptr(k), _ptr(v), refs[0], refs[1], refs[2],
+                                        None if sel is None else _ptr(sel.mask), _ptr(out), _ptr(lse),
+                                        ctypes.byref(c), ws.ptr, ws.nbytes, _ptr(dbg), entry, _stream()),
+          "thrift_debug_attn_dump")
+    return out, lse, dbg
+
+
+def reset_device_status(ws: Workspace) -> None:
+    check(load().thrift_reset_device_status(ws.ptr, _stream()), "thrift_reset_device_status")
+
+
+def device_status(ws: Workspace) -> int:
+    """The device status word (0 = no device-side error).  Synchronises the current stream."""
+    v = ctypes.c_int32(0)
+    check(load().thrift_get_device_status(ws.ptr, _stream(), ctypes.byref(v)), "thrift_get_device_status")
+    return int(v.value)

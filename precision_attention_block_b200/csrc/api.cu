@@ -1,0 +1,249 @@
+// The C ABI of libthrift (include/thrift.h): argument checks, workspace layout, launches on the
+// caller's stream.  The library allocates nothing; every buffer belongs to the caller.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "../../include/thrift.h"
+#include "../../include/thrift_debug.h"
+#include "thrift_internal.h"
+
+namespace thrift {
+
+thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
+                              const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
+                              void* out, float* lse, const thrift_cfg& c, int* status, float* dbg, int dbg_entry,
+                              cudaStream_t stream);
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+namespace {
+
+bool cfg_ok(const thrift_cfg* c) {
+  if (!c) return false;
+  if (c->B <= 0 || c->Hq <= 0 || c->Hkv <= 0 || c->N <= 0) return false;
+  if (c->Hq % c->Hkv != 0) return false;
+  if (c->causal != 0 && c->causal != 1) return false;
+  if (c->topk_abs < -1) return false;
+  if (c->topk_abs == -1 && (c->topk_bp < 0 || c->topk_bp > 10000)) return false;
+  if (!(c->softmax_scale >= 0.0f) || std::isinf(c->softmax_scale)) return false;
+  return true;
+}
+
+thrift_status cfg_supported(const thrift_cfg* c) {
+  if (!cfg_ok(c)) return THRIFT_ERR_INVALID_ARG;
+  if (c->d != 64 && c->d != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (c->block_q != 64 && c->block_q != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (c->block_k != 64 && c->block_k != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (c->N % 128 != 0 || c->N % c->block_k != 0) return THRIFT_ERR_UNSUPPORTED;
+  if (c->N / c->block_k > 32767) return THRIFT_ERR_UNSUPPORTED;
+  if ((int64_t)c->B * c->Hq * c->N > (int64_t)INT32_MAX / 2) return THRIFT_ERR_UNSUPPORTED;
+  return THRIFT_OK;
+}
+
+int attn_mode(const thrift_cfg* c) {
+  if (c->topk_abs == 0 || (c->topk_abs < 0 && c->topk_bp == 0)) return 1;
+  if (c->topk_abs < 0 && c->topk_bp == 10000) return 2;
+  return 0;
+}
+
+bool ws_ok(const void* ws, size_t have, size_t need) {
+  return ws && (reinterpret_cast<uintptr_t>(ws) % 256 == 0) && have >= need;
+}
+
+int* status_ptr(void* ws) { return reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + kWsStatusOff); }
+
+bool nvfp4_ok(const thrift_nvfp4* t, int axis) {
+  return t && t->codes && t->scales && t->scales_mma && t->tensor_scale && t->group_axis == axis;
+}
+
+struct AutoLayout {
+  size_t q4c, q4s, q4m, k4c, k4s, k4m, v4c, v4s, v4m, ts, mask, counts, lists, select, bytes;
+};
+
+AutoLayout auto_layout(const thrift_cfg& c) {
+  AutoLayout L;
+  size_t qn = (size_t)c.B * c.Hq * c.N * c.d, kn = (size_t)c.B * c.Hkv * c.N * c.d;
+  int64_t nqb = c.N / c.block_q, nkb = c.N / c.block_k;
+  size_t off = kWsHeader;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.q4c = take(qn / 2);
+  L.q4s = take(qn / 16);
+  L.q4m = take(scales_mma_bytes((int64_t)c.B * c.Hq, c.N, c.d, 0));
+  L.k4c = take(kn / 2);
+  L.k4s = take(kn / 16);
+  L.k4m = take(scales_mma_bytes((int64_t)c.B * c.Hkv, c.N, c.d, 0));
+  L.v4c = take(kn / 2);
+  L.v4s = take(kn / 16);
+  L.v4m = take(scales_mma_bytes((int64_t)c.B * c.Hkv, c.N, c.d, 1));
+  L.ts = take(3 * sizeof(float));
+  L.mask = take((size_t)c.B * c.Hq * nqb * ((nkb + 31) / 32) * 4);
+  L.counts = take((size_t)c.B * c.Hq * nqb * 4);
+  L.lists = take((size_t)c.B * c.Hq * nqb * nkb * 2);
+  L.select = take(select_layout(c).bytes);
+  L.bytes = off;
+  return L;
+}
+
+}  // namespace
+}  // namespace thrift
+
+using namespace thrift;
+
+extern "C" {
+
+size_t thrift_nvfp4_scales_mma_bytes(int64_t outer, int32_t N, int32_t d, int32_t group_axis) {
+  if (outer <= 0 || N <= 0 || d <= 0 || (group_axis != 0 && group_axis != 1)) return 0;
+  return scales_mma_bytes(outer, N, d, group_axis);
+}
+
+size_t thrift_workspace_bytes(const thrift_cfg* cfg) {
+  if (cfg_supported(cfg) != THRIFT_OK) return 0;
+  return kWsHeader + select_layout(*cfg).bytes;
+}
+
+size_t thrift_auto_workspace_bytes(const thrift_cfg* cfg) {
+  if (cfg_supported(cfg) != THRIFT_OK) return 0;
+  return auto_layout(*cfg).bytes;
+}
+
+thrift_status thrift_quantize_nvfp4(const void* x, int64_t outer, int32_t N, int32_t d, const thrift_nvfp4* out,
+                                    void* ws, size_t ws_bytes, void* stream) {
+  if (!x || outer <= 0 || N <= 0 || !out) return THRIFT_ERR_INVALID_ARG;
+  if (out->group_axis != 0 && out->group_axis != 1) return THRIFT_ERR_INVALID_ARG;
+  if (!nvfp4_ok(out, out->group_axis)) return THRIFT_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (N % 128 != 0) return THRIFT_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(x) % 16 != 0) return THRIFT_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, kWsHeader)) return THRIFT_ERR_WORKSPACE;
+  unsigned int* amax = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + kWsAmaxOff);
+  return quantize_launch(x, outer, N, d, out, amax, static_cast<cudaStream_t>(stream));
+}
+
+thrift_status thrift_block_select(const void* q, const void* k, const thrift_cfg* cfg, uint32_t* mask,
+                                  int32_t* counts, int16_t* lists, double* scores, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  thrift_status st = cfg_supported(cfg);
+  if (st != THRIFT_OK) return st;
+  if (!q || !k || !mask || !counts || !lists) return THRIFT_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, thrift_workspace_bytes(cfg))) return THRIFT_ERR_WORKSPACE;
+  return select_launch(q, k, *cfg, mask, counts, lists, scores, static_cast<uint8_t*>(ws) + kWsHeader,
+                       static_cast<cudaStream_t>(stream));
+}
+
+static thrift_status attn_common(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
+                                 const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, void* out,
+                                 float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes, float* dbg,
+                                 int dbg_entry, void* stream) {
+  thrift_status st = cfg_supported(cfg);
+  if (st != THRIFT_OK) return st;
+  if (!out) return THRIFT_ERR_INVALID_ARG;
+  int mode = attn_mode(cfg);
+  if (mode != 2 && (!nvfp4_ok(q4, 0) || !nvfp4_ok(k4, 0) || !nvfp4_ok(v4, 1))) return THRIFT_ERR_INVALID_ARG;
+  if (mode != 1 && (!q || !k || !v)) return THRIFT_ERR_INVALID_ARG;
+  if (mode == 0 && !mask) return THRIFT_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, kWsHeader)) return THRIFT_ERR_WORKSPACE;
+  return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, lse, *cfg, status_ptr(ws), dbg, dbg_entry,
+                         static_cast<cudaStream_t>(stream));
+}
+
+thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
+                              const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask,
+                              const int32_t* counts, const int16_t* lists, void* out, float* lse,
+                              const thrift_cfg* cfg, void* ws, size_t ws_bytes, void* stream) {
+  (void)counts;
+  (void)lists;
+  return attn_common(q, k, v, q4, k4, v4, mask, out, lse, cfg, ws, ws_bytes, nullptr, -1, stream);
+}
+
+thrift_status thrift_debug_attn_dump(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
+                                     const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask,
+                                     void* out, float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes,
+                                     float* dbg, int32_t dbg_entry, void* stream) {
+  if (!dbg) return THRIFT_ERR_INVALID_ARG;
+  return attn_common(q, k, v, q4, k4, v4, mask, out, lse, cfg, ws, ws_bytes, dbg, dbg_entry, stream);
+}
+
+thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, void* out, float* lse,
+                                   const thrift_cfg* cfg, void* ws, size_t ws_bytes, void* stream) {
+  thrift_status st = cfg_supported(cfg);
+  if (st != THRIFT_OK) return st;
+  if (!q || !k || !v || !out) return THRIFT_ERR_INVALID_ARG;
+  AutoLayout L = auto_layout(*cfg);
+  if (!ws_ok(ws, ws_bytes, L.bytes)) return THRIFT_ERR_WORKSPACE;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* ts = reinterpret_cast<float*>(w + L.ts);
+  thrift_nvfp4 q4 = {w + L.q4c, w + L.q4s, w + L.q4m, ts + 0, 0};
+  thrift_nvfp4 k4 = {w + L.k4c, w + L.k4s, w + L.k4m, ts + 1, 0};
+  thrift_nvfp4 v4 = {w + L.v4c, w + L.v4s, w + L.v4m, ts + 2, 1};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int* amax = reinterpret_cast<unsigned int*>(w + kWsAmaxOff);
+  int mode = attn_mode(cfg);
+  const thrift_cfg& c = *cfg;
+  if (mode != 2) {
+    if ((st = quantize_launch(q, (int64_t)c.B * c.Hq, c.N, c.d, &q4, amax, s)) != THRIFT_OK) return st;
+    if ((st = quantize_launch(k, (int64_t)c.B * c.Hkv, c.N, c.d, &k4, amax, s)) != THRIFT_OK) return st;
+    if ((st = quantize_launch(v, (int64_t)c.B * c.Hkv, c.N, c.d, &v4, amax, s)) != THRIFT_OK) return st;
+  }
+  uint32_t* mask = reinterpret_cast<uint32_t*>(w + L.mask);
+  if (mode == 0) {
+    st = select_launch(q, k, c, mask, reinterpret_cast<int32_t*>(w + L.counts), reinterpret_cast<int16_t*>(w + L.lists),
+                       nullptr, w + L.select, s);
+    if (st != THRIFT_OK) return st;
+  }
+  return attn_launch_dbg(q, k, v, &q4, &k4, &v4, mode == 0 ? mask : nullptr, mode, out, lse, c, status_ptr(ws),
+                         nullptr, -1, s);
+}
+
+thrift_status thrift_reset_device_status(void* ws, void* stream) {
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 != 0) return THRIFT_ERR_WORKSPACE;
+  return cudaMemsetAsync(ws, 0, kWsHeader, static_cast<cudaStream_t>(stream)) == cudaSuccess ? THRIFT_OK
+                                                                                               : THRIFT_ERR_CUDA;
+}
+
+thrift_status thrift_get_device_status(const void* ws, void* stream, int32_t* status_out) {
+  if (!ws || !status_out) return THRIFT_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, static_cast<const uint8_t*>(ws) + kWsStatusOff, sizeof(v), cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return THRIFT_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return THRIFT_ERR_CUDA;
+  *status_out = v;
+  return THRIFT_OK;
+}
+
+thrift_status thrift_debug_wait_timeout(void* ws, int64_t limit_cycles, void* stream) {
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 != 0) return THRIFT_ERR_WORKSPACE;
+  if (limit_cycles <= 0 || limit_cycles > (int64_t)1 << 34) return THRIFT_ERR_INVALID_ARG;
+  return wait_timeout_launch(status_ptr(ws), limit_cycles, static_cast<cudaStream_t>(stream));
+}
+
+const char* thrift_status_str(thrift_status s) {
+  switch (s) {
+    case THRIFT_OK: return "ok";
+    case THRIFT_ERR_INVALID_ARG: return "invalid argument";
+    case THRIFT_ERR_UNSUPPORTED: return "unsupported configuration";
+    case THRIFT_ERR_CUDA: return "CUDA error";
+    case THRIFT_ERR_TIMEOUT: return "device wait timed out";
+    case THRIFT_ERR_WORKSPACE: return "workspace null, misaligned or too small";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

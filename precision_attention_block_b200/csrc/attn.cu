@@ -1,0 +1,784 @@
+// Fused selective mixed-precision attention forward for sm_100a (ThriftAttention technical
+// summary, "Gemengd-Precisie Berekening & Samenvoeging" and the paragraph on its fused kernel).
+//
+// One persistent CTA per SM walks (batch, query head, 128-row query tile) units.  For each unit
+// the key blocks form a list of entries: first every key block that some row of the tile computes
+// in NVFP4, then every key block it computes in FP16 (the order the pages' kernel uses; the FP16
+// query tile is fetched only when the first FP16 entry comes up).  Warp roles:
+//   warp 0      TMA producer: the unit's NVFP4 query tile, the FP16 query tile on demand, and for
+//               every entry its K and V tiles (NVFP4 codes + scales, or FP16) into a slot ring.
+//   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of two TMEM score buffers, then the
+//               previous entry's PV into the TMEM PV buffer.  NVFP4 products use
+//               tcgen05.mma.kind::mxf4nvf4.block_scale.block16 with the E4M3 scale vectors copied
+//               into TMEM by tcgen05.cp; FP16 products use tcgen05.mma.kind::f16.
+//   warps 2-5   one thread per query row: read S from TMEM, causal mask, the row maximum M of the
+//               key block, P^ = exp(S - M); NVFP4 entries re-quantise P' = 2688 P^ with one E4M3
+//               scale per 16 keys into shared memory (the PV MMA's A operand), FP16 entries round
+//               P^ to FP16; then merge the previous entry's PV into the row's FP32 output with
+//               weight exp(M - m) (m = running maximum), and sum the unquantised P^ into l.
+// Every wait is bounded; on timeout the CTA records THRIFT_ERR_TIMEOUT and unwinds.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "sm100.cuh"
+#include "thrift_internal.h"
+
+namespace thrift {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kBQ = 128;
+constexpr long long kWaitLimit = 1ll << 32;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kSW128 = 2, kSW64 = 4, kSW32 = 6;
+
+__host__ __device__ constexpr int round1024(int x) { return (x + 1023) & ~1023; }
+__host__ __device__ constexpr int swz_for_row_bytes(int b) { return b == 128 ? kSW128 : (b == 64 ? kSW64 : kSW32); }
+
+template <int D, int BK>
+struct Layout {
+  static constexpr int Q4_BYTES = kBQ * D / 2;
+  static constexpr int QSF_BYTES = (D / 64) * 512;
+  static constexpr int Q16_BYTES = kBQ * D * 2;
+  static constexpr int SLOT_BYTES = BK * D * 2;
+  static constexpr int NSLOT = BK == 128 ? 3 : 6;
+  static constexpr int P16_BYTES = kBQ * BK * 2;
+  static constexpr int P4_BYTES = kBQ * BK / 2;
+  static constexpr int PSF_BYTES = (BK / 64) * 512;
+  static constexpr int PBUF_BYTES = round1024(P16_BYTES > P4_BYTES + PSF_BYTES ? P16_BYTES : P4_BYTES + PSF_BYTES);
+  static constexpr int OFF_Q4 = 0;
+  static constexpr int OFF_QSF = Q4_BYTES;
+  static constexpr int OFF_Q16 = round1024(OFF_QSF + QSF_BYTES);
+  static constexpr int OFF_SLOTS = OFF_Q16 + Q16_BYTES;
+  static constexpr int OFF_P = OFF_SLOTS + NSLOT * SLOT_BYTES;
+  static constexpr int OFF_BAR = OFF_P + 2 * PBUF_BYTES;
+  static constexpr int BYTES = OFF_BAR + 512 + 1024;  // barriers + alignment slack
+  // TMEM columns
+  static constexpr int COL_S = 0;  // two buffers of BK columns
+  static constexpr int COL_PV = 2 * BK;
+  static constexpr int COL_SFQ = COL_PV + D;
+  static constexpr int SFK_COLS = 4 * (D / 64);
+  static constexpr int SFKV_COLS = 4 * (BK / 64);
+  static constexpr int COL_SFK = COL_SFQ + SFK_COLS;        // two buffers
+  static constexpr int COL_SFV = COL_SFK + 2 * SFK_COLS;    // two buffers
+  static constexpr int COL_SFP = COL_SFV + 2 * SFKV_COLS;   // two buffers
+  static constexpr int TMEM_COLS_USED = COL_SFP + 2 * SFKV_COLS;
+  static_assert(TMEM_COLS_USED <= 512, "TMEM budget");
+  static_assert(BYTES <= 232448, "shared memory budget");
+};
+
+struct Bars {
+  uint64_t q_full, q_empty, q16_full, q16_empty;
+  uint64_t s_full[2], s_free[2], p_full[2];
+  uint64_t pv_full, pv_free;
+  uint64_t kv_full[6], kv_empty[6];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct AttnParams {
+  const uint32_t* mask;
+  const uint8_t* q_sf;
+  const uint8_t* k_sf;
+  const uint8_t* v_sf;
+  const float* q_ts;
+  const float* k_ts;
+  const float* v_ts;
+  __half* out;
+  float* lse;
+  int* status;
+  float* dbg;  // optional dump of one entry (S, P bytes, PV) of the first unit of CTA 0
+  int dbg_entry;
+  int B, Hq, Hkv, N, bq, causal, mode, nqb, nkb, mask_words, n_units;
+  float tau;
+  long long wait_limit;
+};
+
+// The entry list of one unit, regenerated identically by every role.
+struct EntryIter {
+  const uint32_t* m0;
+  const uint32_t* m1;
+  int jmax0, jmax1, jmax, two, mode, phase, j;
+
+  __device__ __forceinline__ int sel(const uint32_t* m, int jj) const {
+    if (mode == 2) return 1;
+    if (mode == 1) return 0;
+    return (int)((__ldg(m + (jj >> 5)) >> (jj & 31)) & 1u);
+  }
+  __device__ __forceinline__ bool next(int& j_out, int& f16_out, int& rm_out) {
+    while (phase < 2) {
+      while (j < jmax) {
+        int jj = j++;
+        int want = phase;
+        int rm = 0;
+        if (jj < jmax0 && sel(m0, jj) == want) rm |= 1;
+        if (two && jj < jmax1 && sel(m1, jj) == want) rm |= 2;
+        if (rm) {
+          j_out = jj;
+          f16_out = want;
+          rm_out = two ? rm : 3;
+          return true;
+        }
+      }
+      ++phase;
+      j = 0;
+    }
+    return false;
+  }
+};
+
+struct UnitInfo {
+  int b, h, hk, t;
+};
+
+__device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, int u) {
+  int bh_count = p.B * p.Hq;
+  int ntiles = p.N / kBQ;
+  UnitInfo ui;
+  ui.t = ntiles - 1 - u / bh_count;
+  int bh = u % bh_count;
+  ui.b = bh / p.Hq;
+  ui.h = bh % p.Hq;
+  ui.hk = ui.h / (p.Hq / p.Hkv);
+  return ui;
+}
+
+template <int BK>
+__device__ __forceinline__ EntryIter make_iter(const AttnParams& p, const UnitInfo& ui) {
+  EntryIter it;
+  it.mode = p.mode;
+  it.two = p.bq == 64;
+  int i0 = it.two ? 2 * ui.t : ui.t;
+  int i1 = i0 + 1;
+  const uint32_t* base = p.mask ? p.mask + ((int64_t)(ui.b * p.Hq + ui.h) * p.nqb) * p.mask_words : nullptr;
+  it.m0 = base ? base + (int64_t)i0 * p.mask_words : nullptr;
+  it.m1 = (base && it.two) ? base + (int64_t)i1 * p.mask_words : nullptr;
+  if (p.causal) {
+    it.jmax0 = ((i0 + 1) * p.bq - 1) / BK + 1;
+    it.jmax1 = it.two ? ((i1 + 1) * p.bq - 1) / BK + 1 : 0;
+  } else {
+    it.jmax0 = p.nkb;
+    it.jmax1 = it.two ? p.nkb : 0;
+  }
+  it.jmax = it.jmax0 > it.jmax1 ? it.jmax0 : it.jmax1;
+  it.phase = 0;
+  it.j = 0;
+  return it;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t a) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
+}
+
+template <int D, int BK>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q4, const __grid_constant__ CUtensorMap tm_k4,
+                const __grid_constant__ CUtensorMap tm_v4, const __grid_constant__ CUtensorMap tm_q16,
+                const __grid_constant__ CUtensorMap tm_k16, const __grid_constant__ CUtensorMap tm_v16,
+                const __grid_constant__ AttnParams p) {
+  using L = Layout<D, BK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023) & ~1023u) - raw_addr);
+  uint8_t* sQ4 = smem + L::OFF_Q4;
+  uint8_t* sQSF = smem + L::OFF_QSF;
+  uint8_t* sQ16 = smem + L::OFF_Q16;
+  uint8_t* sSlots = smem + L::OFF_SLOTS;
+  uint8_t* sP = smem + L::OFF_P;
+  Bars* bars = reinterpret_cast<Bars*>(smem + L::OFF_BAR);
+  volatile int* abort_flag = &bars->abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
+    mbar_init(&bars->q16_full, 1);
+    mbar_init(&bars->q16_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->s_free[i], 128);
+      mbar_init(&bars->p_full[i], 128);
+    }
+    mbar_init(&bars->pv_full, 1);
+    mbar_init(&bars->pv_free, 128);
+    for (int i = 0; i < L::NSLOT; ++i) {
+      mbar_init(&bars->kv_full[i], 1);
+      mbar_init(&bars->kv_empty[i], 1);
+    }
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const long long lim = p.wait_limit;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      if (p.mode != 2) {
+        prefetch_tmap(&tm_q4);
+        prefetch_tmap(&tm_k4);
+        prefetch_tmap(&tm_v4);
+      }
+      if (p.mode != 1) {
+        prefetch_tmap(&tm_q16);
+        prefetch_tmap(&tm_k16);
+        prefetch_tmap(&tm_v16);
+      }
+      uint32_t slot_ctr = 0, unit_ctr = 0, u16_ctr = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_ctr) {
+        UnitInfo ui = decode_unit(p, u);
+        const int qrow0 = (ui.b * p.Hq + ui.h) * p.N + ui.t * kBQ;
+        const int kvh = ui.b * p.Hkv + ui.hk;
+        if (!(ok = mbar_wait(&bars->q_empty, (unit_ctr & 1) ^ 1, abort_flag, p.status, lim))) break;
+        if (p.mode != 2) {
+          mbar_arrive_expect_tx(&bars->q_full, L::Q4_BYTES + L::QSF_BYTES);
+          tma_load_2d(sQ4, &tm_q4, &bars->q_full, 0, qrow0);
+          bulk_load(sQSF, p.q_sf + (size_t)(qrow0 / 128) * L::QSF_BYTES, L::QSF_BYTES, &bars->q_full);
+        } else {
+          mbar_arrive(&bars->q_full);
+        }
+        bool q16_loaded = false;
+        EntryIter it = make_iter<BK>(p, ui);
+        int j, f16, rm;
+        while (it.next(j, f16, rm)) {
+          if (f16 && !q16_loaded) {
+            if (!(ok = mbar_wait(&bars->q16_empty, (u16_ctr & 1) ^ 1, abort_flag, p.status, lim))) break;
+            mbar_arrive_expect_tx(&bars->q16_full, L::Q16_BYTES);
+#pragma unroll
+            for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(sQ16 + cb * kBQ * 128, &tm_q16, &bars->q16_full, cb * 64, qrow0);
+            q16_loaded = true;
+          }
+          const int krow0 = kvh * p.N + j * BK;
+          // K tile
+          {
+            uint32_t s = slot_ctr % L::NSLOT, ph = (slot_ctr / L::NSLOT) & 1;
+            ++slot_ctr;
+            if (!(ok = mbar_wait(&bars->kv_empty[s], ph ^ 1, abort_flag, p.status, lim))) break;
+            uint8_t* dst = sSlots + s * L::SLOT_BYTES;
+            if (f16) {
+              mbar_arrive_expect_tx(&bars->kv_full[s], BK * D * 2);
+#pragma unroll
+              for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(dst + cb * BK * 128, &tm_k16, &bars->kv_full[s], cb * 64, krow0);
+            } else {
+              mbar_arrive_expect_tx(&bars->kv_full[s], BK * D / 2 + L::QSF_BYTES);
+              tma_load_2d(dst, &tm_k4, &bars->kv_full[s], 0, krow0);
+              bulk_load(dst + BK * D / 2, p.k_sf + (size_t)(krow0 / 128) * L::QSF_BYTES, L::QSF_BYTES, &bars->kv_full[s]);
+            }
+          }
+          // V tile
+          {
+            uint32_t s = slot_ctr % L::NSLOT, ph = (slot_ctr / L::NSLOT) & 1;
+            ++slot_ctr;
+            if (!(ok = mbar_wait(&bars->kv_empty[s], ph ^ 1, abort_flag, p.status, lim))) break;
+            uint8_t* dst = sSlots + s * L::SLOT_BYTES;
+            if (f16) {
+              mbar_arrive_expect_tx(&bars->kv_full[s], BK * D * 2);
+#pragma unroll
+              for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(dst + cb * BK * 128, &tm_v16, &bars->kv_full[s], cb * 64, krow0);
+            } else {
+              const int vrow0 = kvh * D;
+              mbar_arrive_expect_tx(&bars->kv_full[s], D * BK / 2 + L::PSF_BYTES);
+              tma_load_2d(dst, &tm_v4, &bars->kv_full[s], j * (BK / 2), vrow0);
+              size_t sf_off = ((size_t)(vrow0 / 128) * (p.N / 64) + (size_t)j * (BK / 64)) * 512;
+              bulk_load(dst + D * BK / 2, p.v_sf + sf_off, L::PSF_BYTES, &bars->kv_full[s]);
+            }
+          }
+        }
+        if (q16_loaded) ++u16_ctr;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk4 = idesc_nvf4(kBQ, BK);
+      const uint32_t idesc_pv4 = idesc_nvf4(kBQ, D);
+      const uint32_t idesc_qk16 = idesc_f16(kBQ, BK, 0, 0);
+      const uint32_t idesc_pv16 = idesc_f16(kBQ, D, 0, 1);
+      constexpr int SWQ = swz_for_row_bytes(D / 2);
+      constexpr int SWP = swz_for_row_bytes(BK / 2);
+      uint32_t slot_ctr = 0, unit_ctr = 0, u16_ctr = 0, g = 0;
+      bool ok = true;
+      struct Pend {
+        uint32_t g, vslot, vph;
+        int f16, sfv_off;
+      } pend = {0, 0, 0, 0, 0};
+      auto do_pv = [&](const Pend& e) -> bool {
+        const uint32_t buf = e.g & 1;
+        if (!mbar_wait(&bars->p_full[buf], (e.g >> 1) & 1, abort_flag, p.status, lim)) return false;
+        if (!mbar_wait(&bars->pv_free, (e.g & 1) ^ 1, abort_flag, p.status, lim)) return false;
+        if (!mbar_wait(&bars->kv_full[e.vslot], e.vph, abort_flag, p.status, lim)) return false;
+        tc_fence_after();
+        const uint32_t pbuf = smem_u32(sP + buf * L::PBUF_BYTES);
+        const uint32_t vbuf = smem_u32(sSlots + e.vslot * L::SLOT_BYTES);
+        if (e.f16) {
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            uint64_t ad = make_sdesc(pbuf + (kk >> 2) * kBQ * 128 + (kk & 3) * 32, 16, 1024, kSW128);
+            uint64_t bd = make_sdesc(vbuf + kk * 16 * 128, BK * 128, 1024, kSW128);
+            mma_f16(tmem + L::COL_PV, ad, bd, idesc_pv16, kk > 0);
+          }
+        } else {
+          const uint32_t sfv = tmem + L::COL_SFV + buf * L::SFKV_COLS;
+          const uint32_t sfp = tmem + L::COL_SFP + buf * L::SFKV_COLS;
+#pragma unroll
+          for (int kb = 0; kb < BK / 64; ++kb) {
+            tc_copy_sf(sfv + 4 * kb, make_sdesc(vbuf + D * BK / 2 + kb * 512, 16, 128, 0));
+            tc_copy_sf(sfp + 4 * kb, make_sdesc(pbuf + L::P4_BYTES + kb * 512, 16, 128, 0));
+          }
+#pragma unroll
+          for (int kb = 0; kb < BK / 64; ++kb) {
+            uint64_t ad = make_sdesc(pbuf + kb * 32, 16, 8 * (BK / 2), SWP);
+            uint64_t bd = make_sdesc(vbuf + kb * 32, 16, 8 * (BK / 2), SWP);
+            mma_nvf4(tmem + L::COL_PV, ad, bd, idesc_pv4, sfp + 4 * kb, sfv + 4 * kb + e.sfv_off, kb > 0);
+          }
+        }
+        tc_commit(&bars->pv_full);
+        tc_commit(&bars->kv_empty[e.vslot]);
+        return true;
+      };
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_ctr) {
+        UnitInfo ui = decode_unit(p, u);
+        const int kvh = ui.b * p.Hkv + ui.hk;
+        if (!(ok = mbar_wait(&bars->q_full, unit_ctr & 1, abort_flag, p.status, lim))) break;
+        tc_fence_after();
+        if (p.mode != 2) {
+#pragma unroll
+          for (int kk = 0; kk < D / 64; ++kk)
+            tc_copy_sf(tmem + L::COL_SFQ + 4 * kk, make_sdesc(smem_u32(sQSF) + kk * 512, 16, 128, 0));
+        }
+        bool any16 = false, have_pend = false;
+        EntryIter it = make_iter<BK>(p, ui);
+        int j, f16, rm;
+        while (ok && it.next(j, f16, rm)) {
+          uint32_t kslot = slot_ctr % L::NSLOT, kph = (slot_ctr / L::NSLOT) & 1;
+          ++slot_ctr;
+          uint32_t vslot = slot_ctr % L::NSLOT, vph = (slot_ctr / L::NSLOT) & 1;
+          ++slot_ctr;
+          if (f16 && !any16) {
+            if (!(ok = mbar_wait(&bars->q16_full, u16_ctr & 1, abort_flag, p.status, lim))) break;
+            any16 = true;
+          }
+          const uint32_t buf = g & 1;
+          if (!(ok = mbar_wait(&bars->kv_full[kslot], kph, abort_flag, p.status, lim))) break;
+          if (!(ok = mbar_wait(&bars->s_free[buf], ((g >> 1) & 1) ^ 1, abort_flag, p.status, lim))) break;
+          tc_fence_after();
+          const uint32_t kbuf = smem_u32(sSlots + kslot * L::SLOT_BYTES);
+          const uint32_t dS = tmem + L::COL_S + buf * BK;
+          if (f16) {
+            const uint32_t qb = smem_u32(sQ16);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              uint64_t ad = make_sdesc(qb + (kk >> 2) * kBQ * 128 + (kk & 3) * 32, 16, 1024, kSW128);
+              uint64_t bd = make_sdesc(kbuf + (kk >> 2) * BK * 128 + (kk & 3) * 32, 16, 1024, kSW128);
+              mma_f16(dS, ad, bd, idesc_qk16, kk > 0);
+            }
+          } else {
+            const int krow0 = kvh * p.N + j * BK;
+            const int sfk_off = (krow0 & 127) >> 5;
+            const uint32_t sfk = tmem + L::COL_SFK + buf * L::SFK_COLS;
+#pragma unroll
+            for (int kk = 0; kk < D / 64; ++kk)
+              tc_copy_sf(sfk + 4 * kk, make_sdesc(kbuf + BK * D / 2 + kk * 512, 16, 128, 0));
+            const uint32_t qb = smem_u32(sQ4);
+#pragma unroll
+            for (int kk = 0; kk < D / 64; ++kk) {
+              uint64_t ad = make_sdesc(qb + kk * 32, 16, 8 * (D / 2), SWQ);
+              uint64_t bd = make_sdesc(kbuf + kk * 32, 16, 8 * (D / 2), SWQ);
+              mma_nvf4(dS, ad, bd, idesc_qk4, tmem + L::COL_SFQ + 4 * kk, sfk + 4 * kk + sfk_off, kk > 0);
+            }
+          }
+          tc_commit(&bars->s_full[buf]);
+          tc_commit(&bars->kv_empty[kslot]);
+          if (have_pend && !(ok = do_pv(pend))) break;
+          pend.g = g;
+          pend.vslot = vslot;
+          pend.vph = vph;
+          pend.f16 = f16;
+          pend.sfv_off = ((kvh * D) & 127) >> 5;
+          have_pend = true;
+          ++g;
+        }
+        if (ok && have_pend) ok = do_pv(pend);
+        if (!ok) break;
+        tc_commit(&bars->q_empty);
+        if (any16) {
+          tc_commit(&bars->q16_empty);
+          ++u16_ctr;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax / merge
+    const int quarter = warp & 3;
+    const int rr = quarter * 32 + lane;  // row of the tile = TMEM lane
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const float q_ts = (p.mode != 2) ? __ldg(p.q_ts) : 1.0f;
+    const float k_ts = (p.mode != 2) ? __ldg(p.k_ts) : 1.0f;
+    const float v_ts = (p.mode != 2) ? __ldg(p.v_ts) : 1.0f;
+    const float sl2_4 = q_ts * k_ts * p.tau * kLog2e;
+    const float sl2_16 = p.tau * kLog2e;
+    const float pv4_scale = v_ts * (1.0f / 2688.0f);
+    const float NEG_INF = -__int_as_float(0x7f800000);
+    uint32_t g = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      UnitInfo ui = decode_unit(p, u);
+      const int row = ui.t * kBQ + rr;
+      const int half = (p.bq == 64) ? (rr >> 6) : 0;
+      float O[D];
+#pragma unroll
+      for (int c = 0; c < D; ++c) O[c] = 0.0f;
+      float m_run = NEG_INF, l_run = 0.0f;
+      float pend_M = NEG_INF, pend_sum = 0.0f;
+      int pend_f16 = 0;
+      bool have_pend = false;
+      const bool dbg_unit = p.dbg && blockIdx.x == 0 && u == (int)blockIdx.x;
+      int local_e = 0;
+
+      auto merge = [&](uint32_t ge) -> bool {
+        if (!mbar_wait(&bars->pv_full, ge & 1, abort_flag, p.status, lim)) return false;
+        tc_fence_after();
+        const float m_new = fmaxf(m_run, pend_M);
+        const float alpha = (m_run == NEG_INF) ? 0.0f : ex2(m_run - m_new);
+        const float gs = (pend_M == NEG_INF) ? 0.0f : ex2(pend_M - m_new);
+        const float gpv = pend_f16 ? gs : gs * pv4_scale;
+        l_run = alpha * l_run + gs * pend_sum;
+        const bool dump = dbg_unit && (local_e - 1) == p.dbg_entry;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + L::COL_PV + 32 * c, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float v = __uint_as_float(r[i]);
+            O[32 * c + i] = fmaf(gpv, v, alpha * O[32 * c + i]);
+            if (dump) p.dbg[kBQ * BK + kBQ * (BK * 2 / 4) + rr * D + 32 * c + i] = v;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->pv_free);
+        m_run = (m_new == NEG_INF) ? m_run : m_new;
+        return true;
+      };
+
+      EntryIter it = make_iter<BK>(p, ui);
+      int j, f16, rm;
+      while (it.next(j, f16, rm)) {
+        const uint32_t buf = g & 1;
+        if (!(ok = mbar_wait(&bars->s_full[buf], (g >> 1) & 1, abort_flag, p.status, lim))) break;
+        tc_fence_after();
+        const bool part = (rm >> half) & 1;
+        const bool diag = p.causal && (j * BK + BK - 1 > ui.t * kBQ);
+        const int key0 = j * BK;
+        const uint32_t saddr = tmem + lane_base + L::COL_S + buf * BK;
+        const float sl2 = f16 ? sl2_16 : sl2_4;
+        const bool dump = dbg_unit && local_e == p.dbg_entry;
+        // pass 1: maxima of every 16-key group
+        float gmax[BK / 16];
+#pragma unroll
+        for (int c = 0; c < BK / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(saddr + 32 * c, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            float mx = NEG_INF;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int col = 32 * c + 16 * h2 + i;
+              float s = __uint_as_float(r[16 * h2 + i]);
+              if (dump) p.dbg[rr * BK + col] = s;
+              const bool masked = !part || (diag && key0 + col > row);
+              mx = masked ? mx : fmaxf(mx, s);
+            }
+            gmax[2 * c + h2] = mx;
+          }
+        }
+        float M = NEG_INF;
+#pragma unroll
+        for (int q = 0; q < BK / 16; ++q) M = fmaxf(M, gmax[q]);
+        const bool valid = M != NEG_INF;
+        const float Ms = valid ? M * sl2 : 0.0f;
+        // pass 2: probabilities, their sum, and the PV operand in shared memory
+        const uint32_t pb = smem_u32(sP + buf * L::PBUF_BYTES);
+        float sum = 0.0f;
+        uint32_t sfw[BK / 64];
+#pragma unroll
+        for (int q = 0; q < BK / 64; ++q) sfw[q] = 0u;
+#pragma unroll
+        for (int c = 0; c < BK / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(saddr + 32 * c, r);
+          tmem_wait_ld();
+          float pr[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int col = 32 * c + i;
+            const bool masked = !valid || !part || (diag && key0 + col > row);
+            pr[i] = masked ? 0.0f : ex2(fmaf(__uint_as_float(r[i]), sl2, -Ms));
+            sum += pr[i];
+          }
+          if (f16) {
+            uint32_t hw[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) hw[i] = pack_half2(pr[2 * i], pr[2 * i + 1]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int chunk = 4 * c + q;  // 16-byte chunk index along the row (8 keys)
+              const int cb = chunk >> 3, c8 = chunk & 7;
+              const uint32_t addr = pb + cb * kBQ * 128 + rr * 128 + ((c8 ^ (rr & 7)) << 4);
+              st_shared_v4(addr, hw[4 * q], hw[4 * q + 1], hw[4 * q + 2], hw[4 * q + 3]);
+            }
+          } else {
+            uint32_t w[4];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const float gm = gmax[2 * c + h2];
+              const float pmax = (valid && gm != NEG_INF) ? 2688.0f * ex2(fmaf(gm, sl2, -Ms)) : 0.0f;
+              const uint32_t sb = cvt_e4m3(__fdiv_rn(pmax, 6.0f));
+              const float sbf = e4m3_to_f32(sb);
+              const float inv = sbf > 0.0f ? __fdiv_rn(2688.0f, sbf) : 0.0f;
+              uint32_t lo = 0, hi = 0;
+#pragma unroll
+              for (int i = 0; i < 8; i += 2) lo |= cvt_e2m1x2(pr[16 * h2 + i] * inv, pr[16 * h2 + i + 1] * inv) << (4 * i);
+#pragma unroll
+              for (int i = 0; i < 8; i += 2)
+                hi |= cvt_e2m1x2(pr[16 * h2 + 8 + i] * inv, pr[16 * h2 + 8 + i + 1] * inv) << (4 * i);
+              w[2 * h2] = lo;
+              w[2 * h2 + 1] = hi;
+              const int grp = 2 * c + h2;  // 16-key group index in the row
+              sfw[grp >> 2] |= sb << (8 * (grp & 3));
+            }
+            // 32 keys = one 16-byte chunk of the row
+            constexpr int ROWB = BK / 2;
+            uint32_t addr;
+            if (ROWB == 32)
+              addr = pb + rr * 32 + ((c ^ ((rr >> 2) & 1)) << 4);
+            else
+              addr = pb + rr * 64 + ((c ^ ((rr >> 1) & 3)) << 4);
+            st_shared_v4(addr, w[0], w[1], w[2], w[3]);
+          }
+        }
+        if (!f16) {
+#pragma unroll
+          for (int q = 0; q < BK / 64; ++q)
+            st_shared_u32(pb + L::P4_BYTES + q * 512 + (rr & 31) * 16 + (rr >> 5) * 4, sfw[q]);
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->s_free[buf]);
+        if (dump) {
+          // raw bytes of this row of the PV operand (FP16: BK halves; NVFP4: codes + scale bytes)
+          float* db = p.dbg + kBQ * BK + rr * (BK * 2 / 4);
+          const uint8_t* base = sP + buf * L::PBUF_BYTES;
+          if (f16) {
+            for (int ch = 0; ch < BK / 8; ++ch) {
+              const int cb = ch >> 3, c8 = ch & 7;
+              const uint4 v = *reinterpret_cast<const uint4*>(base + cb * kBQ * 128 + rr * 128 + ((c8 ^ (rr & 7)) << 4));
+              reinterpret_cast<uint4*>(db)[ch] = v;
+            }
+          } else {
+            constexpr int ROWB = BK / 2;
+            for (int ch = 0; ch < ROWB / 16; ++ch) {
+              int phys = ROWB == 32 ? (ch ^ ((rr >> 2) & 1)) : (ch ^ ((rr >> 1) & 3));
+              reinterpret_cast<uint4*>(db)[ch] = *reinterpret_cast<const uint4*>(base + rr * ROWB + (phys << 4));
+            }
+            for (int q = 0; q < BK / 64; ++q)
+              reinterpret_cast<uint32_t*>(db)[ROWB / 4 + q] = sfw[q];
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->p_full[buf]);
+        if (have_pend && !(ok = merge(g - 1))) break;
+        pend_M = valid ? Ms : NEG_INF;
+        pend_sum = sum;
+        pend_f16 = f16;
+        have_pend = true;
+        ++g;
+        ++local_e;
+      }
+      if (ok && have_pend) ok = merge(g - 1);
+      if (!ok) break;
+      // epilogue: O / l in FP16, lse in natural-log units of the tau-scaled scores
+      const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+      const int64_t orow = (int64_t)(ui.b * p.Hq + ui.h) * p.N + row;
+      uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        uint4 v;
+        v.x = pack_half2(O[8 * c] * inv_l, O[8 * c + 1] * inv_l);
+        v.y = pack_half2(O[8 * c + 2] * inv_l, O[8 * c + 3] * inv_l);
+        v.z = pack_half2(O[8 * c + 4] * inv_l, O[8 * c + 5] * inv_l);
+        v.w = pack_half2(O[8 * c + 6] * inv_l, O[8 * c + 7] * inv_l);
+        dst[c] = v;
+      }
+      if (p.lse) p.lse[orow] = (m_run + __log2f(l_run)) * kLn2;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2D map over a row-major [rows, inner] array (inner contiguous).
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t inner, uint64_t rows,
+              uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * (uint64_t)esize};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+CUtensorMapSwizzle swz_enum(int row_bytes) {
+  return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
+template <int D, int BK>
+thrift_status launch_t(const void* q, const void* k, const void* v, const thrift_nvfp4* q4, const thrift_nvfp4* k4,
+                       const thrift_nvfp4* v4, AttnParams& prm, cudaStream_t stream) {
+  using L = Layout<D, BK>;
+  CUtensorMap maps[6];
+  memset(maps, 0, sizeof(maps));
+  const uint64_t qrows = (uint64_t)prm.B * prm.Hq * prm.N, krows = (uint64_t)prm.B * prm.Hkv * prm.N;
+  bool ok = true;
+  if (prm.mode != 2) {
+    ok &= make_map(&maps[0], q4->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D / 2, qrows, D / 2, kBQ, swz_enum(D / 2));
+    ok &= make_map(&maps[1], k4->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D / 2, krows, D / 2, BK, swz_enum(D / 2));
+    ok &= make_map(&maps[2], v4->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)prm.N / 2,
+                   (uint64_t)prm.B * prm.Hkv * D, BK / 2, D, swz_enum(BK / 2));
+  }
+  if (prm.mode != 1) {
+    ok &= make_map(&maps[3], q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, D, qrows, 64, kBQ, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&maps[4], k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, D, krows, 64, BK, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&maps[5], v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, D, krows, 64, BK, CU_TENSOR_MAP_SWIZZLE_128B);
+  }
+  if (!ok) return THRIFT_ERR_CUDA;
+  auto kern = attn_kernel<D, BK>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES) != cudaSuccess)
+    return THRIFT_ERR_CUDA;
+  int grid = num_sms();
+  if (grid > prm.n_units) grid = prm.n_units;
+  kern<<<grid, kThreads, L::BYTES, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], prm);
+  return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
+}
+
+__global__ void wait_timeout_kernel(int* status, long long limit) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`: the wait must give up and record the timeout.
+  mbar_wait(&bar, 0, &abort_flag, threadIdx.x == 0 ? status : nullptr, limit);
+}
+
+}  // namespace
+
+thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
+                              const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
+                              void* out, float* lse, const thrift_cfg& c, int* status, float* dbg, int dbg_entry,
+                              cudaStream_t stream) {
+  AttnParams prm;
+  memset(&prm, 0, sizeof(prm));
+  prm.mask = mask;
+  if (mode != 2) {
+    prm.q_sf = q4->scales_mma;
+    prm.k_sf = k4->scales_mma;
+    prm.v_sf = v4->scales_mma;
+    prm.q_ts = q4->tensor_scale;
+    prm.k_ts = k4->tensor_scale;
+    prm.v_ts = v4->tensor_scale;
+  }
+  prm.out = reinterpret_cast<__half*>(out);
+  prm.lse = lse;
+  prm.status = status;
+  prm.dbg = dbg;
+  prm.dbg_entry = dbg_entry;
+  prm.B = c.B;
+  prm.Hq = c.Hq;
+  prm.Hkv = c.Hkv;
+  prm.N = c.N;
+  prm.bq = c.block_q;
+  prm.causal = c.causal;
+  prm.mode = mode;
+  prm.nqb = c.N / c.block_q;
+  prm.nkb = c.N / c.block_k;
+  prm.mask_words = (prm.nkb + 31) / 32;
+  prm.n_units = c.B * c.Hq * (c.N / kBQ);
+  prm.tau = c.softmax_scale > 0.0f ? c.softmax_scale : 1.0f / sqrtf((float)c.d);
+  prm.wait_limit = kWaitLimit;
+  if (c.d == 128 && c.block_k == 64) return launch_t<128, 64>(q, k, v, q4, k4, v4, prm, stream);
+  if (c.d == 128 && c.block_k == 128) return launch_t<128, 128>(q, k, v, q4, k4, v4, prm, stream);
+  if (c.d == 64 && c.block_k == 64) return launch_t<64, 64>(q, k, v, q4, k4, v4, prm, stream);
+  if (c.d == 64 && c.block_k == 128) return launch_t<64, 128>(q, k, v, q4, k4, v4, prm, stream);
+  return THRIFT_ERR_UNSUPPORTED;
+}
+
+thrift_status attn_launch(const void* q, const void* k, const void* v, const thrift_nvfp4* q4, const thrift_nvfp4* k4,
+                          const thrift_nvfp4* v4, const uint32_t* mask, int mode, void* out, float* lse,
+                          const thrift_cfg& c, int* status, cudaStream_t stream) {
+  return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, lse, c, status, nullptr, -1, stream);
+}
+
+thrift_status wait_timeout_launch(int* status, long long limit, cudaStream_t stream) {
+  wait_timeout_kernel<<<1, 32, 0, stream>>>(status, limit);
+  return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
+}
+
+}  // namespace thrift

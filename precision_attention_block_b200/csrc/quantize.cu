@@ -1,0 +1,188 @@
+// NVFP4 quantisation of FP16 tensors (ThriftAttention technical summary, "FP4-pad": the NVFP4
+// microscaling format -- E2M1 values, one E4M3 scale per 16 elements, one FP32 tensor scale).
+//
+// Two HBM-bound passes:
+//   1. amax: every thread max-reduces 16-byte vectors of |x|, warp shuffles, one atomicMax per
+//      block on the float bits (non-negative floats order like unsigned ints).
+//   2. encode: per 16-element group s_b = E4M3(amax16 / 6 / s_t), codes = E2M1(x / (s_b s_t)),
+//      with IEEE divisions (round to nearest) so that codes and scales are bit-identical to any
+//      other correctly rounded implementation of the same steps.
+//      Groups along d (Q, K): one thread per group, 32-byte loads, 8-byte code stores.
+//      Groups along tokens (V): a 64-token x d tile is staged in shared memory and transposed.
+#include <cuda_runtime.h>
+
+#include "sm100.cuh"
+#include "thrift_internal.h"
+
+namespace thrift {
+
+namespace {
+
+__global__ void __launch_bounds__(256) amax_kernel(const uint4* __restrict__ x, int64_t n_vec,
+                                                   unsigned int* __restrict__ amax_bits) {
+  __half2 m2 = __float2half2_rn(0.0f);
+  int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n_vec; i += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = __ldg(x + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const __half2* h = reinterpret_cast<const __half2*>(&v[u]);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) m2 = __hmax2(m2, __habs2(h[t]));
+    }
+  }
+  for (; i < n_vec; i += stride) {
+    uint4 v = __ldg(x + i);
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) m2 = __hmax2(m2, __habs2(h[t]));
+  }
+  float m = fmaxf(__low2float(m2), __high2float(m2));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0) atomicMax(amax_bits, __float_as_uint(m));
+  }
+}
+
+__device__ __forceinline__ float tensor_scale_from(unsigned int amax_bits) {
+  float amax = __uint_as_float(amax_bits);
+  return amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+}
+
+// Quantise one group of 16 values; returns the E4M3 scale code, writes 8 code bytes.
+__device__ __forceinline__ uint32_t quant16(const float (&x)[16], float s_t, uint2& packed) {
+  float amax16 = 0.0f;
+#pragma unroll
+  for (int t = 0; t < 16; ++t) amax16 = fmaxf(amax16, fabsf(x[t]));
+  float r = __fdiv_rn(amax16, 6.0f);
+  uint32_t sb = cvt_e4m3(__fdiv_rn(r, s_t));
+  float eff = __fmul_rn(e4m3_to_f32(sb), s_t);
+  uint32_t w[2] = {0u, 0u};
+  if (eff != 0.0f) {
+#pragma unroll
+    for (int t = 0; t < 16; t += 2) {
+      uint32_t b = cvt_e2m1x2(__fdiv_rn(x[t], eff), __fdiv_rn(x[t + 1], eff));
+      w[t >> 3] |= b << ((t & 7) * 4);
+    }
+  }
+  packed = make_uint2(w[0], w[1]);
+  return sb;
+}
+
+__device__ __forceinline__ int64_t sf_mma_offset(int64_t row, int64_t group, int64_t n_kblocks) {
+  int64_t rb = row >> 7, kb = group >> 2;
+  return (rb * n_kblocks + kb) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (group & 3);
+}
+
+// Groups along d: one thread per group of 16 consecutive elements of a row.
+__global__ void __launch_bounds__(256) encode_rows_kernel(const uint4* __restrict__ x, int64_t n_groups, int d,
+                                                          const unsigned int* __restrict__ amax_bits,
+                                                          uint2* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                          uint8_t* __restrict__ scales_mma,
+                                                          float* __restrict__ tensor_scale) {
+  float s_t = tensor_scale_from(*amax_bits);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
+  int gpr = d >> 4;  // groups per row
+  int64_t n_kblocks = d >> 6;
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n_groups;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    uint4 v0 = __ldg(x + 2 * g), v1 = __ldg(x + 2 * g + 1);
+    float f[16];
+    const __half2* h0 = reinterpret_cast<const __half2*>(&v0);
+    const __half2* h1 = reinterpret_cast<const __half2*>(&v1);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      float2 a = __half22float2(h0[t]), b = __half22float2(h1[t]);
+      f[2 * t] = a.x; f[2 * t + 1] = a.y; f[8 + 2 * t] = b.x; f[8 + 2 * t + 1] = b.y;
+    }
+    uint2 packed;
+    uint32_t sb = quant16(f, s_t, packed);
+    codes[g] = packed;
+    scales[g] = (uint8_t)sb;
+    int64_t row = g / gpr;
+    int64_t grp = g - row * gpr;
+    scales_mma[sf_mma_offset(row, grp, n_kblocks)] = (uint8_t)sb;
+  }
+}
+
+// Groups along tokens: one CTA per (outer index, 64-token tile); 256 threads.
+template <int D>
+__global__ void __launch_bounds__(256) encode_cols_kernel(const __half* __restrict__ x, int N,
+                                                          const unsigned int* __restrict__ amax_bits,
+                                                          uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                          uint8_t* __restrict__ scales_mma,
+                                                          float* __restrict__ tensor_scale) {
+  __shared__ __align__(16) __half tile[64 * D];
+  float s_t = tensor_scale_from(*amax_bits);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *tensor_scale = s_t;
+  int64_t o = blockIdx.y;
+  int t0 = blockIdx.x * 64;
+  const uint4* src = reinterpret_cast<const uint4*>(x + ((int64_t)o * N + t0) * D);
+  uint4* dst = reinterpret_cast<uint4*>(tile);
+  constexpr int VECS = 64 * D / 8;
+#pragma unroll
+  for (int v = threadIdx.x; v < VECS; v += 256) dst[v] = __ldg(src + v);
+  __syncthreads();
+  int64_t n_kblocks = N >> 6;
+  for (int p = threadIdx.x; p < 4 * D; p += 256) {
+    int c = p % D, g = p / D;
+    float f[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) f[t] = __half2float(tile[(g * 16 + t) * D + c]);
+    uint2 packed;
+    uint32_t sb = quant16(f, s_t, packed);
+    int64_t row = o * D + c;
+    *reinterpret_cast<uint2*>(codes + row * (N / 2) + (t0 + g * 16) / 2) = packed;
+    int64_t grp = (t0 >> 4) + g;
+    scales[row * (N / 16) + grp] = (uint8_t)sb;
+    scales_mma[sf_mma_offset(row, grp, n_kblocks)] = (uint8_t)sb;
+  }
+}
+
+}  // namespace
+
+size_t scales_mma_bytes(int64_t outer, int32_t N, int32_t d, int32_t group_axis) {
+  int64_t rows = group_axis == 0 ? outer * N : outer * d;
+  int64_t len = group_axis == 0 ? d : N;
+  int64_t nrb = (rows + 127) / 128;
+  return (size_t)(nrb * (len / 64) * 512);
+}
+
+thrift_status quantize_launch(const void* x, int64_t outer, int32_t N, int32_t d, const thrift_nvfp4* out,
+                              unsigned int* amax_slot, cudaStream_t stream) {
+  int64_t total = outer * (int64_t)N * d;
+  if (cudaMemsetAsync(amax_slot, 0, sizeof(unsigned int), stream) != cudaSuccess) return THRIFT_ERR_CUDA;
+  int sms = num_sms();
+  amax_kernel<<<sms * 8, 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), total / 8, amax_slot);
+  if (out->group_axis == 0) {
+    int64_t groups = total / 16;
+    int64_t blocks = (groups + 255) / 256;
+    if (blocks > (int64_t)sms * 32) blocks = (int64_t)sms * 32;
+    encode_rows_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+        reinterpret_cast<const uint4*>(x), groups, d, amax_slot, reinterpret_cast<uint2*>(out->codes),
+        out->scales, out->scales_mma, out->tensor_scale);
+  } else {
+    dim3 grid(N / 64, (unsigned)outer);
+    if (d == 128)
+      encode_cols_kernel<128><<<grid, 256, 0, stream>>>(reinterpret_cast<const __half*>(x), N, amax_slot,
+                                                         out->codes, out->scales, out->scales_mma,
+                                                         out->tensor_scale);
+    else
+      encode_cols_kernel<64><<<grid, 256, 0, stream>>>(reinterpret_cast<const __half*>(x), N, amax_slot,
+                                                        out->codes, out->scales, out->scales_mma,
+                                                        out->tensor_scale);
+  }
+  return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
+}
+
+}  // namespace thrift

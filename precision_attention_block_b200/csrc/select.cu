@@ -1,0 +1,235 @@
+// Block selection (ThriftAttention technical summary, "Heuristische Blokkenselectie"):
+// block means of Q and K, the score S^_ij = qbar_i . kbar_j of every valid (query block, key
+// block) pair, the k highest pairs per (batch, query head), and their per-row lists.
+//
+//   means   FP16 sums in float64 are exact (|partial sums| < 2^23 on a 2^-24 grid), divided by
+//           the block size (a power of two, exact).
+//   scores  float64 products and sums in the order c = 0 .. d-1 with no fused multiply-add, so
+//           every score is the correctly rounded result of one fixed evaluation order.
+//   top-k   one CTA per (batch, query head): a most-significant-digit-first radix select over
+//           order-preserving 64-bit keys finds the k-th largest score; keys above it are taken,
+//           ties at it are taken in index order (smaller i * nKb + j first) through a block scan.
+//   lists   one thread per query block walks its mask words in ascending order.
+#include <cuda_runtime.h>
+
+#include "sm100.cuh"
+#include "thrift_internal.h"
+
+namespace thrift {
+
+namespace {
+
+// Block sums: one CTA per (batch*head, block); thread c sums column c over the block's tokens.
+__global__ void block_mean_kernel(const __half* __restrict__ x, int N, int d, int bs, double* __restrict__ mean) {
+  int64_t bh = blockIdx.y;
+  int blk = blockIdx.x;
+  const __half* base = x + (bh * N + (int64_t)blk * bs) * d;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    double s = 0.0;
+    for (int t = 0; t < bs; ++t) s = __dadd_rn(s, (double)__half2float(base[(int64_t)t * d + c]));
+    mean[(bh * (N / bs) + blk) * d + c] = s / (double)bs;
+  }
+}
+
+constexpr int kTileQ = 16, kTileK = 16;
+
+// Scores for a 16 x 16 tile of (query block, key block) pairs of one (batch, query head).
+__global__ void __launch_bounds__(256) block_score_kernel(const double* __restrict__ qbar,
+                                                          const double* __restrict__ kbar, int Hq, int Hkv,
+                                                          int nqb, int nkb, int d, int bq, int bk, int causal,
+                                                          double* __restrict__ scores) {
+  extern __shared__ double sm[];
+  double* qs = sm;                          // [kTileQ][d+1]
+  double* ks = sm + kTileQ * (d + 1);       // [kTileK][d+1]
+  int bh = blockIdx.z;
+  int b = bh / Hq, h = bh % Hq, hk = h / (Hq / Hkv);
+  int i0 = blockIdx.y * kTileQ, j0 = blockIdx.x * kTileK;
+  const double* qb = qbar + ((int64_t)bh * nqb) * d;
+  const double* kb = kbar + ((int64_t)(b * Hkv + hk) * nkb) * d;
+  for (int e = threadIdx.x; e < kTileQ * d; e += blockDim.x) {
+    int r = e / d, c = e % d;
+    qs[r * (d + 1) + c] = (i0 + r < nqb) ? qb[(int64_t)(i0 + r) * d + c] : 0.0;
+  }
+  for (int e = threadIdx.x; e < kTileK * d; e += blockDim.x) {
+    int r = e / d, c = e % d;
+    ks[r * (d + 1) + c] = (j0 + r < nkb) ? kb[(int64_t)(j0 + r) * d + c] : 0.0;
+  }
+  __syncthreads();
+  int ii = threadIdx.x / kTileK, jj = threadIdx.x % kTileK;
+  int i = i0 + ii, j = j0 + jj;
+  if (i >= nqb || j >= nkb) return;
+  double out;
+  if (causal && (int64_t)j * bk > (int64_t)(i + 1) * bq - 1) {
+    out = -__longlong_as_double(0x7ff0000000000000LL);
+  } else {
+    double s = 0.0;
+    const double* qr = qs + ii * (d + 1);
+    const double* kr = ks + jj * (d + 1);
+    for (int c = 0; c < d; ++c) s = __dadd_rn(s, __dmul_rn(qr[c], kr[c]));
+    out = s;
+  }
+  scores[((int64_t)bh * nqb + i) * nkb + j] = out;
+}
+
+// Order-preserving key of a score: larger score -> larger key; invalid (-inf) -> 0.
+__device__ __forceinline__ uint64_t score_key(double s) {
+  if (s == -__longlong_as_double(0x7ff0000000000000LL)) return 0ull;
+  uint64_t u = (uint64_t)__double_as_longlong(s);
+  return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
+}
+
+constexpr int kSelThreads = 1024;
+
+__device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int& total) {
+  int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < (kSelThreads / 32) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sums[lane] = w;  // inclusive prefix of warp totals
+  }
+  __syncthreads();
+  int before = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
+  total = warp_sums[kSelThreads / 32 - 1];
+  __syncthreads();
+  return before;
+}
+
+// One CTA per (batch, query head).
+__global__ void __launch_bounds__(kSelThreads) topk_kernel(const double* __restrict__ scores, int64_t n,
+                                                           int nkb, int topk_abs, int topk_bp, int mask_words,
+                                                           uint32_t* __restrict__ mask) {
+  __shared__ unsigned int hist[256];
+  __shared__ int warp_sums[32];
+  __shared__ unsigned long long s_prefix;
+  __shared__ long long s_need;
+  __shared__ unsigned long long s_nvalid;
+  const double* sc = scores + (int64_t)blockIdx.x * n;
+  int nqb = (int)(n / nkb);
+  uint32_t* mk = mask + (int64_t)blockIdx.x * nqb * mask_words;
+
+  // count valid pairs
+  if (threadIdx.x == 0) s_nvalid = 0;
+  __syncthreads();
+  unsigned long long cnt = 0;
+  for (int64_t t = threadIdx.x; t < n; t += kSelThreads) cnt += score_key(sc[t]) != 0ull;
+  atomicAdd(&s_nvalid, cnt);
+  __syncthreads();
+  long long nvalid = (long long)s_nvalid;
+  long long k = topk_abs >= 0 ? (long long)topk_abs : ((long long)topk_bp * nvalid + 9999) / 10000;
+  if (k > nvalid) k = nvalid;
+  if (k <= 0) return;  // mask already zeroed by the caller
+
+  // radix select: prefix of the k-th largest key, 8 bits at a time from the top
+  unsigned long long prefix = 0ull;
+  long long need = k;  // rank (1-based) of the wanted key among keys matching the prefix
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int b = threadIdx.x; b < 256; b += kSelThreads) hist[b] = 0;
+    __syncthreads();
+    unsigned long long hi_mask = shift == 56 ? 0ull : (~0ull << (shift + 8));
+    for (int64_t t = threadIdx.x; t < n; t += kSelThreads) {
+      uint64_t key = score_key(sc[t]);
+      if (key != 0ull && (key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      long long acc = 0;
+      int b = 255;
+      for (; b >= 0; --b) {
+        if (acc + (long long)hist[b] >= need) break;
+        acc += hist[b];
+      }
+      s_prefix = prefix | ((unsigned long long)b << shift);
+      s_need = need - acc;
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    need = s_need;
+    __syncthreads();
+  }
+  // prefix is now the k-th largest key; take every key above it and the first `need` ties.
+  long long taken_ties = 0;
+  for (int64_t base = 0; base < n; base += kSelThreads) {
+    int64_t t = base + threadIdx.x;
+    uint64_t key = t < n ? score_key(sc[t]) : 0ull;
+    int tie = (key != 0ull && key == prefix) ? 1 : 0;
+    int total;
+    int before = block_excl_scan(tie, warp_sums, total);
+    bool take = (key > prefix) || (tie && (taken_ties + before) < need);
+    if (take) {
+      int i = (int)(t / nkb), j = (int)(t % nkb);
+      atomicOr(&mk[(int64_t)i * mask_words + (j >> 5)], 1u << (j & 31));
+    }
+    taken_ties += total;
+  }
+}
+
+__global__ void lists_kernel(const uint32_t* __restrict__ mask, int64_t rows, int nkb, int mask_words,
+                             int32_t* __restrict__ counts, int16_t* __restrict__ lists) {
+  int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= rows) return;
+  const uint32_t* mw = mask + r * mask_words;
+  int16_t* out = lists + r * nkb;
+  int c = 0;
+  for (int w = 0; w < mask_words; ++w) {
+    uint32_t bits = mw[w];
+    while (bits) {
+      int b = __ffs(bits) - 1;
+      bits &= bits - 1;
+      out[c++] = (int16_t)(w * 32 + b);
+    }
+  }
+  counts[r] = c;
+  for (int t = c; t < nkb; ++t) out[t] = -1;
+}
+
+}  // namespace
+
+SelectLayout select_layout(const thrift_cfg& c) {
+  SelectLayout L;
+  int64_t nqb = c.N / c.block_q, nkb = c.N / c.block_k;
+  L.qbar_off = 0;
+  L.kbar_off = align256(L.qbar_off + (size_t)c.B * c.Hq * nqb * c.d * sizeof(double));
+  L.scores_off = align256(L.kbar_off + (size_t)c.B * c.Hkv * nkb * c.d * sizeof(double));
+  L.bytes = align256(L.scores_off + (size_t)c.B * c.Hq * nqb * nkb * sizeof(double));
+  return L;
+}
+
+thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, uint32_t* mask, int32_t* counts,
+                            int16_t* lists, double* scores_out, uint8_t* scratch, cudaStream_t stream) {
+  SelectLayout L = select_layout(c);
+  int nqb = c.N / c.block_q, nkb = c.N / c.block_k;
+  int mask_words = (nkb + 31) / 32;
+  double* qbar = reinterpret_cast<double*>(scratch + L.qbar_off);
+  double* kbar = reinterpret_cast<double*>(scratch + L.kbar_off);
+  double* scores = scores_out ? scores_out : reinterpret_cast<double*>(scratch + L.scores_off);
+  int tpb = c.d >= 128 ? 128 : c.d;
+  block_mean_kernel<<<dim3(nqb, c.B * c.Hq), tpb, 0, stream>>>(reinterpret_cast<const __half*>(q), c.N, c.d,
+                                                               c.block_q, qbar);
+  block_mean_kernel<<<dim3(nkb, c.B * c.Hkv), tpb, 0, stream>>>(reinterpret_cast<const __half*>(k), c.N, c.d,
+                                                                c.block_k, kbar);
+  size_t smem = (size_t)(kTileQ + kTileK) * (c.d + 1) * sizeof(double);
+  dim3 g((nkb + kTileK - 1) / kTileK, (nqb + kTileQ - 1) / kTileQ, c.B * c.Hq);
+  block_score_kernel<<<g, kTileQ * kTileK, smem, stream>>>(qbar, kbar, c.Hq, c.Hkv, nqb, nkb, c.d, c.block_q,
+                                                           c.block_k, c.causal, scores);
+  size_t mask_bytes = (size_t)c.B * c.Hq * nqb * mask_words * sizeof(uint32_t);
+  if (cudaMemsetAsync(mask, 0, mask_bytes, stream) != cudaSuccess) return THRIFT_ERR_CUDA;
+  topk_kernel<<<c.B * c.Hq, kSelThreads, 0, stream>>>(scores, (int64_t)nqb * nkb, nkb, c.topk_abs, c.topk_bp,
+                                                      mask_words, mask);
+  int64_t rows = (int64_t)c.B * c.Hq * nqb;
+  lists_kernel<<<(unsigned)((rows + 127) / 128), 128, 0, stream>>>(mask, rows, nkb, mask_words, counts, lists);
+  return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
+}
+
+}  // namespace thrift

@@ -1,0 +1,41 @@
+// Host-side declarations shared by the library's translation units (not part of the C ABI).
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/thrift.h"
+
+namespace thrift {
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int num_sms();
+
+// Workspace: [0, 256) status word and small scalars; then per-call scratch.
+constexpr size_t kWsHeader = 256;
+constexpr size_t kWsStatusOff = 0;    // int32 device status
+constexpr size_t kWsAmaxOff = 16;     // uint32 amax bits for the quantiser
+
+struct SelectLayout {
+  size_t qbar_off, kbar_off, scores_off, bytes;
+};
+SelectLayout select_layout(const thrift_cfg& c);
+
+size_t scales_mma_bytes(int64_t outer, int32_t N, int32_t d, int32_t group_axis);
+
+thrift_status quantize_launch(const void* x, int64_t outer, int32_t N, int32_t d, const thrift_nvfp4* out,
+                              unsigned int* amax_slot, cudaStream_t stream);
+
+thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, uint32_t* mask, int32_t* counts,
+                            int16_t* lists, double* scores_out, uint8_t* scratch, cudaStream_t stream);
+
+// mode: 0 = FP16 pairs from the mask, 1 = every pair NVFP4, 2 = every pair FP16.
+thrift_status attn_launch(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
+                          const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
+                          void* out, float* lse, const thrift_cfg& c, int* status, cudaStream_t stream);
+
+thrift_status wait_timeout_launch(int* status, long long limit, cudaStream_t stream);
+
+}  // namespace thrift

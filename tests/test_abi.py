@@ -1,0 +1,97 @@
+"""The C ABI without a GPU: the library loads, exports every function the headers declare, sizes
+its buffers, and rejects bad arguments on the host with a status code before touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from precision_attention_block_b200 import build
+    build.build()
+    from precision_attention_block_b200 import _lib
+    return _lib.load()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"^\s*(?:const\s+char\s*\*|size_t|thrift_status)\s+(thrift_\w+)\s*\(", src, re.M))
+    return names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert {"thrift_quantize_nvfp4", "thrift_block_select", "thrift_attn_fwd"} <= names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_binding_covers_every_declared_symbol():
+    from precision_attention_block_b200 import _lib
+    assert declared_functions() <= set(_lib.SIGNATURES)
+
+
+def cfg(**kw):
+    from precision_attention_block_b200 import Config
+    base = dict(B=1, Hq=32, Hkv=8, N=32768, d=128, causal=True, block_q=128, block_k=64, topk_bp=500)
+    base.update(kw)
+    return Config(**base).c()
+
+
+def test_workspace_sizes(L):
+    c = cfg()
+    n = L.thrift_workspace_bytes(ctypes.byref(c))
+    # block means (float64) + dense score matrix (float64) + header
+    assert n >= 256 + 32 * 256 * 128 * 8 + 8 * 512 * 128 * 8 + 32 * 256 * 512 * 8
+    auto = L.thrift_auto_workspace_bytes(ctypes.byref(c))
+    assert auto > n + (32 + 16) * 32768 * 128 // 2
+    assert L.thrift_nvfp4_scales_mma_bytes(32, 32768, 128, 0) == 32 * 32768 * 128 // 16
+    assert L.thrift_nvfp4_scales_mma_bytes(8, 32768, 128, 1) == 8 * 128 * 32768 // 16
+    assert L.thrift_nvfp4_scales_mma_bytes(3, 256, 64, 1) == 2 * (256 // 64) * 512  # rows padded to 128
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), 2), (dict(Hkv=5), 1), (dict(block_k=32), 2), (dict(N=1000), 2), (dict(topk_bp=20000), 1),
+    (dict(causal=2), 1), (dict(topk_abs=-2), 1), (dict(block_q=256), 2)])
+def test_bad_config_rejected_on_host(L, kw, status):
+    c = cfg(**kw)
+    assert L.thrift_workspace_bytes(ctypes.byref(c)) == 0
+    from precision_attention_block_b200 import _lib
+    out = ctypes.c_void_p(0x1000)
+    rc = L.thrift_attn_fwd(out, out, out, None, None, None, out, out, out, out, None, ctypes.byref(c),
+                           ctypes.c_void_p(0x100000), 1 << 20, None)
+    assert rc == status
+    rc = L.thrift_block_select(out, out, ctypes.byref(c), out, out, out, None, ctypes.c_void_p(0x100000),
+                               1 << 30, None)
+    assert rc == status
+
+
+def test_null_and_workspace_errors(L):
+    from precision_attention_block_b200 import _lib
+    c = cfg()
+    p = ctypes.c_void_p(0x1000)
+    assert L.thrift_attn_fwd_auto(None, p, p, p, None, ctypes.byref(c), p, 1 << 40, None) == 1
+    assert L.thrift_attn_fwd_auto(p, p, p, p, None, ctypes.byref(c), ctypes.c_void_p(0x1001), 1 << 40, None) == 5
+    assert L.thrift_attn_fwd_auto(p, p, p, p, None, ctypes.byref(c), ctypes.c_void_p(0x1000), 16, None) == 5
+    assert L.thrift_quantize_nvfp4(None, 1, 128, 128, None, p, 256, None) == 1
+    nv = _lib.CNVFP4(0x1000, 0x1000, 0x1000, 0x1000, 0)
+    assert L.thrift_quantize_nvfp4(p, 1, 128, 96, ctypes.byref(nv), p, 256, None) == 2
+    assert L.thrift_quantize_nvfp4(p, 1, 100, 128, ctypes.byref(nv), p, 256, None) == 2
+    assert L.thrift_quantize_nvfp4(p, 1, 128, 128, ctypes.byref(nv), None, 256, None) == 5
+    assert L.thrift_reset_device_status(None, None) == 5
+    assert L.thrift_get_device_status(p, None, None) == 1
+    assert L.thrift_debug_wait_timeout(p, 0, None) == 1
+    # uniform NVFP4 needs the NVFP4 tensors; all-FP16 needs the FP16 ones; mixed needs the mask
+    assert L.thrift_attn_fwd(p, p, p, None, None, None, p, p, p, p, None, ctypes.byref(cfg(topk_bp=0)),
+                             p, 256, None) == 1
+    assert L.thrift_attn_fwd(None, None, None, ctypes.byref(nv), ctypes.byref(nv), ctypes.byref(nv), p, p, p, p,
+                             None, ctypes.byref(cfg(topk_bp=10000)), p, 256, None) == 1
+    assert L.thrift_status_str(4) == b"device wait timed out"

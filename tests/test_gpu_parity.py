@@ -1,0 +1,205 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on the same seeded inputs.
+
+Bar: NVFP4 codes and scales bit-exact; block scores and the selected set exact (ties go to the
+smaller index on both sides, and both evaluate S^ with the same float64 operation order; a pair
+within 1e-6 relative of the k-th score may differ); attention output within rel-L2 <= 1e-3 and
+max-abs <= 1e-2 of the oracle, LSE within 1e-3.  Full tensors for the small workloads, a seeded
+stratified sample of (batch, head, query block) units for the long ones.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 1e-3
+MAX_ABS = 1e-2
+LSE_ABS = 1e-3
+TIE_REL = 1e-6
+
+_cache = {}
+
+
+@pytest.fixture(scope="module")
+def pab(cuda_device):
+    from precision_attention_block_b200 import build
+    build.build()
+    import precision_attention_block_b200 as pab
+    pab.load()
+    return pab
+
+
+def inputs(name):
+    if name not in _cache:
+        w = workloads.WORKLOADS[name]
+        q, k, v = workloads.make_qkv(w)
+        _cache[name] = dict(w=w, q=q, k=k, v=v)
+    return _cache[name]
+
+
+def oracle_quant(name):
+    d = inputs(name)
+    if "q4" not in d:
+        d["q4"], d["k4"], d["v4"] = oracle.quantize_all(d["q"], d["k"], d["v"])
+        d["scores"] = oracle.block_scores(d["q"], d["k"], d["w"])
+    return d
+
+
+def dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def gpu_qkv(name):
+    d = inputs(name)
+    if "gq" not in d:
+        d["gq"], d["gk"], d["gv"] = dev(d["q"]), dev(d["k"]), dev(d["v"])
+    return d["gq"], d["gk"], d["gv"]
+
+
+def sf_mma_index(rows, len_):
+    """Index map canonical scale (row, group) -> byte offset in the MMA scale layout."""
+    r = np.arange(rows)[:, None]
+    g = np.arange(len_ // 16)[None, :]
+    nkb = len_ // 64
+    return ((r >> 7) * nkb + (g >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (g & 3)
+
+
+@pytest.mark.parametrize("name", ["tiny", "n4k", "diffusion", "prefill32k"])
+def test_quantize_bit_exact(pab, name):
+    d = oracle_quant(name)
+    gq, gk, gv = gpu_qkv(name)
+    g4 = pab.quantize_qkv(gq, gk, gv)
+    torch.cuda.synchronize()
+    for o, g in zip((d["q4"], d["k4"], d["v4"]), g4):
+        assert g.tensor_scale.item() == float(o.tensor_scale)
+        codes = g.codes.cpu().numpy().reshape(o.codes.shape)
+        scales = g.scales.cpu().numpy().reshape(o.scales.shape)
+        assert np.array_equal(scales, o.scales), "E4M3 scales differ"
+        assert np.array_equal(codes, o.codes), "E2M1 codes differ"
+        rows = int(np.prod(o.scales.shape[:-1]))
+        len_ = o.scales.shape[-1] * 16
+        mma = g.scales_mma.cpu().numpy()
+        idx = sf_mma_index(rows, len_)
+        assert np.array_equal(mma[idx], o.scales.reshape(rows, -1))
+
+
+def check_selection(d, w, sel_g, scores_g):
+    scores_o = d["scores"] if w.topk_bp == d["w"].topk_bp and w.topk_abs == d["w"].topk_abs else None
+    s_o = oracle.block_scores(d["q"], d["k"], w) if scores_o is None else scores_o
+    sel_o, kth, kc = oracle.select(s_o, w)
+    s_g = scores_g.cpu().numpy()
+    fin = np.isfinite(s_o)
+    assert np.array_equal(np.isfinite(s_g), fin)
+    assert np.array_equal(s_g[fin], s_o[fin]), "block scores differ"
+    mask = sel_g.mask.cpu().numpy().view(np.uint32)
+    nkb = w.n_kb
+    bits = ((mask[..., :, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(*mask.shape[:-1], -1)[..., :nkb]
+    diff = bits.astype(bool) != sel_o.astype(bool)
+    if diff.any():
+        # only pairs tied with the k-th score (within 1e-6 relative) may differ
+        band = np.abs(s_o - kth[..., None, None]) <= TIE_REL * np.abs(kth[..., None, None])
+        assert not (diff & ~band).any(), "selected sets differ outside the tie band"
+    counts = sel_g.counts.cpu().numpy()
+    assert np.array_equal(counts, bits.sum(-1))
+    lists = sel_g.lists.cpu().numpy()
+    for idx in [(0, 0, 0), (0, w.Hq - 1, w.n_qb - 1), (w.B - 1, w.Hq // 2, w.n_qb // 2)]:
+        js = np.nonzero(bits[idx])[0]
+        assert np.array_equal(lists[idx][:len(js)], js)
+        assert np.all(lists[idx][len(js):] == -1)
+    return bits
+
+
+@pytest.mark.parametrize("name,bp", [("tiny", None), ("n4k", None), ("prefill32k", None),
+                                     ("diffusion", 100), ("diffusion", 2000)])
+def test_select_exact(pab, name, bp):
+    d = oracle_quant(name)
+    w = d["w"] if bp is None else d["w"].with_budget(bp)
+    gq, gk, _ = gpu_qkv(name)
+    cfg = pab.Config.from_workload(w)
+    sel = pab.block_select(gq, gk, cfg, want_scores=True)
+    torch.cuda.synchronize()
+    check_selection(d, w, sel, sel.scores)
+
+
+def compare_attention(out_g, lse_g, out_o, lse_o, w, units):
+    og = out_g.cpu().numpy().astype(np.float64)
+    lg = lse_g.cpu().numpy().astype(np.float64)
+    oo = out_o.astype(np.float64)
+    lo = lse_o.astype(np.float64)
+    rows_g, rows_o, lse_rg, lse_ro = [], [], [], []
+    for (b, h, i) in units:
+        sl = slice(i * w.block_q, (i + 1) * w.block_q)
+        rows_g.append(og[b, h, sl])
+        rows_o.append(oo[b, h, sl])
+        lse_rg.append(lg[b, h, sl])
+        lse_ro.append(lo[b, h, sl])
+    a, e = np.concatenate(rows_g), np.concatenate(rows_o)
+    rel = np.linalg.norm(a - e) / np.linalg.norm(e)
+    mx = np.abs(a - e).max()
+    lmx = np.abs(np.concatenate(lse_rg) - np.concatenate(lse_ro)).max()
+    assert np.isfinite(a).all()
+    assert rel <= REL_L2 and mx <= MAX_ABS and lmx <= LSE_ABS, (rel, mx, lmx)
+    return rel, mx, lmx
+
+
+def run_pair(pab, name, bp=None, n_units=None, auto=False):
+    d = oracle_quant(name)
+    w = d["w"] if bp is None else d["w"].with_budget(bp)
+    gq, gk, gv = gpu_qkv(name)
+    cfg = pab.Config.from_workload(w)
+    if auto:
+        out_g, lse_g = pab.attn_fwd_auto(gq, gk, gv, cfg)
+    else:
+        q4, k4, v4 = pab.quantize_qkv(gq, gk, gv)
+        sel = pab.block_select(gq, gk, cfg)
+        out_g, lse_g = pab.attn_fwd(gq, gk, gv, q4, k4, v4, sel, cfg)
+    torch.cuda.synchronize()
+    scores = d["scores"] if bp is None else oracle.block_scores(d["q"], d["k"], w)
+    sel_o, _, _ = oracle.select(scores, w)
+    if n_units is None:
+        units = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.n_qb)]
+    else:
+        units = workloads.sample_units(w, n_units)
+    out_o, lse_o, _ = oracle.attn(d["q"], d["k"], d["v"], d["q4"], d["k4"], d["v4"], sel_o, w, units=units)
+    return compare_attention(out_g, lse_g, out_o, lse_o, w, units)
+
+
+@pytest.mark.parametrize("bp", [None, 0, 10000])
+def test_attn_tiny(pab, bp):
+    run_pair(pab, "tiny", bp)
+
+
+@pytest.mark.parametrize("bp", [None, 0, 10000])
+def test_attn_n4k(pab, bp):
+    run_pair(pab, "n4k", bp)
+
+
+def test_attn_auto_equals_steps(pab):
+    run_pair(pab, "n4k", None, auto=True)
+
+
+@pytest.mark.parametrize("bp", workloads.DIFFUSION_BUDGETS_BP)
+def test_attn_diffusion_sampled(pab, bp):
+    run_pair(pab, "diffusion", bp, n_units=12)
+
+
+def test_attn_prefill32k_sampled(pab):
+    run_pair(pab, "prefill32k", None, n_units=24)
+
+
+@pytest.mark.slow
+def test_attn_long131k_sampled(pab):
+    run_pair(pab, "long131k", None, n_units=10)
+
+
+def test_device_wait_timeout_is_reported(pab):
+    ws = pab.Workspace(256, torch.device("cuda"))
+    assert pab.device_status(ws) == 0
+    pab.load().thrift_debug_wait_timeout(ws.ptr, 200000, pab._stream())
+    assert pab.device_status(ws) == 4  # THRIFT_ERR_TIMEOUT
+    pab.reset_device_status(ws)
+    assert pab.device_status(ws) == 0
