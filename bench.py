@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark of the selective mixed-precision (NVFP4 + FP16) attention forward on B200.
+
+Metric: attention-forward effective TFLOPS (4 B Hq N^2 d, halved when causal) of one whole step
+-- NVFP4 quantisation of Q, K, V, block selection, attention -- on the 32K causal LLM-prefill
+workload (B=1, 32 query / 8 KV heads, d=128, 128x64 blocks, k = 5 % of the valid pairs), plus
+the attention kernel's fraction of the blended NVFP4/FP16 tensor-core roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One process per GPU (torchrun for N > 1); each rank runs its own copy of the workload (weak
+scaling, no collective on the data path); timing is CUDA events on the launching stream, max over
+ranks.  Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "attn fwd effective TFLOPS & % of NVFP4/FP16 tensor roofline, N=32K causal k=5%"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_traffic.json")
+ATTN_SRC = os.path.join(ROOT, "precision_attention_block_b200", "csrc", "attn.cu")
+NVFP4_PER_FP16 = 4.0  # nominal dense NVFP4 : FP16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill32k", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--budget-bp", type=int, default=None, help="override the FP16 budget (basis points)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-units", type=int, default=8)
+    return ap.parse_args()
+
+
+def effective_flops(w) -> float:
+    f = 4.0 * w.B * w.Hq * w.N * w.N * w.d
+    return f / 2 if w.causal else f
+
+
+def unit_effective_flops(w, i) -> float:
+    """Effective FLOPs of one (b, h, query block i) unit under the same convention."""
+    if not w.causal:
+        return 4.0 * w.block_q * w.N * w.d
+    keys = sum(min(w.N, r + 1) for r in range(i * w.block_q, (i + 1) * w.block_q))
+    return 4.0 * keys * w.d
+
+
+def valid_pairs_per_head(w) -> int:
+    if not w.causal:
+        return w.n_qb * w.n_kb
+    return sum(((i + 1) * w.block_q - 1) // w.block_k + 1 for i in range(w.n_qb))
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), \
+            float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, 1400.0, 6650.0, "fallback"
+
+
+def attn_src_hash() -> str:
+    with open(ATTN_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def stored_traffic(workload: str):
+    """DRAM bytes per attention launch from a committed ncu capture, if the kernel source is
+    unchanged since it was taken; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        e = t.get(workload)
+        if e and e.get("attn_src_sha256_16") == attn_src_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+             0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+             0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            props = torch.cuda.get_device_properties(device_index)
+            uuid = str(getattr(props, "uuid", ""))
+            if uuid:
+                u = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+                try:
+                    self.h = pynvml.nvmlDeviceGetHandleByUUID(u)
+                except Exception:
+                    self.h = None
+            if self.h is None:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                idx = int(vis.split(",")[device_index]) if vis and vis.split(",")[0].isdigit() else device_index
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.h = None
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                try:
+                    r = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    r = n.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.reasons |= int(r) & ~0x1
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.h is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": [v for k, v in self.NAMES.items() if self.reasons & k], "samples": len(self.samples)}
+
+
+def cpu_baseline(w, q, k, v, n_units: int):
+    """The oracle, as it stands, on the host cores: full NVFP4 quantisation and selection of the
+    workload, then attention on a stratified sample of (b, h, query block) units; the value is the
+    sample's effective FLOPs over its time plus the sample's share of quantise + select."""
+    import oracle
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    q4, k4, v4 = oracle.quantize_all(q, k, v)
+    scores = oracle.block_scores(q, k, w)
+    sel, _, _ = oracle.select(scores, w)
+    t_prep = time.perf_counter() - t0
+    units = workloads.sample_units(w, n_units, seed_offset=3)
+    t0 = time.perf_counter()
+    oracle.attn(q, k, v, q4, k4, v4, sel, w, units=units, threads=threads)
+    t_attn = time.perf_counter() - t0
+    f_sample = sum(unit_effective_flops(w, i) for (_, _, i) in units)
+    share = f_sample / effective_flops(w)
+    t = t_attn + t_prep * share
+    return {"value": f_sample / t / 1e12, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+            "sample": f"{len(units)} stratified (b, head, 128-row query block) units of {w.name}; attention "
+                      f"{t_attn:.1f} s on {threads} threads + their {share:.2e} share of the full "
+                      f"quantise/select ({t_prep:.1f} s)"}
+
+
+def run_reference(args, rank):
+    """--impl reference: the oracle on the host cores, one bounded sample per step."""
+    if rank != 0:
+        return
+    import oracle
+    w = workloads.WORKLOADS[args.workload]
+    if args.budget_bp is not None:
+        w = w.with_budget(args.budget_bp)
+    q, k, v = workloads.make_qkv(w)
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    q4, k4, v4 = oracle.quantize_all(q, k, v)
+    scores = oracle.block_scores(q, k, w)
+    sel, _, _ = oracle.select(scores, w)
+    t_prep = time.perf_counter() - t0
+    per_step = max(1, min(threads, 8))
+    pool = workloads.sample_units(w, per_step * 8, seed_offset=5)
+    flops, secs = 0.0, 0.0
+    for s in range(args.warmup + args.steps):
+        units = [pool[(s * per_step + u) % len(pool)] for u in range(per_step)]
+        t0 = time.perf_counter()
+        oracle.attn(q, k, v, q4, k4, v4, sel, w, units=units, threads=threads)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            f = sum(unit_effective_flops(w, i) for (_, _, i) in units)
+            flops += f
+            secs += dt + t_prep * f / effective_flops(w)
+    value = flops / secs / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                       "causal": w.causal, "block_q": w.block_q, "block_k": w.block_k, "topk_bp": w.topk_bp},
+            "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                             "sample": f"{per_step} (b, head, query block) units per step, cycled from a "
+                                       f"stratified sample, plus their share of the full quantise/select"},
+            "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        if args.impl == "ours":
+            torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl" if args.impl == "ours" else "gloo",
+                                timeout=datetime.timedelta(seconds=300))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        if dist:
+            dist.destroy_process_group()
+        return
+
+    import precision_attention_block_b200 as pab
+    from precision_attention_block_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    if dist:
+        dist.barrier()
+    pab.load()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+
+    w = workloads.WORKLOADS[args.workload]
+    if args.budget_bp is not None:
+        w = w.with_budget(args.budget_bp)
+    cfg = pab.Config.from_workload(w)
+    q, k, v = workloads.make_qkv(w)
+    gq, gk, gv = (torch.from_numpy(x).to(device) for x in (q, k, v))
+    q4 = pab.NVFP4Tensor.empty(w.B * w.Hq, w.N, w.d, 0, device)
+    k4 = pab.NVFP4Tensor.empty(w.B * w.Hkv, w.N, w.d, 0, device)
+    v4 = pab.NVFP4Tensor.empty(w.B * w.Hkv, w.N, w.d, 1, device)
+    ws = pab.Workspace.for_config(cfg, device)
+    sel = pab.block_select(gq, gk, cfg, ws=ws)
+    out = torch.empty_like(gq)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        pab.quantize_nvfp4(gq, 0, out=q4, ws=ws)
+        pab.quantize_nvfp4(gk, 0, out=k4, ws=ws)
+        pab.quantize_nvfp4(gv, 1, out=v4, ws=ws)
+        if evs:
+            evs[0].record(stream)
+        pab.block_select(gq, gk, cfg, ws=ws, out=sel)
+        if evs:
+            evs[1].record(stream)
+        pab.attn_fwd(gq, gk, gv, q4, k4, v4, sel, cfg, out=out, lse=lse, ws=ws)
+        if evs:
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    launches_per_step = 3 * 2 + 5 + 1  # amax + encode per tensor; means x2, scores, top-k, lists; attention
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    ev_start = torch.cuda.Event(enable_timing=True)
+    ev_end = torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        ev_start.record(stream)
+        prev = ev_start
+        step_starts = []
+        for s in range(args.steps):
+            step_starts.append(prev)
+            step(evs[s])
+            prev = evs[s][2]
+        ev_end.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    total_ms = ev_start.elapsed_time(ev_end)
+    attn_ms = [evs[s][1].elapsed_time(evs[s][2]) for s in range(args.steps)]
+    sel_ms = [evs[s][0].elapsed_time(evs[s][1]) for s in range(args.steps)]
+    quant_ms = [step_starts[s].elapsed_time(evs[s][0]) for s in range(args.steps)]
+    t = torch.tensor([total_ms, statistics.mean(attn_ms)], dtype=torch.float64, device=device)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, attn_mean_ms = float(t[0]), float(t[1])
+
+    # status word: any device-side timeout invalidates the run
+    status = pab.device_status(ws)
+
+    # roofline of the attention kernel: algorithmic FLOPs of the valid block pairs by precision
+    counts = sel.counts.sum().item()
+    mode_fp16_all = cfg.topk_abs < 0 and cfg.topk_bp == 10000
+    mode_fp4_all = cfg.topk_abs == 0 or (cfg.topk_abs < 0 and cfg.topk_bp == 0)
+    valid_total = valid_pairs_per_head(w) * w.B * w.Hq
+    k_total = valid_total if mode_fp16_all else (0 if mode_fp4_all else counts)
+    per_pair = 4.0 * w.block_q * w.block_k * w.d
+    F16, F4 = k_total * per_pair, (valid_total - k_total) * per_pair
+    bf16_burst, bf16_sustained, hbm_gbs, peak_src = peaks()
+    p16, p4 = bf16_burst * 1e12, bf16_burst * NVFP4_PER_FP16 * 1e12
+    t_roof = F16 / p16 + F4 / p4
+    achieved = (F16 + F4) / (attn_mean_ms * 1e-3) / 1e12
+    peak_blend = (F16 + F4) / t_roof / 1e12
+    traffic = stored_traffic(w.name) if args.budget_bp is None else None
+
+    eff = effective_flops(w)
+    qkv_mb = (q.nbytes + k.nbytes + v.nbytes) / 1e6
+    value = world * eff * args.steps / (total_ms * 1e-3) / 1e12
+    line = {"metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4+fp16 (fp32 accumulate)",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                       "causal": w.causal, "block_q": w.block_q, "block_k": w.block_k, "topk_bp": w.topk_bp,
+                       "parallelism": f"replica x{world} (each rank its own batch)",
+                       "l2": (f"inputs larger than L2 (Q, K, V {qkv_mb:.0f} MB FP16)" if qkv_mb > 126
+                              else f"inputs smaller than L2 ({qkv_mb:.0f} MB); no flush")},
+            "breakdown_ms": {"quantize": statistics.mean(quant_ms), "select": statistics.mean(sel_ms),
+                             "attention": attn_mean_ms},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_blend, "unit": "TFLOP/s",
+                         "frac": achieved / peak_blend, "traffic": traffic,
+                         "peak_note": f"blend of {peak_src} bf16 burst {bf16_burst:.1f} TF/s (FP16) and "
+                                      f"x{NVFP4_PER_FP16:.0f} for NVFP4; F16={F16:.3e} F4={F4:.3e}"},
+            "gpu_launches": launches_per_step * args.steps,
+            "device_status": status}
+
+    if not args.no_e2e:
+        line["e2e"] = e2e_measure(pab, torch, w, cfg, q, k, v, device, args, world, dist)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, q, k, v, args.cpu_units)
+    line["clocks"] = sampler.summary()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+def e2e_measure(pab, torch, w, cfg, q, k, v, device, args, world, dist):
+    """The same metric through thrift_attn_fwd_auto with host buffers: every step copies Q, K, V
+    from pinned host memory, runs quantise + select + attend, and copies O and lse back."""
+    hq, hk, hv = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
+    gq, gk, gv = (torch.empty(x.shape, dtype=torch.float16, device=device) for x in (q, k, v))
+    out = torch.empty_like(gq)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=device)
+    ho = torch.empty(out.shape, dtype=torch.float16).pin_memory()
+    hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    ws = pab.Workspace.for_config(cfg, device, auto=True)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        gq.copy_(hq, non_blocking=True)
+        gk.copy_(hk, non_blocking=True)
+        gv.copy_(hv, non_blocking=True)
+        pab.attn_fwd_auto(gq, gk, gv, cfg, out=out, lse=lse, ws=ws)
+        ho.copy_(out, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    steps = max(3, min(args.steps, 20))
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=device)
+    if dist:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    value = world * effective_flops(w) * steps / (float(ms[0]) * 1e-3) / 1e12
+    return {"value": value, "unit": "TFLOPS", "steps": steps,
+            "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
+            "d2h_bytes_per_step": int(ho.numel() * 2 + hl.numel() * 4),
+            "ms_per_step": float(ms[0]) / steps}
+
+
+if __name__ == "__main__":
+    main()

@@ -3,7 +3,8 @@
 Bar: NVFP4 codes and scales bit-exact; block scores and the selected set exact (ties go to the
 smaller index on both sides, and both evaluate S^ with the same float64 operation order; a pair
 within 1e-6 relative of the k-th score may differ); attention output within rel-L2 <= 1e-3 and
-max-abs <= 1e-2 of the oracle, LSE within 1e-3.  Full tensors for the small workloads, a seeded
+max-abs <= 1e-2 of the oracle (one FP16 step where that step is larger, |O| >= 16), LSE within
+1e-3.  Full tensors for the small workloads, a seeded
 stratified sample of (batch, head, query block) units for the long ones.
 """
 
@@ -139,11 +140,22 @@ def compare_attention(out_g, lse_g, out_o, lse_o, w, units):
         lse_ro.append(lo[b, h, sl])
     a, e = np.concatenate(rows_g), np.concatenate(rows_o)
     rel = np.linalg.norm(a - e) / np.linalg.norm(e)
-    mx = np.abs(a - e).max()
+    err = np.abs(a - e)
+    mx = err.max()
     lmx = np.abs(np.concatenate(lse_rg) - np.concatenate(lse_ro)).max()
     assert np.isfinite(a).all()
-    assert rel <= REL_L2 and mx <= MAX_ABS and lmx <= LSE_ABS, (rel, mx, lmx)
+    # Both sides round their result to FP16 independently: where one FP16 step exceeds 1e-2
+    # (|O| >= 16) the outputs may differ by that one step.
+    bound = np.maximum(MAX_ABS, fp16_ulp(e))
+    print(f"parity: rel-L2 {rel:.3e} max-abs {mx:.3e} lse {lmx:.3e} worst err/bound {(err / bound).max():.3f}")
+    assert rel <= REL_L2 and lmx <= LSE_ABS and np.all(err <= bound), (rel, mx, lmx)
     return rel, mx, lmx
+
+
+def fp16_ulp(x):
+    """Spacing of FP16 numbers at |x| (normal range)."""
+    a = np.maximum(np.abs(x), 2.0 ** -14)
+    return 2.0 ** (np.floor(np.log2(a)) - 10)
 
 
 def run_pair(pab, name, bp=None, n_units=None, auto=False):

@@ -138,6 +138,9 @@ WORKLOADS = {
     "n4k": Workload("n4k", 1, 1, 8, 8, 4096, 128, False, 128, 64, -1, 500, "heavy_bias"),
     "prefill32k": Workload("prefill32k", 2, 1, 32, 8, 32768, 128, True, 128, 64, -1, 500,
                            "heavy_bias"),
+    # same distribution and blocking as the 32K prefill at half the length: a profiling size
+    "prefill16k": Workload("prefill16k", 5, 1, 32, 8, 16384, 128, True, 128, 64, -1, 500,
+                           "heavy_bias"),
     "long131k": Workload("long131k", 3, 1, 32, 8, 131072, 128, True, 128, 128, -1, 200,
                          "student_t"),
     "diffusion": Workload("diffusion", 4, 2, 24, 24, 16384, 64, False, 128, 64, -1, 500,
