@@ -27,7 +27,8 @@ namespace thrift {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // warp 0 producer, warp 1 MMA, warps 2-9 softmax (two per TMEM lane quarter)
+constexpr int kSoftmaxThreads = 256;
 constexpr int kBQ = 128;
 constexpr long long kWaitLimit = 1ll << 32;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -54,7 +55,7 @@ struct Layout {
   static constexpr int OFF_SLOTS = OFF_Q16 + Q16_BYTES;
   static constexpr int OFF_P = OFF_SLOTS + NSLOT * SLOT_BYTES;
   static constexpr int OFF_BAR = OFF_P + 2 * PBUF_BYTES;
-  static constexpr int BYTES = OFF_BAR + 512 + 1024;  // barriers + alignment slack
+  static constexpr int BYTES = OFF_BAR + 2048 + 1024;  // barriers + alignment slack
   // TMEM columns
   static constexpr int COL_S = 0;  // two buffers of BK columns
   static constexpr int COL_PV = 2 * BK;
@@ -76,6 +77,7 @@ struct Bars {
   uint64_t kv_full[6], kv_empty[6];
   uint32_t tmem_base;
   int abort_flag;
+  float lpart[2][128];  // per-row partial softmax denominators of the two key halves
 };
 
 struct AttnParams {
@@ -187,7 +189,129 @@ __device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t a) {
   asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
 }
 
-template <int D, int BK>
+
+constexpr float kNegInf = -__builtin_huge_valf();
+constexpr float kRescale = 8.0f;  // log2 units: rescale O only when the block max grows past 256x
+
+__device__ __forceinline__ void load_s64(uint32_t taddr, float (&s)[64]) {
+  uint32_t r0[32], r1[32];
+  tmem_ld32(taddr, r0);
+  tmem_ld32(taddr + 32, r1);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    s[i] = __uint_as_float(r0[i]);
+    s[32 + i] = __uint_as_float(r1[i]);
+  }
+}
+
+__device__ __forceinline__ void load_s32(uint32_t taddr, float (&s)[32]) {
+  uint32_t r0[32];
+  tmem_ld32(taddr, r0);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(r0[i]);
+}
+
+// Rows that do not take part in this block, and keys above the query (causal), become -inf.
+template <int n>
+__device__ __forceinline__ void mask_s(float (&s)[n], bool part, bool diag, int key0, int row) {
+  if (!part) {
+#pragma unroll
+    for (int i = 0; i < n; ++i) s[i] = kNegInf;
+  } else if (diag) {
+#pragma unroll
+    for (int i = 0; i < n; ++i) s[i] = (key0 + i > row) ? kNegInf : s[i];
+  }
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+template <int n>
+__device__ __forceinline__ void group_max(const float (&s)[n], float* gm) {
+#pragma unroll
+  for (int q = 0; q < n / 16; ++q) {
+    const float* x = s + 16 * q;
+    float a = max3(x[0], x[1], x[2]), b = max3(x[3], x[4], x[5]), c = max3(x[6], x[7], x[8]);
+    float d = max3(x[9], x[10], x[11]), e = max3(x[12], x[13], x[14]);
+    gm[q] = max3(max3(a, b, c), max3(d, e, x[15]), kNegInf);
+  }
+}
+
+// FP16 probabilities of 32 keys: exp2(s * sl2 - Ms) rounded to FP16 pairs; returns their FP32 sum.
+__device__ __forceinline__ float probs_fp16_32(const float (&s)[32], float sl2, float Ms, uint32_t (&hw)[16]) {
+  const float2 a2 = make_float2(sl2, sl2), b2 = make_float2(-Ms, -Ms);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    float2 x = __ffma2_rn(make_float2(s[i], s[i + 1]), a2, b2);
+    float2 pr = make_float2(ex2(x.x), ex2(x.y));
+    acc[(i >> 1) & 3] = __fadd2_rn(acc[(i >> 1) & 3], pr);
+    hw[i >> 1] = pack_half2(pr.x, pr.y);
+  }
+  float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  return t.x + t.y;
+}
+
+// Eight FP32 values to eight E2M1 codes packed in one word (element 0 in the low nibble).
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float* y) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+  return out;
+}
+
+// NVFP4 re-quantisation of 32 keys (two 16-key groups) of one row:
+//   P^ = exp2(s*sl2 - Ms); per group s_b = E4M3(2688 max(P^) / 6); codes = E2M1(2688 P^ / s_b).
+// 2688 / s_b is folded into the exponent, so each key costs one FMA and one exp2.  A group whose
+// scale underflows to 0 gets all-zero codes (its values are below 2688 * 2^-10 / 6 / 448).
+// Returns the FP32 sum of the unquantised P^; writes 4 code words and 2 scale bytes into sfw at
+// bit offset `shift`.
+__device__ __forceinline__ float probs_nvfp4_32(const float (&s)[32], const float* gm, float sl2, float Ms,
+                                                uint32_t (&cw)[4], uint32_t& sfw, int shift) {
+  float sum = 0.0f;
+  const float2 a2 = make_float2(sl2, sl2);
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const bool live = gm[q] != kNegInf;
+    const float pmax = live ? 2688.0f * ex2(fmaf(gm[q], sl2, -Ms)) : 0.0f;
+    const uint32_t sb = cvt_e4m3(__fdiv_rn(pmax, 6.0f));
+    const float sbf = e4m3_to_f32(sb);
+    const float sbe = sbf > 0.0f ? sbf : 448.0f;
+    const float bias = live ? (11.392317422778761f - __log2f(sbe)) - Ms : kNegInf;  // log2(2688 / s_b) - Ms
+    const float2 b2 = make_float2(bias, bias);
+    float y[16];
+    float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int t = 0; t < 16; t += 2) {
+      float2 x = __ffma2_rn(make_float2(s[16 * q + t], s[16 * q + t + 1]), a2, b2);
+      y[t] = ex2(x.x);
+      y[t + 1] = ex2(x.y);
+      if (t & 2)
+        acc1 = __fadd2_rn(acc1, make_float2(y[t], y[t + 1]));
+      else
+        acc0 = __fadd2_rn(acc0, make_float2(y[t], y[t + 1]));
+    }
+    cw[2 * q] = cvt_e2m1x8(y);
+    cw[2 * q + 1] = cvt_e2m1x8(y + 8);
+    const float2 t2 = __fadd2_rn(acc0, acc1);
+    sum = fmaf(t2.x + t2.y, sbe * (1.0f / 2688.0f), sum);
+    sfw |= sb << (shift + 8 * q);
+  }
+  return sum;
+}
+
+template <int D, int BK, bool DBG>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q4, const __grid_constant__ CUtensorMap tm_k4,
                 const __grid_constant__ CUtensorMap tm_v4, const __grid_constant__ CUtensorMap tm_q16,
@@ -214,11 +338,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->q16_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->s_free[i], 128);
-      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->s_free[i], kSoftmaxThreads);
+      mbar_init(&bars->p_full[i], kSoftmaxThreads);
     }
     mbar_init(&bars->pv_full, 1);
-    mbar_init(&bars->pv_free, 128);
+    mbar_init(&bars->pv_free, kSoftmaxThreads);
     for (int i = 0; i < L::NSLOT; ++i) {
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
@@ -435,56 +559,78 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax / merge
+    // Two warps share each TMEM lane quarter (the same 32 rows): both read the whole score row
+    // and find the same block and group maxima; warp half `hh` then produces the probabilities
+    // of keys [hh*BK/2, (hh+1)*BK/2) and accumulates output columns [hh*D/2, (hh+1)*D/2).
+    const int sw = warp - 2;
     const int quarter = warp & 3;
+    const int hh = sw >> 2;
     const int rr = quarter * 32 + lane;  // row of the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    constexpr int DH = D / 2, KH = BK / 2;
     const float q_ts = (p.mode != 2) ? __ldg(p.q_ts) : 1.0f;
     const float k_ts = (p.mode != 2) ? __ldg(p.k_ts) : 1.0f;
     const float v_ts = (p.mode != 2) ? __ldg(p.v_ts) : 1.0f;
     const float sl2_4 = q_ts * k_ts * p.tau * kLog2e;
     const float sl2_16 = p.tau * kLog2e;
     const float pv4_scale = v_ts * (1.0f / 2688.0f);
-    const float NEG_INF = -__int_as_float(0x7f800000);
     uint32_t g = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       UnitInfo ui = decode_unit(p, u);
       const int row = ui.t * kBQ + rr;
       const int half = (p.bq == 64) ? (rr >> 6) : 0;
-      float O[D];
+      float O[DH];
 #pragma unroll
-      for (int c = 0; c < D; ++c) O[c] = 0.0f;
-      float m_run = NEG_INF, l_run = 0.0f;
-      float pend_M = NEG_INF, pend_sum = 0.0f;
+      for (int c = 0; c < DH; ++c) O[c] = 0.0f;
+      // running state: O and l are relative to exp2(m_ref); m_ref moves only when a block's
+      // maximum exceeds it by more than 2^kRescale (the final O / l does not depend on m_ref)
+      float m_ref = kNegInf, l_run = 0.0f;
+      float pend_M = kNegInf, pend_sum = 0.0f;
       int pend_f16 = 0;
       bool have_pend = false;
-      const bool dbg_unit = p.dbg && blockIdx.x == 0 && u == (int)blockIdx.x;
+      const bool dbg_unit = DBG && p.dbg && blockIdx.x == 0 && u == (int)blockIdx.x;
       int local_e = 0;
 
       auto merge = [&](uint32_t ge) -> bool {
         if (!mbar_wait(&bars->pv_full, ge & 1, abort_flag, p.status, lim)) return false;
         tc_fence_after();
-        const float m_new = fmaxf(m_run, pend_M);
-        const float alpha = (m_run == NEG_INF) ? 0.0f : ex2(m_run - m_new);
-        const float gs = (pend_M == NEG_INF) ? 0.0f : ex2(pend_M - m_new);
+        const bool need = pend_M != kNegInf && (m_ref == kNegInf || pend_M > m_ref + kRescale);
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? (m_ref == kNegInf ? 0.0f : ex2(m_ref - pend_M)) : 1.0f;
+          const float2 a2 = make_float2(alpha, alpha);
+          l_run *= alpha;
+#pragma unroll
+          for (int c = 0; c < DH; c += 2) {
+            float2 o = __fmul2_rn(make_float2(O[c], O[c + 1]), a2);
+            O[c] = o.x;
+            O[c + 1] = o.y;
+          }
+          if (need) m_ref = pend_M;
+        }
+        const float gs = (pend_M == kNegInf) ? 0.0f : ex2(pend_M - m_ref);
+        l_run = fmaf(gs, pend_sum, l_run);
         const float gpv = pend_f16 ? gs : gs * pv4_scale;
-        l_run = alpha * l_run + gs * pend_sum;
-        const bool dump = dbg_unit && (local_e - 1) == p.dbg_entry;
+        const float2 g2 = make_float2(gpv, gpv);
+        uint32_t r[DH];
+        const uint32_t pva = tmem + lane_base + L::COL_PV + hh * DH;
+        tmem_ld32(pva, *reinterpret_cast<uint32_t(*)[32]>(r));
+        if constexpr (DH == 64) tmem_ld32(pva + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + L::COL_PV + 32 * c, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float v = __uint_as_float(r[i]);
-            O[32 * c + i] = fmaf(gpv, v, alpha * O[32 * c + i]);
-            if (dump) p.dbg[kBQ * BK + kBQ * (BK * 2 / 4) + rr * D + 32 * c + i] = v;
+        for (int i = 0; i < DH; i += 2) {
+          float2 o = __ffma2_rn(g2, make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])),
+                                make_float2(O[i], O[i + 1]));
+          O[i] = o.x;
+          O[i + 1] = o.y;
+        }
+        if constexpr (DBG) {
+          if (dbg_unit && (local_e - 1) == p.dbg_entry) {
+            for (int i = 0; i < DH; ++i) p.dbg[kBQ * BK + kBQ * (BK / 2) + rr * D + hh * DH + i] = __uint_as_float(r[i]);
           }
         }
         tc_fence_before();
         mbar_arrive(&bars->pv_free);
-        m_run = (m_new == NEG_INF) ? m_run : m_new;
         return true;
       };
 
@@ -499,124 +645,88 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int key0 = j * BK;
         const uint32_t saddr = tmem + lane_base + L::COL_S + buf * BK;
         const float sl2 = f16 ? sl2_16 : sl2_4;
-        const bool dump = dbg_unit && local_e == p.dbg_entry;
-        // pass 1: maxima of every 16-key group
+        const bool dumpP = dbg_unit && local_e == p.dbg_entry;
+        const bool dump = dumpP && hh == 0;
+        const uint32_t pb = smem_u32(sP + buf * L::PBUF_BYTES);
+
+        // pass 1: the score row (32 columns per TMEM round trip), masked, and its 16-key group
+        // maxima (both warps of the lane quarter find the same values)
         float gmax[BK / 16];
 #pragma unroll
         for (int c = 0; c < BK / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(saddr + 32 * c, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            float mx = NEG_INF;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int col = 32 * c + 16 * h2 + i;
-              float s = __uint_as_float(r[16 * h2 + i]);
-              if (dump) p.dbg[rr * BK + col] = s;
-              const bool masked = !part || (diag && key0 + col > row);
-              mx = masked ? mx : fmaxf(mx, s);
-            }
-            gmax[2 * c + h2] = mx;
+          float s[32];
+          load_s32(saddr + 32 * c, s);
+          if constexpr (DBG) {
+            if (dump)
+              for (int i = 0; i < 32; ++i) p.dbg[rr * BK + 32 * c + i] = s[i];
           }
+          mask_s(s, part, diag, key0 + 32 * c, row);
+          group_max<32>(s, gmax + 2 * c);
         }
-        float M = NEG_INF;
+        float M = kNegInf;
 #pragma unroll
         for (int q = 0; q < BK / 16; ++q) M = fmaxf(M, gmax[q]);
-        const bool valid = M != NEG_INF;
+        const bool valid = M != kNegInf;  // false when every key of the block is masked for this row
         const float Ms = valid ? M * sl2 : 0.0f;
-        // pass 2: probabilities, their sum, and the PV operand in shared memory
-        const uint32_t pb = smem_u32(sP + buf * L::PBUF_BYTES);
+
+        // pass 2: probabilities of this warp's keys relative to the block maximum, their partial
+        // sum, and this warp's part of the PV operand in shared memory
         float sum = 0.0f;
-        uint32_t sfw[BK / 64];
 #pragma unroll
-        for (int q = 0; q < BK / 64; ++q) sfw[q] = 0u;
-#pragma unroll
-        for (int c = 0; c < BK / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(saddr + 32 * c, r);
-          tmem_wait_ld();
-          float pr[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int col = 32 * c + i;
-            const bool masked = !valid || !part || (diag && key0 + col > row);
-            pr[i] = masked ? 0.0f : ex2(fmaf(__uint_as_float(r[i]), sl2, -Ms));
-            sum += pr[i];
+        for (int c2 = 0; c2 < KH / 32; ++c2) {
+          const int c = hh * (KH / 32) + c2;  // 32-key chunk index within the row
+          float s32[32];
+          load_s32(saddr + 32 * c, s32);
+          mask_s(s32, part, diag, key0 + 32 * c, row);
+          float gm2[2];  // this chunk's two group maxima, selected without dynamic register indexing
+          gm2[0] = gmax[2 * c2];
+          gm2[1] = gmax[2 * c2 + 1];
+          if (hh) {
+            gm2[0] = gmax[KH / 16 + 2 * c2];
+            gm2[1] = gmax[KH / 16 + 2 * c2 + 1];
           }
           if (f16) {
             uint32_t hw[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) hw[i] = pack_half2(pr[2 * i], pr[2 * i + 1]);
+            sum += probs_fp16_32(s32, sl2, Ms, hw);
+            if constexpr (DBG) {
+              if (dumpP)
+                for (int i = 0; i < 16; ++i) reinterpret_cast<uint32_t*>(p.dbg + kBQ * BK + rr * (BK / 2))[16 * c + i] = hw[i];
+            }
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const int chunk = 4 * c + q;  // 16-byte chunk index along the row (8 keys)
+              const int chunk = 4 * c + q;  // 16-byte chunk of the row (8 keys)
               const int cb = chunk >> 3, c8 = chunk & 7;
-              const uint32_t addr = pb + cb * kBQ * 128 + rr * 128 + ((c8 ^ (rr & 7)) << 4);
-              st_shared_v4(addr, hw[4 * q], hw[4 * q + 1], hw[4 * q + 2], hw[4 * q + 3]);
+              st_shared_v4(pb + cb * kBQ * 128 + rr * 128 + ((c8 ^ (rr & 7)) << 4), hw[4 * q], hw[4 * q + 1],
+                           hw[4 * q + 2], hw[4 * q + 3]);
             }
           } else {
-            uint32_t w[4];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const float gm = gmax[2 * c + h2];
-              const float pmax = (valid && gm != NEG_INF) ? 2688.0f * ex2(fmaf(gm, sl2, -Ms)) : 0.0f;
-              const uint32_t sb = cvt_e4m3(__fdiv_rn(pmax, 6.0f));
-              const float sbf = e4m3_to_f32(sb);
-              const float inv = sbf > 0.0f ? __fdiv_rn(2688.0f, sbf) : 0.0f;
-              uint32_t lo = 0, hi = 0;
-#pragma unroll
-              for (int i = 0; i < 8; i += 2) lo |= cvt_e2m1x2(pr[16 * h2 + i] * inv, pr[16 * h2 + i + 1] * inv) << (4 * i);
-#pragma unroll
-              for (int i = 0; i < 8; i += 2)
-                hi |= cvt_e2m1x2(pr[16 * h2 + 8 + i] * inv, pr[16 * h2 + 8 + i + 1] * inv) << (4 * i);
-              w[2 * h2] = lo;
-              w[2 * h2 + 1] = hi;
-              const int grp = 2 * c + h2;  // 16-key group index in the row
-              sfw[grp >> 2] |= sb << (8 * (grp & 3));
+            uint32_t cw[4], sfw = 0u;
+            sum += probs_nvfp4_32(s32, gm2, sl2, Ms, cw, sfw, 0);
+            if constexpr (DBG) {
+              if (dumpP) {
+                uint8_t* db = reinterpret_cast<uint8_t*>(p.dbg + kBQ * BK + rr * (BK / 2));
+                for (int i = 0; i < 4; ++i) reinterpret_cast<uint32_t*>(db + 16 * c)[i] = cw[i];
+                db[BK / 2 + 2 * c] = (uint8_t)(sfw & 255u);
+                db[BK / 2 + 2 * c + 1] = (uint8_t)(sfw >> 8);
+              }
             }
-            // 32 keys = one 16-byte chunk of the row
-            constexpr int ROWB = BK / 2;
             uint32_t addr;
-            if (ROWB == 32)
+            if (BK == 64)
               addr = pb + rr * 32 + ((c ^ ((rr >> 2) & 1)) << 4);
             else
               addr = pb + rr * 64 + ((c ^ ((rr >> 1) & 3)) << 4);
-            st_shared_v4(addr, w[0], w[1], w[2], w[3]);
+            st_shared_v4(addr, cw[0], cw[1], cw[2], cw[3]);
+            // the two scale bytes of this chunk's 16-key groups
+            const uint32_t sfa = pb + L::P4_BYTES + (c >> 1) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + 2 * (c & 1);
+            asm volatile("st.shared.b16 [%0], %1;" ::"r"(sfa), "h"((uint16_t)sfw) : "memory");
           }
-        }
-        if (!f16) {
-#pragma unroll
-          for (int q = 0; q < BK / 64; ++q)
-            st_shared_u32(pb + L::P4_BYTES + q * 512 + (rr & 31) * 16 + (rr >> 5) * 4, sfw[q]);
         }
         tc_fence_before();
         mbar_arrive(&bars->s_free[buf]);
-        if (dump) {
-          // raw bytes of this row of the PV operand (FP16: BK halves; NVFP4: codes + scale bytes)
-          float* db = p.dbg + kBQ * BK + rr * (BK * 2 / 4);
-          const uint8_t* base = sP + buf * L::PBUF_BYTES;
-          if (f16) {
-            for (int ch = 0; ch < BK / 8; ++ch) {
-              const int cb = ch >> 3, c8 = ch & 7;
-              const uint4 v = *reinterpret_cast<const uint4*>(base + cb * kBQ * 128 + rr * 128 + ((c8 ^ (rr & 7)) << 4));
-              reinterpret_cast<uint4*>(db)[ch] = v;
-            }
-          } else {
-            constexpr int ROWB = BK / 2;
-            for (int ch = 0; ch < ROWB / 16; ++ch) {
-              int phys = ROWB == 32 ? (ch ^ ((rr >> 2) & 1)) : (ch ^ ((rr >> 1) & 3));
-              reinterpret_cast<uint4*>(db)[ch] = *reinterpret_cast<const uint4*>(base + rr * ROWB + (phys << 4));
-            }
-            for (int q = 0; q < BK / 64; ++q)
-              reinterpret_cast<uint32_t*>(db)[ROWB / 4 + q] = sfw[q];
-          }
-        }
         fence_proxy_async_smem();
         mbar_arrive(&bars->p_full[buf]);
         if (have_pend && !(ok = merge(g - 1))) break;
-        pend_M = valid ? Ms : NEG_INF;
+        pend_M = valid ? Ms : kNegInf;
         pend_sum = sum;
         pend_f16 = f16;
         have_pend = true;
@@ -625,12 +735,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok && have_pend) ok = merge(g - 1);
       if (!ok) break;
+      // combine the two halves' partial denominators
+      bars->lpart[hh][rr] = l_run;
+      asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
+      const float l_tot = l_run + bars->lpart[1 - hh][rr];
+      asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
       // epilogue: O / l in FP16, lse in natural-log units of the tau-scaled scores
-      const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+      const float inv_l = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
       const int64_t orow = (int64_t)(ui.b * p.Hq + ui.h) * p.N + row;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D + hh * DH);
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
+      for (int c = 0; c < DH / 8; ++c) {
         uint4 v;
         v.x = pack_half2(O[8 * c] * inv_l, O[8 * c + 1] * inv_l);
         v.y = pack_half2(O[8 * c + 2] * inv_l, O[8 * c + 3] * inv_l);
@@ -638,7 +753,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         v.w = pack_half2(O[8 * c + 6] * inv_l, O[8 * c + 7] * inv_l);
         dst[c] = v;
       }
-      if (p.lse) p.lse[orow] = (m_run + __log2f(l_run)) * kLn2;
+      if (p.lse && hh == 0) p.lse[orow] = (m_ref + __log2f(l_tot)) * kLn2;
     }
   }
 
@@ -706,7 +821,7 @@ thrift_status launch_t(const void* q, const void* k, const void* v, const thrift
     ok &= make_map(&maps[5], v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, D, krows, 64, BK, CU_TENSOR_MAP_SWIZZLE_128B);
   }
   if (!ok) return THRIFT_ERR_CUDA;
-  auto kern = attn_kernel<D, BK>;
+  auto kern = prm.dbg ? attn_kernel<D, BK, true> : attn_kernel<D, BK, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES) != cudaSuccess)
     return THRIFT_ERR_CUDA;
   int grid = num_sms();

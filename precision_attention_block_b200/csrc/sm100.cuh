@@ -45,21 +45,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Shared abort state of one CTA: once any wait gives up, every later wait returns at once so
-// that all warps reach the kernel's end, release TMEM and exit.
-struct AbortState {
-  int flag;
-};
+// try_wait that lets the hardware suspend the thread (up to `hint_ns`) until the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 
 // Bounded wait for the phase with the given parity.  Gives up after `limit` clock cycles,
-// records the timeout in the global status word and raises the CTA's abort flag.
+// records the timeout in the global status word and raises the CTA's abort flag (a shared flag:
+// once any wait of the CTA gives up, every later wait returns at once, so that all warps reach
+// the kernel's end, release TMEM and exit).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int* status, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
     if (*abort_flag) return false;
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
     if (clock64() - t0 > limit) {
       *abort_flag = 1;
       if (status) atomicOr(status, kStatusTimeout);
