@@ -55,7 +55,7 @@ struct Layout {
   static constexpr int OFF_SLOTS = OFF_Q16 + Q16_BYTES;
   static constexpr int OFF_P = OFF_SLOTS + NSLOT * SLOT_BYTES;
   static constexpr int OFF_BAR = OFF_P + 2 * PBUF_BYTES;
-  static constexpr int BYTES = OFF_BAR + 2048 + 1024;  // barriers + alignment slack
+  static constexpr int BYTES = OFF_BAR + 4096 + 1024;  // barriers + alignment slack
   // TMEM columns
   static constexpr int COL_S = 0;  // two buffers of BK columns
   static constexpr int COL_PV = 2 * BK;
@@ -77,7 +77,8 @@ struct Bars {
   uint64_t kv_full[6], kv_empty[6];
   uint32_t tmem_base;
   int abort_flag;
-  float lpart[2][128];  // per-row partial softmax denominators of the two key halves
+  float lpart[2][128];      // per-row partial softmax denominators of the two key halves
+  float mswap[2][2][128];   // per-entry half-row maxima swapped between the two warps of a row
 };
 
 struct AttnParams {
@@ -285,7 +286,7 @@ __device__ __forceinline__ float probs_nvfp4_32(const float (&s)[32], const floa
   for (int q = 0; q < 2; ++q) {
     const bool live = gm[q] != kNegInf;
     const float pmax = live ? 2688.0f * ex2(fmaf(gm[q], sl2, -Ms)) : 0.0f;
-    const uint32_t sb = cvt_e4m3(__fdiv_rn(pmax, 6.0f));
+    const uint32_t sb = cvt_e4m3(pmax * (1.0f / 6.0f));
     const float sbf = e4m3_to_f32(sb);
     const float sbe = sbf > 0.0f ? sbf : 448.0f;
     const float bias = live ? (11.392317422778761f - __log2f(sbe)) - Ms : kNegInf;  // log2(2688 / s_b) - Ms
@@ -646,45 +647,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t saddr = tmem + lane_base + L::COL_S + buf * BK;
         const float sl2 = f16 ? sl2_16 : sl2_4;
         const bool dumpP = dbg_unit && local_e == p.dbg_entry;
-        const bool dump = dumpP && hh == 0;
         const uint32_t pb = smem_u32(sP + buf * L::PBUF_BYTES);
 
-        // pass 1: the score row (32 columns per TMEM round trip), masked, and its 16-key group
-        // maxima (both warps of the lane quarter find the same values)
-        float gmax[BK / 16];
+        // this warp's keys [hh*BK/2, (hh+1)*BK/2) of the score row: one TMEM round trip, then the
+        // scores live in registers and the buffer goes back to the MMA warp
+        float sv[KH];
 #pragma unroll
-        for (int c = 0; c < BK / 32; ++c) {
-          float s[32];
-          load_s32(saddr + 32 * c, s);
-          if constexpr (DBG) {
-            if (dump)
-              for (int i = 0; i < 32; ++i) p.dbg[rr * BK + 32 * c + i] = s[i];
-          }
-          mask_s(s, part, diag, key0 + 32 * c, row);
-          group_max<32>(s, gmax + 2 * c);
+        for (int c2 = 0; c2 < KH / 32; ++c2) tmem_ld32(saddr + KH * hh + 32 * c2, *reinterpret_cast<uint32_t(*)[32]>(sv + 32 * c2));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->s_free[buf]);
+        if constexpr (DBG) {
+          if (dumpP)
+            for (int i = 0; i < KH; ++i) p.dbg[rr * BK + KH * hh + i] = sv[i];
         }
-        float M = kNegInf;
+        float gmax[KH / 16];
 #pragma unroll
-        for (int q = 0; q < BK / 16; ++q) M = fmaxf(M, gmax[q]);
+        for (int c2 = 0; c2 < KH / 32; ++c2) {
+          float* s32 = sv + 32 * c2;
+          mask_s(*reinterpret_cast<float(*)[32]>(s32), part, diag, key0 + KH * hh + 32 * c2, row);
+          group_max<32>(*reinterpret_cast<float(*)[32]>(s32), gmax + 2 * c2);
+        }
+        float Mh = kNegInf;
+#pragma unroll
+        for (int q = 0; q < KH / 16; ++q) Mh = fmaxf(Mh, gmax[q]);
+        // the block maximum over both halves: swap half maxima with the partner warp of this lane
+        // quarter through shared memory (two buffers, alternating per entry)
+        bars->mswap[buf][hh][rr] = Mh;
+        asm volatile("bar.sync %0, 64;" ::"r"(2 + quarter) : "memory");
+        const float M = fmaxf(Mh, bars->mswap[buf][1 - hh][rr]);
         const bool valid = M != kNegInf;  // false when every key of the block is masked for this row
         const float Ms = valid ? M * sl2 : 0.0f;
 
-        // pass 2: probabilities of this warp's keys relative to the block maximum, their partial
-        // sum, and this warp's part of the PV operand in shared memory
+        // probabilities of this warp's keys relative to the block maximum, their partial sum, and
+        // this warp's part of the PV operand in shared memory
         float sum = 0.0f;
 #pragma unroll
         for (int c2 = 0; c2 < KH / 32; ++c2) {
           const int c = hh * (KH / 32) + c2;  // 32-key chunk index within the row
-          float s32[32];
-          load_s32(saddr + 32 * c, s32);
-          mask_s(s32, part, diag, key0 + 32 * c, row);
-          float gm2[2];  // this chunk's two group maxima, selected without dynamic register indexing
-          gm2[0] = gmax[2 * c2];
-          gm2[1] = gmax[2 * c2 + 1];
-          if (hh) {
-            gm2[0] = gmax[KH / 16 + 2 * c2];
-            gm2[1] = gmax[KH / 16 + 2 * c2 + 1];
-          }
+          float(&s32)[32] = *reinterpret_cast<float(*)[32]>(sv + 32 * c2);
           if (f16) {
             uint32_t hw[16];
             sum += probs_fp16_32(s32, sl2, Ms, hw);
@@ -701,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else {
             uint32_t cw[4], sfw = 0u;
-            sum += probs_nvfp4_32(s32, gm2, sl2, Ms, cw, sfw, 0);
+            sum += probs_nvfp4_32(s32, gmax + 2 * c2, sl2, Ms, cw, sfw, 0);
             if constexpr (DBG) {
               if (dumpP) {
                 uint8_t* db = reinterpret_cast<uint8_t*>(p.dbg + kBQ * BK + rr * (BK / 2));
@@ -721,8 +722,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             asm volatile("st.shared.b16 [%0], %1;" ::"r"(sfa), "h"((uint16_t)sfw) : "memory");
           }
         }
-        tc_fence_before();
-        mbar_arrive(&bars->s_free[buf]);
         fence_proxy_async_smem();
         mbar_arrive(&bars->p_full[buf]);
         if (have_pend && !(ok = merge(g - 1))) break;
