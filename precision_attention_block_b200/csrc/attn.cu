@@ -54,7 +54,9 @@ struct Layout {
   static constexpr int OFF_Q16 = round1024(OFF_QSF + QSF_BYTES);
   static constexpr int OFF_SLOTS = OFF_Q16 + Q16_BYTES;
   static constexpr int OFF_P = OFF_SLOTS + NSLOT * SLOT_BYTES;
-  static constexpr int OFF_BAR = OFF_P + 2 * PBUF_BYTES;
+  static constexpr int MAXE = 4096;  // entries per unit (two phases of at most 2048 key blocks)
+  static constexpr int OFF_LIST = OFF_P + 2 * PBUF_BYTES;
+  static constexpr int OFF_BAR = OFF_LIST + 2 * MAXE * 2;
   static constexpr int BYTES = OFF_BAR + 4096 + 1024;  // barriers + alignment slack
   // TMEM columns
   static constexpr int COL_S = 0;  // two buffers of BK columns
@@ -75,6 +77,8 @@ struct Bars {
   uint64_t s_full[2], s_free[2], p_full[2];
   uint64_t pv_full, pv_free;
   uint64_t kv_full[6], kv_empty[6];
+  uint64_t list_full[2], list_empty[2];  // per-unit entry lists, double-buffered by unit parity
+  int list_count[2];
   uint32_t tmem_base;
   int abort_flag;
   float lpart[2][128];      // per-row partial softmax denominators of the two key halves
@@ -169,6 +173,27 @@ __device__ __forceinline__ EntryIter make_iter(const AttnParams& p, const UnitIn
   it.phase = 0;
   it.j = 0;
   return it;
+}
+
+// The unit's entry list, built once by a whole warp: NVFP4 entries, then FP16 entries, each as
+// j | fp16 << 13 | row-half mask << 14.  Returns the number of entries (same in every lane).
+template <int BK>
+__device__ int build_list(const AttnParams& p, const UnitInfo& ui, uint16_t* list, int lane) {
+  EntryIter it = make_iter<BK>(p, ui);
+  int n = 0;
+  for (int phase = 0; phase < 2; ++phase) {
+    for (int jb = 0; jb < it.jmax; jb += 32) {
+      const int jj = jb + lane;
+      int rm = 0;
+      if (jj < it.jmax0 && it.sel(it.m0, jj) == phase) rm |= 1;
+      if (it.two && jj < it.jmax1 && it.sel(it.m1, jj) == phase) rm |= 2;
+      if (!it.two && rm) rm = 3;
+      const unsigned b = __ballot_sync(0xffffffffu, rm != 0);
+      if (rm) list[n + __popc(b & ((1u << lane) - 1u))] = (uint16_t)(jj | (phase << 13) | (rm << 14));
+      n += __popc(b);
+    }
+  }
+  return n;
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -348,6 +373,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->list_full[i], 1);
+      mbar_init(&bars->list_empty[i], 1 + kSoftmaxThreads);
+    }
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -363,6 +392,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
+    // The whole warp builds each unit's entry list; lane 0 then issues the unit's loads.
+    uint16_t* lists = reinterpret_cast<uint16_t*>(smem + L::OFF_LIST);
     if (lane == 0) {
       if (p.mode != 2) {
         prefetch_tmap(&tm_q4);
@@ -374,68 +405,88 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_k16);
         prefetch_tmap(&tm_v16);
       }
+    }
+    {
       uint32_t slot_ctr = 0, unit_ctr = 0, u16_ctr = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_ctr) {
+      // lane 0: every load of one unit (returns false after a timeout)
+      auto issue_unit = [&](const UnitInfo& ui, const uint16_t* list, int n_entries) -> bool {
+          const int qrow0 = (ui.b * p.Hq + ui.h) * p.N + ui.t * kBQ;
+          const int kvh = ui.b * p.Hkv + ui.hk;
+          if (!mbar_wait(&bars->q_empty, (unit_ctr & 1) ^ 1, abort_flag, p.status, lim)) return false;
+          if (p.mode != 2) {
+            mbar_arrive_expect_tx(&bars->q_full, L::Q4_BYTES + L::QSF_BYTES);
+            tma_load_2d(sQ4, &tm_q4, &bars->q_full, 0, qrow0);
+            bulk_load(sQSF, p.q_sf + (size_t)(qrow0 / 128) * L::QSF_BYTES, L::QSF_BYTES, &bars->q_full);
+          } else {
+            mbar_arrive(&bars->q_full);
+          }
+          bool q16_loaded = false;
+          for (int e = 0; e < n_entries; ++e) {
+            const uint32_t x = list[e];
+            const int j = x & 0x1fff, f16 = (x >> 13) & 1;
+            if (f16 && !q16_loaded) {
+              if (!(ok = mbar_wait(&bars->q16_empty, (u16_ctr & 1) ^ 1, abort_flag, p.status, lim))) break;
+              mbar_arrive_expect_tx(&bars->q16_full, L::Q16_BYTES);
+  #pragma unroll
+              for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(sQ16 + cb * kBQ * 128, &tm_q16, &bars->q16_full, cb * 64, qrow0);
+              q16_loaded = true;
+            }
+            const int krow0 = kvh * p.N + j * BK;
+            // K tile
+            {
+              uint32_t s = slot_ctr % L::NSLOT, ph = (slot_ctr / L::NSLOT) & 1;
+              ++slot_ctr;
+              if (!(ok = mbar_wait(&bars->kv_empty[s], ph ^ 1, abort_flag, p.status, lim))) break;
+              uint8_t* dst = sSlots + s * L::SLOT_BYTES;
+              if (f16) {
+                mbar_arrive_expect_tx(&bars->kv_full[s], BK * D * 2);
+  #pragma unroll
+                for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(dst + cb * BK * 128, &tm_k16, &bars->kv_full[s], cb * 64, krow0);
+              } else {
+                mbar_arrive_expect_tx(&bars->kv_full[s], BK * D / 2 + L::QSF_BYTES);
+                tma_load_2d(dst, &tm_k4, &bars->kv_full[s], 0, krow0);
+                bulk_load(dst + BK * D / 2, p.k_sf + (size_t)(krow0 / 128) * L::QSF_BYTES, L::QSF_BYTES, &bars->kv_full[s]);
+              }
+            }
+            // V tile
+            {
+              uint32_t s = slot_ctr % L::NSLOT, ph = (slot_ctr / L::NSLOT) & 1;
+              ++slot_ctr;
+              if (!(ok = mbar_wait(&bars->kv_empty[s], ph ^ 1, abort_flag, p.status, lim))) break;
+              uint8_t* dst = sSlots + s * L::SLOT_BYTES;
+              if (f16) {
+                mbar_arrive_expect_tx(&bars->kv_full[s], BK * D * 2);
+  #pragma unroll
+                for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(dst + cb * BK * 128, &tm_v16, &bars->kv_full[s], cb * 64, krow0);
+              } else {
+                const int vrow0 = kvh * D;
+                mbar_arrive_expect_tx(&bars->kv_full[s], D * BK / 2 + L::PSF_BYTES);
+                tma_load_2d(dst, &tm_v4, &bars->kv_full[s], j * (BK / 2), vrow0);
+                size_t sf_off = ((size_t)(vrow0 / 128) * (p.N / 64) + (size_t)j * (BK / 64)) * 512;
+                bulk_load(dst + D * BK / 2, p.v_sf + sf_off, L::PSF_BYTES, &bars->kv_full[s]);
+              }
+            }
+          }
+          if (q16_loaded) ++u16_ctr;
+          return ok;
+      };
+      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x, ++unit_ctr) {
         UnitInfo ui = decode_unit(p, u);
-        const int qrow0 = (ui.b * p.Hq + ui.h) * p.N + ui.t * kBQ;
-        const int kvh = ui.b * p.Hkv + ui.hk;
-        if (!(ok = mbar_wait(&bars->q_empty, (unit_ctr & 1) ^ 1, abort_flag, p.status, lim))) break;
-        if (p.mode != 2) {
-          mbar_arrive_expect_tx(&bars->q_full, L::Q4_BYTES + L::QSF_BYTES);
-          tma_load_2d(sQ4, &tm_q4, &bars->q_full, 0, qrow0);
-          bulk_load(sQSF, p.q_sf + (size_t)(qrow0 / 128) * L::QSF_BYTES, L::QSF_BYTES, &bars->q_full);
-        } else {
-          mbar_arrive(&bars->q_full);
+        const uint32_t lb = unit_ctr & 1;
+        uint16_t* list = lists + lb * L::MAXE;
+        // the warp is converged here: every exit below is taken by all 32 lanes together
+        const bool free_ok = mbar_wait(&bars->list_empty[lb], ((unit_ctr >> 1) & 1) ^ 1, abort_flag, p.status, lim);
+        if (!__all_sync(0xffffffffu, free_ok)) break;
+        const int n_entries = build_list<BK>(p, ui, list, lane);
+        __syncwarp();
+        if (lane == 0) {
+          bars->list_count[lb] = n_entries;
+          mbar_arrive(&bars->list_full[lb]);
+          ok = issue_unit(ui, list, n_entries);
         }
-        bool q16_loaded = false;
-        EntryIter it = make_iter<BK>(p, ui);
-        int j, f16, rm;
-        while (it.next(j, f16, rm)) {
-          if (f16 && !q16_loaded) {
-            if (!(ok = mbar_wait(&bars->q16_empty, (u16_ctr & 1) ^ 1, abort_flag, p.status, lim))) break;
-            mbar_arrive_expect_tx(&bars->q16_full, L::Q16_BYTES);
-#pragma unroll
-            for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(sQ16 + cb * kBQ * 128, &tm_q16, &bars->q16_full, cb * 64, qrow0);
-            q16_loaded = true;
-          }
-          const int krow0 = kvh * p.N + j * BK;
-          // K tile
-          {
-            uint32_t s = slot_ctr % L::NSLOT, ph = (slot_ctr / L::NSLOT) & 1;
-            ++slot_ctr;
-            if (!(ok = mbar_wait(&bars->kv_empty[s], ph ^ 1, abort_flag, p.status, lim))) break;
-            uint8_t* dst = sSlots + s * L::SLOT_BYTES;
-            if (f16) {
-              mbar_arrive_expect_tx(&bars->kv_full[s], BK * D * 2);
-#pragma unroll
-              for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(dst + cb * BK * 128, &tm_k16, &bars->kv_full[s], cb * 64, krow0);
-            } else {
-              mbar_arrive_expect_tx(&bars->kv_full[s], BK * D / 2 + L::QSF_BYTES);
-              tma_load_2d(dst, &tm_k4, &bars->kv_full[s], 0, krow0);
-              bulk_load(dst + BK * D / 2, p.k_sf + (size_t)(krow0 / 128) * L::QSF_BYTES, L::QSF_BYTES, &bars->kv_full[s]);
-            }
-          }
-          // V tile
-          {
-            uint32_t s = slot_ctr % L::NSLOT, ph = (slot_ctr / L::NSLOT) & 1;
-            ++slot_ctr;
-            if (!(ok = mbar_wait(&bars->kv_empty[s], ph ^ 1, abort_flag, p.status, lim))) break;
-            uint8_t* dst = sSlots + s * L::SLOT_BYTES;
-            if (f16) {
-              mbar_arrive_expect_tx(&bars->kv_full[s], BK * D * 2);
-#pragma unroll
-              for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(dst + cb * BK * 128, &tm_v16, &bars->kv_full[s], cb * 64, krow0);
-            } else {
-              const int vrow0 = kvh * D;
-              mbar_arrive_expect_tx(&bars->kv_full[s], D * BK / 2 + L::PSF_BYTES);
-              tma_load_2d(dst, &tm_v4, &bars->kv_full[s], j * (BK / 2), vrow0);
-              size_t sf_off = ((size_t)(vrow0 / 128) * (p.N / 64) + (size_t)j * (BK / 64)) * 512;
-              bulk_load(dst + D * BK / 2, p.v_sf + sf_off, L::PSF_BYTES, &bars->kv_full[s]);
-            }
-          }
-        }
-        if (q16_loaded) ++u16_ctr;
+        __syncwarp();
+        if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
       }
     }
   } else if (warp == 1) {
@@ -498,9 +549,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_copy_sf(tmem + L::COL_SFQ + 4 * kk, make_sdesc(smem_u32(sQSF) + kk * 512, 16, 128, 0));
         }
         bool any16 = false, have_pend = false;
-        EntryIter it = make_iter<BK>(p, ui);
-        int j, f16, rm;
-        while (ok && it.next(j, f16, rm)) {
+        const uint32_t lb = unit_ctr & 1;
+        const uint16_t* list = reinterpret_cast<const uint16_t*>(smem + L::OFF_LIST) + lb * L::MAXE;
+        if (!(ok = mbar_wait(&bars->list_full[lb], (unit_ctr >> 1) & 1, abort_flag, p.status, lim))) break;
+        const int n_entries = bars->list_count[lb];
+        for (int e = 0; ok && e < n_entries; ++e) {
+          const uint32_t x = list[e];
+          const int j = x & 0x1fff, f16 = (x >> 13) & 1;
           uint32_t kslot = slot_ctr % L::NSLOT, kph = (slot_ctr / L::NSLOT) & 1;
           ++slot_ctr;
           uint32_t vslot = slot_ctr % L::NSLOT, vph = (slot_ctr / L::NSLOT) & 1;
@@ -551,6 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok && have_pend) ok = do_pv(pend);
         if (!ok) break;
+        mbar_arrive(&bars->list_empty[lb]);
         tc_commit(&bars->q_empty);
         if (any16) {
           tc_commit(&bars->q16_empty);
@@ -575,9 +631,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2_4 = q_ts * k_ts * p.tau * kLog2e;
     const float sl2_16 = p.tau * kLog2e;
     const float pv4_scale = v_ts * (1.0f / 2688.0f);
-    uint32_t g = 0;
+    uint32_t g = 0, unit_ctr = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_ctr) {
       UnitInfo ui = decode_unit(p, u);
       const int row = ui.t * kBQ + rr;
       const int half = (p.bq == 64) ? (rr >> 6) : 0;
@@ -635,9 +691,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
 
-      EntryIter it = make_iter<BK>(p, ui);
-      int j, f16, rm;
-      while (it.next(j, f16, rm)) {
+      const uint32_t lb = unit_ctr & 1;
+      const uint16_t* list = reinterpret_cast<const uint16_t*>(smem + L::OFF_LIST) + lb * L::MAXE;
+      if (!(ok = mbar_wait(&bars->list_full[lb], (unit_ctr >> 1) & 1, abort_flag, p.status, lim))) break;
+      const int n_entries = bars->list_count[lb];
+      for (int e = 0; e < n_entries; ++e) {
+        const uint32_t x = list[e];
+        const int j = x & 0x1fff, f16 = (x >> 13) & 1, rm = x >> 14;
         const uint32_t buf = g & 1;
         if (!(ok = mbar_wait(&bars->s_full[buf], (g >> 1) & 1, abort_flag, p.status, lim))) break;
         tc_fence_after();
@@ -734,6 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok && have_pend) ok = merge(g - 1);
       if (!ok) break;
+      mbar_arrive(&bars->list_empty[lb]);
       // combine the two halves' partial denominators
       bars->lpart[hh][rr] = l_run;
       asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
@@ -876,6 +937,7 @@ thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const
   prm.mask_words = (prm.nkb + 31) / 32;
   prm.n_units = c.B * c.Hq * (c.N / kBQ);
   prm.tau = c.softmax_scale > 0.0f ? c.softmax_scale : 1.0f / sqrtf((float)c.d);
+  if (2 * prm.nkb > 4096) return THRIFT_ERR_UNSUPPORTED;  // the per-unit entry list holds 4096 entries
   prm.wait_limit = kWaitLimit;
   if (c.d == 128 && c.block_k == 64) return launch_t<128, 64>(q, k, v, q4, k4, v4, prm, stream);
   if (c.d == 128 && c.block_k == 128) return launch_t<128, 128>(q, k, v, q4, k4, v4, prm, stream);
