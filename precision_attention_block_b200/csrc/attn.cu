@@ -81,8 +81,8 @@ struct Bars {
   int list_count[2];
   uint32_t tmem_base;
   int abort_flag;
-  float lpart[2][128];      // per-row partial softmax denominators of the two key halves
-  float mswap[2][2][128];   // per-entry half-row maxima swapped between the two warps of a row
+  uint64_t pair[4];         // the two softmax warps of each TMEM lane quarter exchange values
+  float xch[2][2][128];     // exchange buffers of the lane-quarter warp pairs: [parity][half][row]
 };
 
 struct AttnParams {
@@ -369,6 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->pv_full, 1);
     mbar_init(&bars->pv_free, kSoftmaxThreads);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars->pair[i], 64);
     for (int i = 0; i < L::NSLOT; ++i) {
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
@@ -631,8 +632,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2_4 = q_ts * k_ts * p.tau * kLog2e;
     const float sl2_16 = p.tau * kLog2e;
     const float pv4_scale = v_ts * (1.0f / 2688.0f);
-    uint32_t g = 0, unit_ctr = 0;
+    uint32_t g = 0, unit_ctr = 0, xk = 0;
     bool ok = true;
+    // value of the partner warp of this lane quarter (bounded wait; `ok` drops on timeout)
+    auto exchange = [&](float v) -> float {
+      const uint32_t par = xk & 1;
+      bars->xch[par][hh][rr] = v;
+      mbar_arrive(&bars->pair[quarter]);
+      const bool got = mbar_wait(&bars->pair[quarter], par, abort_flag, p.status, lim);
+      ++xk;
+      if (!got) {
+        ok = false;
+        return v;
+      }
+      return bars->xch[par][1 - hh][rr];
+    };
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_ctr) {
       UnitInfo ui = decode_unit(p, u);
       const int row = ui.t * kBQ + rr;
@@ -733,9 +747,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q = 0; q < KH / 16; ++q) Mh = fmaxf(Mh, gmax[q]);
         // the block maximum over both halves: swap half maxima with the partner warp of this lane
         // quarter through shared memory (two buffers, alternating per entry)
-        bars->mswap[buf][hh][rr] = Mh;
-        asm volatile("bar.sync %0, 64;" ::"r"(2 + quarter) : "memory");
-        const float M = fmaxf(Mh, bars->mswap[buf][1 - hh][rr]);
+        const float M = fmaxf(Mh, exchange(Mh));
+        if (!ok) break;
         const bool valid = M != kNegInf;  // false when every key of the block is masked for this row
         const float Ms = valid ? M * sl2 : 0.0f;
 
@@ -796,10 +809,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       mbar_arrive(&bars->list_empty[lb]);
       // combine the two halves' partial denominators
-      bars->lpart[hh][rr] = l_run;
-      asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
-      const float l_tot = l_run + bars->lpart[1 - hh][rr];
-      asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
+      const float l_tot = l_run + exchange(l_run);
+      if (!ok) break;
       // epilogue: O / l in FP16, lse in natural-log units of the tau-scaled scores
       const float inv_l = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
       const int64_t orow = (int64_t)(ui.b * p.Hq + ui.h) * p.N + row;
