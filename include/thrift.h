@@ -111,6 +111,23 @@ thrift_status thrift_block_select(const void* q, const void* k, const thrift_cfg
                                   uint32_t* mask, int32_t* counts, int16_t* lists,
                                   double* scores, void* ws, size_t ws_bytes, void* stream);
 
+/* Block selection without any allocation, for callers that cannot allocate device memory:
+ * hosts that own every byte of device memory through their own allocator and hand the library
+ * only input and output buffers, or latency-bound callers that must not allocate (or grow a
+ * workspace) while a request is in flight.  The paper has no counterpart of this entry point.
+ * Same inputs, outputs and results as thrift_block_select, but the scratch (block means and the
+ * score matrix) lives in a fixed device array inside the library: 16 MiB, held by every GPU that
+ * loads the library until the process exits.  A configuration whose thrift_workspace_bytes()
+ * exceeds 16 MiB + 256 needs more scratch than that and is rejected with THRIFT_ERR_WORKSPACE
+ * before anything is launched.  The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before any stream
+ * capture.  It calls no cudaMalloc or cudaFree and no allocating library routine.  All calls
+ * share the one array and the scratch contents of a call are overwritten by the next; calls
+ * that overlap on the GPU (different streams, different host threads) race on it. */
+thrift_status thrift_block_select_noalloc(const void* q, const void* k, const thrift_cfg* cfg,
+                                          uint32_t* mask, int32_t* counts, int16_t* lists,
+                                          double* scores, void* stream);
+
 /* Attention forward (ThriftAttention "Gemengd-Precisie Berekening & Samenvoeging").
  * q, k, v: device FP16 [B,Hq,N,d], [B,Hkv,N,d], [B,Hkv,N,d] (used for the FP16 pairs);
  * q4, k4 (group_axis 0) and v4 (group_axis 1): NVFP4 copies (used for the other pairs);

@@ -57,6 +57,7 @@ SIGNATURES = {
     "thrift_auto_workspace_bytes": (_sz, [_cfgp]),
     "thrift_quantize_nvfp4": (ctypes.c_int, [_vp, _i64, _i32, _i32, _nvp, _vp, _sz, _vp]),
     "thrift_block_select": (ctypes.c_int, [_vp, _vp, _cfgp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "thrift_block_select_noalloc": (ctypes.c_int, [_vp, _vp, _cfgp, _vp, _vp, _vp, _vp, _vp]),
     "thrift_attn_fwd": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _nvp, _vp, _vp, _vp, _vp, _vp, _cfgp,
                                        _vp, _sz, _vp]),
     "thrift_attn_fwd_auto": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _cfgp, _vp, _sz, _vp]),

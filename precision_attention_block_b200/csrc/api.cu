@@ -146,6 +146,17 @@ thrift_status thrift_block_select(const void* q, const void* k, const thrift_cfg
                        static_cast<cudaStream_t>(stream));
 }
 
+thrift_status thrift_block_select_noalloc(const void* q, const void* k, const thrift_cfg* cfg, uint32_t* mask,
+                                          int32_t* counts, int16_t* lists, double* scores, void* stream) {
+  thrift_status st = cfg_supported(cfg);
+  if (st != THRIFT_OK) return st;
+  if (!q || !k || !mask || !counts || !lists) return THRIFT_ERR_INVALID_ARG;
+  if (select_layout(*cfg).bytes > noalloc_select_scratch_bytes()) return THRIFT_ERR_WORKSPACE;
+  uint8_t* scratch = nullptr;
+  if ((st = noalloc_select_scratch(&scratch)) != THRIFT_OK) return st;
+  return select_launch(q, k, *cfg, mask, counts, lists, scores, scratch, static_cast<cudaStream_t>(stream));
+}
+
 static thrift_status attn_common(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
                                  const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, void* out,
                                  float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes, float* dbg,

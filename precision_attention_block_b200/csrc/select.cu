@@ -12,10 +12,18 @@
 //   lists   one thread per query block walks its mask words in ascending order.
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "sm100.cuh"
 #include "thrift_internal.h"
 
 namespace thrift {
+
+// Fixed device scratch for thrift_block_select_noalloc.  Every GPU that loads the library holds
+// these kNoAllocSelectScratchBytes until the process exits; all calls of that entry point share
+// it, so calls that overlap on the GPU race on it.
+constexpr size_t kNoAllocSelectScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) uint8_t g_select_scratch[kNoAllocSelectScratchBytes];
 
 namespace {
 
@@ -204,6 +212,26 @@ SelectLayout select_layout(const thrift_cfg& c) {
   L.scores_off = align256(L.kbar_off + (size_t)c.B * c.Hkv * nkb * c.d * sizeof(double));
   L.bytes = align256(L.scores_off + (size_t)c.B * c.Hq * nqb * nkb * sizeof(double));
   return L;
+}
+
+size_t noalloc_select_scratch_bytes() { return kNoAllocSelectScratchBytes; }
+
+// Device address of g_select_scratch on the current device.  In host code the array's name is
+// only a host-side stand-in, so the address comes from cudaGetSymbolAddress, looked up once per
+// device (with that device current) and cached.
+thrift_status noalloc_select_scratch(uint8_t** out) {
+  static std::mutex mu;
+  static void* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return THRIFT_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_select_scratch) != cudaSuccess || !ptr) return THRIFT_ERR_CUDA;
+    cache[dev] = ptr;
+  }
+  *out = static_cast<uint8_t*>(cache[dev]);
+  return THRIFT_OK;
 }
 
 thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, uint32_t* mask, int32_t* counts,

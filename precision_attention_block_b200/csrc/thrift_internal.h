@@ -31,6 +31,9 @@ thrift_status quantize_launch(const void* x, int64_t outer, int32_t N, int32_t d
 thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, uint32_t* mask, int32_t* counts,
                             int16_t* lists, double* scores_out, uint8_t* scratch, cudaStream_t stream);
 
+size_t noalloc_select_scratch_bytes();
+thrift_status noalloc_select_scratch(uint8_t** out);
+
 // mode: 0 = FP16 pairs from the mask, 1 = every pair NVFP4, 2 = every pair FP16.
 thrift_status attn_launch(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
                           const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
