@@ -15,7 +15,7 @@
  * defined on FP32 values and is evaluated with IEEE FP32 operations here;
  * the build uses -ffp-contract=off so no product is fused).
  *
- * Readings of points the pages leave open (each also listed in the design doc):
+ * Readings of points the pages leave open:
  *   R-amax   one FP32 tensor scale per tensor: s_t = amax|X| / 2688 (2688 =
  *            6 * 448 maps the largest element onto the largest NVFP4 value);
  *            s_t = 1 when the tensor is all zero.
