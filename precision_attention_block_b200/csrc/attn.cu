@@ -27,8 +27,9 @@ namespace thrift {
 
 namespace {
 
-constexpr int kThreads = 320;  // warp 0 producer, warp 1 MMA, warps 2-9 softmax (two per TMEM lane quarter)
-constexpr int kSoftmaxThreads = 256;
+constexpr int kThreads = 608;  // warp 0 producer, 1 QK^T issuer, 2 PV issuer, 3-18 softmax (four per TMEM lane quarter)
+constexpr int kSoftmaxThreads = 512;
+constexpr int kFirstSoftmaxWarp = 3;
 constexpr int kBQ = 128;
 constexpr long long kWaitLimit = 1ll << 32;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -57,7 +58,7 @@ struct Layout {
   static constexpr int MAXE = 4096;  // entries per unit (two phases of at most 2048 key blocks)
   static constexpr int OFF_LIST = OFF_P + 2 * PBUF_BYTES;
   static constexpr int OFF_BAR = OFF_LIST + 2 * MAXE * 2;
-  static constexpr int BYTES = OFF_BAR + 4096 + 1024;  // barriers + alignment slack
+  static constexpr int BYTES = OFF_BAR + 6144 + 1024;  // barriers + alignment slack
   // TMEM columns
   static constexpr int COL_S = 0;  // two buffers of BK columns
   static constexpr int COL_PV = 2 * BK;
@@ -81,9 +82,11 @@ struct Bars {
   int list_count[2];
   uint32_t tmem_base;
   int abort_flag;
-  uint64_t pair[4];         // the two softmax warps of each TMEM lane quarter exchange values
-  float xch[2][2][128];     // exchange buffers of the lane-quarter warp pairs: [parity][half][row]
+  uint64_t pair[4];         // the four softmax warps of each TMEM lane quarter exchange values
+  float xch[2][4][128];     // exchange buffers of the four warps of each lane quarter: [parity][warp][row]
 };
+
+static_assert(sizeof(Bars) <= 6144, "barrier block");
 
 struct AttnParams {
   const uint32_t* mask;
@@ -219,26 +222,6 @@ __device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t a) {
 constexpr float kNegInf = -__builtin_huge_valf();
 constexpr float kRescale = 8.0f;  // log2 units: rescale O only when the block max grows past 256x
 
-__device__ __forceinline__ void load_s64(uint32_t taddr, float (&s)[64]) {
-  uint32_t r0[32], r1[32];
-  tmem_ld32(taddr, r0);
-  tmem_ld32(taddr + 32, r1);
-  tmem_wait_ld();
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    s[i] = __uint_as_float(r0[i]);
-    s[32 + i] = __uint_as_float(r1[i]);
-  }
-}
-
-__device__ __forceinline__ void load_s32(uint32_t taddr, float (&s)[32]) {
-  uint32_t r0[32];
-  tmem_ld32(taddr, r0);
-  tmem_wait_ld();
-#pragma unroll
-  for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(r0[i]);
-}
-
 // Rows that do not take part in this block, and keys above the query (causal), become -inf.
 template <int n>
 __device__ __forceinline__ void mask_s(float (&s)[n], bool part, bool diag, int key0, int row) {
@@ -268,18 +251,36 @@ __device__ __forceinline__ void group_max(const float (&s)[n], float* gm) {
   }
 }
 
-// FP16 probabilities of 32 keys: exp2(s * sl2 - Ms) rounded to FP16 pairs; returns their FP32 sum.
-__device__ __forceinline__ float probs_fp16_32(const float (&s)[32], float sl2, float Ms, uint32_t (&hw)[16]) {
+// N consecutive 32-bit TMEM columns of this thread's lane (N = 16 or 32).
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]);
+template <>
+__device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, uint32_t (&r)[32]) {
+  tmem_ld32(taddr, r);
+}
+template <>
+__device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// FP16 probabilities of N keys: exp2(s * sl2 - Ms) rounded to FP16 pairs; returns their FP32 sum.
+template <int N>
+__device__ __forceinline__ float probs_fp16(const float (&s)[N], float sl2, float Ms, uint32_t (&hw)[N / 2]) {
   const float2 a2 = make_float2(sl2, sl2), b2 = make_float2(-Ms, -Ms);
-  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-  for (int i = 0; i < 32; i += 2) {
+  for (int i = 0; i < N; i += 2) {
     float2 x = __ffma2_rn(make_float2(s[i], s[i + 1]), a2, b2);
     float2 pr = make_float2(ex2(x.x), ex2(x.y));
-    acc[(i >> 1) & 3] = __fadd2_rn(acc[(i >> 1) & 3], pr);
+    acc[(i >> 1) & 1] = __fadd2_rn(acc[(i >> 1) & 1], pr);
     hw[i >> 1] = pack_half2(pr.x, pr.y);
   }
-  float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  float2 t = __fadd2_rn(acc[0], acc[1]);
   return t.x + t.y;
 }
 
@@ -297,18 +298,19 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float* y) {
   return out;
 }
 
-// NVFP4 re-quantisation of 32 keys (two 16-key groups) of one row:
+// NVFP4 re-quantisation of NG 16-key groups of one row:
 //   P^ = exp2(s*sl2 - Ms); per group s_b = E4M3(2688 max(P^) / 6); codes = E2M1(2688 P^ / s_b).
 // 2688 / s_b is folded into the exponent, so each key costs one FMA and one exp2.  A group whose
 // scale underflows to 0 gets all-zero codes (its values are below 2688 * 2^-10 / 6 / 448).
-// Returns the FP32 sum of the unquantised P^; writes 4 code words and 2 scale bytes into sfw at
-// bit offset `shift`.
-__device__ __forceinline__ float probs_nvfp4_32(const float (&s)[32], const float* gm, float sl2, float Ms,
-                                                uint32_t (&cw)[4], uint32_t& sfw, int shift) {
+// Returns the FP32 sum of the unquantised P^; writes 2*NG code words and NG scale bytes (sfw).
+template <int NG>
+__device__ __forceinline__ float probs_nvfp4(const float (&s)[16 * NG], const float* gm, float sl2, float Ms,
+                                             uint32_t (&cw)[2 * NG], uint32_t& sfw) {
   float sum = 0.0f;
+  sfw = 0u;
   const float2 a2 = make_float2(sl2, sl2);
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {
+  for (int q = 0; q < NG; ++q) {
     const bool live = gm[q] != kNegInf;
     const float pmax = live ? 2688.0f * ex2(fmaf(gm[q], sl2, -Ms)) : 0.0f;
     const uint32_t sb = cvt_e4m3(pmax * (1.0f / 6.0f));
@@ -332,7 +334,7 @@ __device__ __forceinline__ float probs_nvfp4_32(const float (&s)[32], const floa
     cw[2 * q + 1] = cvt_e2m1x8(y + 8);
     const float2 t2 = __fadd2_rn(acc0, acc1);
     sum = fmaf(t2.x + t2.y, sbe * (1.0f / 2688.0f), sum);
-    sfw |= sb << (shift + 8 * q);
+    sfw |= sb << (8 * q);
   }
   return sum;
 }
@@ -369,14 +371,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->pv_full, 1);
     mbar_init(&bars->pv_free, kSoftmaxThreads);
-    for (int i = 0; i < 4; ++i) mbar_init(&bars->pair[i], 64);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars->pair[i], 128);
     for (int i = 0; i < L::NSLOT; ++i) {
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->list_full[i], 1);
-      mbar_init(&bars->list_empty[i], 1 + kSoftmaxThreads);
+      mbar_init(&bars->list_empty[i], 2 + kSoftmaxThreads);
     }
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -491,54 +493,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------------ QK^T issuer
     if (lane == 0) {
       const uint32_t idesc_qk4 = idesc_nvf4(kBQ, BK);
-      const uint32_t idesc_pv4 = idesc_nvf4(kBQ, D);
       const uint32_t idesc_qk16 = idesc_f16(kBQ, BK, 0, 0);
-      const uint32_t idesc_pv16 = idesc_f16(kBQ, D, 0, 1);
       constexpr int SWQ = swz_for_row_bytes(D / 2);
-      constexpr int SWP = swz_for_row_bytes(BK / 2);
+      const uint32_t qb4 = smem_u32(sQ4), qb16 = smem_u32(sQ16);
       uint32_t slot_ctr = 0, unit_ctr = 0, u16_ctr = 0, g = 0;
       bool ok = true;
-      struct Pend {
-        uint32_t g, vslot, vph;
-        int f16, sfv_off;
-      } pend = {0, 0, 0, 0, 0};
-      auto do_pv = [&](const Pend& e) -> bool {
-        const uint32_t buf = e.g & 1;
-        if (!mbar_wait(&bars->p_full[buf], (e.g >> 1) & 1, abort_flag, p.status, lim)) return false;
-        if (!mbar_wait(&bars->pv_free, (e.g & 1) ^ 1, abort_flag, p.status, lim)) return false;
-        if (!mbar_wait(&bars->kv_full[e.vslot], e.vph, abort_flag, p.status, lim)) return false;
-        tc_fence_after();
-        const uint32_t pbuf = smem_u32(sP + buf * L::PBUF_BYTES);
-        const uint32_t vbuf = smem_u32(sSlots + e.vslot * L::SLOT_BYTES);
-        if (e.f16) {
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            uint64_t ad = make_sdesc(pbuf + (kk >> 2) * kBQ * 128 + (kk & 3) * 32, 16, 1024, kSW128);
-            uint64_t bd = make_sdesc(vbuf + kk * 16 * 128, BK * 128, 1024, kSW128);
-            mma_f16(tmem + L::COL_PV, ad, bd, idesc_pv16, kk > 0);
-          }
-        } else {
-          const uint32_t sfv = tmem + L::COL_SFV + buf * L::SFKV_COLS;
-          const uint32_t sfp = tmem + L::COL_SFP + buf * L::SFKV_COLS;
-#pragma unroll
-          for (int kb = 0; kb < BK / 64; ++kb) {
-            tc_copy_sf(sfv + 4 * kb, make_sdesc(vbuf + D * BK / 2 + kb * 512, 16, 128, 0));
-            tc_copy_sf(sfp + 4 * kb, make_sdesc(pbuf + L::P4_BYTES + kb * 512, 16, 128, 0));
-          }
-#pragma unroll
-          for (int kb = 0; kb < BK / 64; ++kb) {
-            uint64_t ad = make_sdesc(pbuf + kb * 32, 16, 8 * (BK / 2), SWP);
-            uint64_t bd = make_sdesc(vbuf + kb * 32, 16, 8 * (BK / 2), SWP);
-            mma_nvf4(tmem + L::COL_PV, ad, bd, idesc_pv4, sfp + 4 * kb, sfv + 4 * kb + e.sfv_off, kb > 0);
-          }
-        }
-        tc_commit(&bars->pv_full);
-        tc_commit(&bars->kv_empty[e.vslot]);
-        return true;
-      };
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_ctr) {
         UnitInfo ui = decode_unit(p, u);
         const int kvh = ui.b * p.Hkv + ui.hk;
@@ -549,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < D / 64; ++kk)
             tc_copy_sf(tmem + L::COL_SFQ + 4 * kk, make_sdesc(smem_u32(sQSF) + kk * 512, 16, 128, 0));
         }
-        bool any16 = false, have_pend = false;
+        bool any16 = false;
         const uint32_t lb = unit_ctr & 1;
         const uint16_t* list = reinterpret_cast<const uint16_t*>(smem + L::OFF_LIST) + lb * L::MAXE;
         if (!(ok = mbar_wait(&bars->list_full[lb], (unit_ctr >> 1) & 1, abort_flag, p.status, lim))) break;
@@ -557,10 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; ok && e < n_entries; ++e) {
           const uint32_t x = list[e];
           const int j = x & 0x1fff, f16 = (x >> 13) & 1;
-          uint32_t kslot = slot_ctr % L::NSLOT, kph = (slot_ctr / L::NSLOT) & 1;
-          ++slot_ctr;
-          uint32_t vslot = slot_ctr % L::NSLOT, vph = (slot_ctr / L::NSLOT) & 1;
-          ++slot_ctr;
+          const uint32_t kslot = slot_ctr % L::NSLOT, kph = (slot_ctr / L::NSLOT) & 1;
+          slot_ctr += 2;  // this entry's V tile takes the next slot (the PV issuer consumes it)
           if (f16 && !any16) {
             if (!(ok = mbar_wait(&bars->q16_full, u16_ctr & 1, abort_flag, p.status, lim))) break;
             any16 = true;
@@ -572,10 +532,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t kbuf = smem_u32(sSlots + kslot * L::SLOT_BYTES);
           const uint32_t dS = tmem + L::COL_S + buf * BK;
           if (f16) {
-            const uint32_t qb = smem_u32(sQ16);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              uint64_t ad = make_sdesc(qb + (kk >> 2) * kBQ * 128 + (kk & 3) * 32, 16, 1024, kSW128);
+              uint64_t ad = make_sdesc(qb16 + (kk >> 2) * kBQ * 128 + (kk & 3) * 32, 16, 1024, kSW128);
               uint64_t bd = make_sdesc(kbuf + (kk >> 2) * BK * 128 + (kk & 3) * 32, 16, 1024, kSW128);
               mma_f16(dS, ad, bd, idesc_qk16, kk > 0);
             }
@@ -586,26 +545,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < D / 64; ++kk)
               tc_copy_sf(sfk + 4 * kk, make_sdesc(kbuf + BK * D / 2 + kk * 512, 16, 128, 0));
-            const uint32_t qb = smem_u32(sQ4);
 #pragma unroll
             for (int kk = 0; kk < D / 64; ++kk) {
-              uint64_t ad = make_sdesc(qb + kk * 32, 16, 8 * (D / 2), SWQ);
+              uint64_t ad = make_sdesc(qb4 + kk * 32, 16, 8 * (D / 2), SWQ);
               uint64_t bd = make_sdesc(kbuf + kk * 32, 16, 8 * (D / 2), SWQ);
               mma_nvf4(dS, ad, bd, idesc_qk4, tmem + L::COL_SFQ + 4 * kk, sfk + 4 * kk + sfk_off, kk > 0);
             }
           }
           tc_commit(&bars->s_full[buf]);
           tc_commit(&bars->kv_empty[kslot]);
-          if (have_pend && !(ok = do_pv(pend))) break;
-          pend.g = g;
-          pend.vslot = vslot;
-          pend.vph = vph;
-          pend.f16 = f16;
-          pend.sfv_off = ((kvh * D) & 127) >> 5;
-          have_pend = true;
           ++g;
         }
-        if (ok && have_pend) ok = do_pv(pend);
         if (!ok) break;
         mbar_arrive(&bars->list_empty[lb]);
         tc_commit(&bars->q_empty);
@@ -615,17 +565,73 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------------ PV issuer
+    if (lane == 0) {
+      const uint32_t idesc_pv4 = idesc_nvf4(kBQ, D);
+      const uint32_t idesc_pv16 = idesc_f16(kBQ, D, 0, 1);
+      constexpr int SWP = swz_for_row_bytes(BK / 2);
+      uint32_t slot_ctr = 0, unit_ctr = 0, g = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_ctr) {
+        UnitInfo ui = decode_unit(p, u);
+        const int sfv_off = (((ui.b * p.Hkv + ui.hk) * D) & 127) >> 5;
+        const uint32_t lb = unit_ctr & 1;
+        const uint16_t* list = reinterpret_cast<const uint16_t*>(smem + L::OFF_LIST) + lb * L::MAXE;
+        if (!(ok = mbar_wait(&bars->list_full[lb], (unit_ctr >> 1) & 1, abort_flag, p.status, lim))) break;
+        const int n_entries = bars->list_count[lb];
+        for (int e = 0; ok && e < n_entries; ++e) {
+          const int f16 = (list[e] >> 13) & 1;
+          const uint32_t vslot = (slot_ctr + 1) % L::NSLOT, vph = ((slot_ctr + 1) / L::NSLOT) & 1;
+          slot_ctr += 2;
+          const uint32_t buf = g & 1;
+          if (!(ok = mbar_wait(&bars->p_full[buf], (g >> 1) & 1, abort_flag, p.status, lim))) break;
+          if (!(ok = mbar_wait(&bars->pv_free, (g & 1) ^ 1, abort_flag, p.status, lim))) break;
+          if (!(ok = mbar_wait(&bars->kv_full[vslot], vph, abort_flag, p.status, lim))) break;
+          tc_fence_after();
+          const uint32_t pbuf = smem_u32(sP + buf * L::PBUF_BYTES);
+          const uint32_t vbuf = smem_u32(sSlots + vslot * L::SLOT_BYTES);
+          if (f16) {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              uint64_t ad = make_sdesc(pbuf + (kk >> 2) * kBQ * 128 + (kk & 3) * 32, 16, 1024, kSW128);
+              uint64_t bd = make_sdesc(vbuf + kk * 16 * 128, BK * 128, 1024, kSW128);
+              mma_f16(tmem + L::COL_PV, ad, bd, idesc_pv16, kk > 0);
+            }
+          } else {
+            const uint32_t sfv = tmem + L::COL_SFV + buf * L::SFKV_COLS;
+            const uint32_t sfp = tmem + L::COL_SFP + buf * L::SFKV_COLS;
+#pragma unroll
+            for (int kb = 0; kb < BK / 64; ++kb) {
+              tc_copy_sf(sfv + 4 * kb, make_sdesc(vbuf + D * BK / 2 + kb * 512, 16, 128, 0));
+              tc_copy_sf(sfp + 4 * kb, make_sdesc(pbuf + L::P4_BYTES + kb * 512, 16, 128, 0));
+            }
+#pragma unroll
+            for (int kb = 0; kb < BK / 64; ++kb) {
+              uint64_t ad = make_sdesc(pbuf + kb * 32, 16, 8 * (BK / 2), SWP);
+              uint64_t bd = make_sdesc(vbuf + kb * 32, 16, 8 * (BK / 2), SWP);
+              mma_nvf4(tmem + L::COL_PV, ad, bd, idesc_pv4, sfp + 4 * kb, sfv + 4 * kb + sfv_off, kb > 0);
+            }
+          }
+          tc_commit(&bars->pv_full);
+          tc_commit(&bars->kv_empty[vslot]);
+          ++g;
+        }
+        if (!ok) break;
+        mbar_arrive(&bars->list_empty[lb]);
+      }
+    }
   } else {
     // ------------------------------------------------------------------ softmax / merge
-    // Two warps share each TMEM lane quarter (the same 32 rows): both read the whole score row
-    // and find the same block and group maxima; warp half `hh` then produces the probabilities
-    // of keys [hh*BK/2, (hh+1)*BK/2) and accumulates output columns [hh*D/2, (hh+1)*D/2).
-    const int sw = warp - 2;
+    // Four warps share each TMEM lane quarter (the same 32 query rows).  Warp `kq` of the quarter
+    // reads keys [kq*BK/4, (kq+1)*BK/4) of the score row, the four swap their maxima to get the
+    // row maximum M of the key block, and each produces its keys' probabilities and accumulates
+    // output columns [kq*D/4, (kq+1)*D/4).
     const int quarter = warp & 3;
-    const int hh = sw >> 2;
+    const int kq = (warp - kFirstSoftmaxWarp) >> 2;
     const int rr = quarter * 32 + lane;  // row of the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    constexpr int DH = D / 2, KH = BK / 2;
+    constexpr int DW = D / 4, KW = BK / 4;
     const float q_ts = (p.mode != 2) ? __ldg(p.q_ts) : 1.0f;
     const float k_ts = (p.mode != 2) ? __ldg(p.k_ts) : 1.0f;
     const float v_ts = (p.mode != 2) ? __ldg(p.v_ts) : 1.0f;
@@ -634,10 +640,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float pv4_scale = v_ts * (1.0f / 2688.0f);
     uint32_t g = 0, unit_ctr = 0, xk = 0;
     bool ok = true;
-    // value of the partner warp of this lane quarter (bounded wait; `ok` drops on timeout)
-    auto exchange = [&](float v) -> float {
+    // combine a value over the four warps of this lane quarter (max or sum; bounded wait)
+    auto exchange = [&](float v, bool take_max) -> float {
       const uint32_t par = xk & 1;
-      bars->xch[par][hh][rr] = v;
+      bars->xch[par][kq][rr] = v;
       mbar_arrive(&bars->pair[quarter]);
       const bool got = mbar_wait(&bars->pair[quarter], par, abort_flag, p.status, lim);
       ++xk;
@@ -645,15 +651,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
         return v;
       }
-      return bars->xch[par][1 - hh][rr];
+      const float a = bars->xch[par][0][rr], b = bars->xch[par][1][rr];
+      const float c = bars->xch[par][2][rr], d = bars->xch[par][3][rr];
+      return take_max ? max3(a, b, fmaxf(c, d)) : (a + b) + (c + d);
     };
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_ctr) {
       UnitInfo ui = decode_unit(p, u);
       const int row = ui.t * kBQ + rr;
       const int half = (p.bq == 64) ? (rr >> 6) : 0;
-      float O[DH];
+      float O[DW];
 #pragma unroll
-      for (int c = 0; c < DH; ++c) O[c] = 0.0f;
+      for (int c = 0; c < DW; ++c) O[c] = 0.0f;
       // running state: O and l are relative to exp2(m_ref); m_ref moves only when a block's
       // maximum exceeds it by more than 2^kRescale (the final O / l does not depend on m_ref)
       float m_ref = kNegInf, l_run = 0.0f;
@@ -672,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 a2 = make_float2(alpha, alpha);
           l_run *= alpha;
 #pragma unroll
-          for (int c = 0; c < DH; c += 2) {
+          for (int c = 0; c < DW; c += 2) {
             float2 o = __fmul2_rn(make_float2(O[c], O[c + 1]), a2);
             O[c] = o.x;
             O[c + 1] = o.y;
@@ -683,25 +691,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run = fmaf(gs, pend_sum, l_run);
         const float gpv = pend_f16 ? gs : gs * pv4_scale;
         const float2 g2 = make_float2(gpv, gpv);
-        uint32_t r[DH];
-        const uint32_t pva = tmem + lane_base + L::COL_PV + hh * DH;
-        tmem_ld32(pva, *reinterpret_cast<uint32_t(*)[32]>(r));
-        if constexpr (DH == 64) tmem_ld32(pva + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+        uint32_t r[DW];
+        tmem_ld<DW>(tmem + lane_base + L::COL_PV + kq * DW, r);
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->pv_free);
 #pragma unroll
-        for (int i = 0; i < DH; i += 2) {
+        for (int i = 0; i < DW; i += 2) {
           float2 o = __ffma2_rn(g2, make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])),
                                 make_float2(O[i], O[i + 1]));
           O[i] = o.x;
           O[i + 1] = o.y;
         }
         if constexpr (DBG) {
-          if (dbg_unit && (local_e - 1) == p.dbg_entry) {
-            for (int i = 0; i < DH; ++i) p.dbg[kBQ * BK + kBQ * (BK / 2) + rr * D + hh * DH + i] = __uint_as_float(r[i]);
-          }
+          if (dbg_unit && (local_e - 1) == p.dbg_entry)
+            for (int i = 0; i < DW; ++i) p.dbg[kBQ * BK + kBQ * (BK / 2) + rr * D + kq * DW + i] = __uint_as_float(r[i]);
         }
-        tc_fence_before();
-        mbar_arrive(&bars->pv_free);
         return true;
       };
 
@@ -717,81 +722,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const bool part = (rm >> half) & 1;
         const bool diag = p.causal && (j * BK + BK - 1 > ui.t * kBQ);
-        const int key0 = j * BK;
-        const uint32_t saddr = tmem + lane_base + L::COL_S + buf * BK;
+        const int key0 = j * BK + kq * KW;  // first key of this warp's columns
         const float sl2 = f16 ? sl2_16 : sl2_4;
         const bool dumpP = dbg_unit && local_e == p.dbg_entry;
         const uint32_t pb = smem_u32(sP + buf * L::PBUF_BYTES);
 
-        // this warp's keys [hh*BK/2, (hh+1)*BK/2) of the score row: one TMEM round trip, then the
-        // scores live in registers and the buffer goes back to the MMA warp
-        float sv[KH];
-#pragma unroll
-        for (int c2 = 0; c2 < KH / 32; ++c2) tmem_ld32(saddr + KH * hh + 32 * c2, *reinterpret_cast<uint32_t(*)[32]>(sv + 32 * c2));
+        // this warp's KW scores of the row: one TMEM round trip, then the buffer goes back
+        float sv[KW];
+        tmem_ld<KW>(tmem + lane_base + L::COL_S + buf * BK + kq * KW, *reinterpret_cast<uint32_t(*)[KW]>(sv));
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&bars->s_free[buf]);
         if constexpr (DBG) {
           if (dumpP)
-            for (int i = 0; i < KH; ++i) p.dbg[rr * BK + KH * hh + i] = sv[i];
+            for (int i = 0; i < KW; ++i) p.dbg[rr * BK + kq * KW + i] = sv[i];
         }
-        float gmax[KH / 16];
+        mask_s(sv, part, diag, key0, row);
+        float gmax[KW / 16];
+        group_max<KW>(sv, gmax);
+        float Mh = gmax[0];
 #pragma unroll
-        for (int c2 = 0; c2 < KH / 32; ++c2) {
-          float* s32 = sv + 32 * c2;
-          mask_s(*reinterpret_cast<float(*)[32]>(s32), part, diag, key0 + KH * hh + 32 * c2, row);
-          group_max<32>(*reinterpret_cast<float(*)[32]>(s32), gmax + 2 * c2);
-        }
-        float Mh = kNegInf;
-#pragma unroll
-        for (int q = 0; q < KH / 16; ++q) Mh = fmaxf(Mh, gmax[q]);
-        // the block maximum over both halves: swap half maxima with the partner warp of this lane
-        // quarter through shared memory (two buffers, alternating per entry)
-        const float M = fmaxf(Mh, exchange(Mh));
+        for (int q = 1; q < KW / 16; ++q) Mh = fmaxf(Mh, gmax[q]);
+        const float M = exchange(Mh, true);  // the block maximum over the four warps
         if (!ok) break;
-        const bool valid = M != kNegInf;  // false when every key of the block is masked for this row
+        const bool valid = M != kNegInf;     // false when every key of the block is masked for this row
         const float Ms = valid ? M * sl2 : 0.0f;
 
-        // probabilities of this warp's keys relative to the block maximum, their partial sum, and
-        // this warp's part of the PV operand in shared memory
-        float sum = 0.0f;
+        // this warp's probabilities, their partial sum, and its part of the PV operand
+        float sum;
+        if (f16) {
+          uint32_t hw[KW / 2];
+          sum = probs_fp16<KW>(sv, sl2, Ms, hw);
+          if constexpr (DBG) {
+            if (dumpP)
+              for (int i = 0; i < KW / 2; ++i) reinterpret_cast<uint32_t*>(p.dbg + kBQ * BK + rr * (BK / 2))[kq * (KW / 2) + i] = hw[i];
+          }
 #pragma unroll
-        for (int c2 = 0; c2 < KH / 32; ++c2) {
-          const int c = hh * (KH / 32) + c2;  // 32-key chunk index within the row
-          float(&s32)[32] = *reinterpret_cast<float(*)[32]>(sv + 32 * c2);
-          if (f16) {
-            uint32_t hw[16];
-            sum += probs_fp16_32(s32, sl2, Ms, hw);
-            if constexpr (DBG) {
-              if (dumpP)
-                for (int i = 0; i < 16; ++i) reinterpret_cast<uint32_t*>(p.dbg + kBQ * BK + rr * (BK / 2))[16 * c + i] = hw[i];
+          for (int q = 0; q < KW / 8; ++q) {
+            const int chunk = kq * (KW / 8) + q;  // 16-byte chunk of the row (8 keys)
+            const int cb = chunk >> 3, c8 = chunk & 7;
+            st_shared_v4(pb + cb * kBQ * 128 + rr * 128 + ((c8 ^ (rr & 7)) << 4), hw[4 * q], hw[4 * q + 1],
+                         hw[4 * q + 2], hw[4 * q + 3]);
+          }
+        } else {
+          uint32_t cw[KW / 8], sfw = 0u;
+          sum = probs_nvfp4<KW / 16>(sv, gmax, sl2, Ms, cw, sfw);
+          if constexpr (DBG) {
+            if (dumpP) {
+              uint8_t* db = reinterpret_cast<uint8_t*>(p.dbg + kBQ * BK + rr * (BK / 2));
+              for (int i = 0; i < KW / 8; ++i) reinterpret_cast<uint32_t*>(db + kq * (KW / 2))[i] = cw[i];
+              for (int q = 0; q < KW / 16; ++q) db[BK / 2 + kq * (KW / 16) + q] = (uint8_t)(sfw >> (8 * q));
             }
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int chunk = 4 * c + q;  // 16-byte chunk of the row (8 keys)
-              const int cb = chunk >> 3, c8 = chunk & 7;
-              st_shared_v4(pb + cb * kBQ * 128 + rr * 128 + ((c8 ^ (rr & 7)) << 4), hw[4 * q], hw[4 * q + 1],
-                           hw[4 * q + 2], hw[4 * q + 3]);
-            }
+          }
+          if constexpr (BK == 64) {
+            // 8 code bytes: half of the row's 16-byte chunk kq/2
+            const uint32_t addr = pb + rr * 32 + (((kq >> 1) ^ ((rr >> 2) & 1)) << 4) + 8 * (kq & 1);
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(cw[0]), "r"(cw[1]) : "memory");
+            const uint32_t sfa = pb + L::P4_BYTES + (rr & 31) * 16 + (rr >> 5) * 4 + kq;
+            asm volatile("st.shared.b8 [%0], %1;" ::"r"(sfa), "r"(sfw) : "memory");
           } else {
-            uint32_t cw[4], sfw = 0u;
-            sum += probs_nvfp4_32(s32, gmax + 2 * c2, sl2, Ms, cw, sfw, 0);
-            if constexpr (DBG) {
-              if (dumpP) {
-                uint8_t* db = reinterpret_cast<uint8_t*>(p.dbg + kBQ * BK + rr * (BK / 2));
-                for (int i = 0; i < 4; ++i) reinterpret_cast<uint32_t*>(db + 16 * c)[i] = cw[i];
-                db[BK / 2 + 2 * c] = (uint8_t)(sfw & 255u);
-                db[BK / 2 + 2 * c + 1] = (uint8_t)(sfw >> 8);
-              }
-            }
-            uint32_t addr;
-            if (BK == 64)
-              addr = pb + rr * 32 + ((c ^ ((rr >> 2) & 1)) << 4);
-            else
-              addr = pb + rr * 64 + ((c ^ ((rr >> 1) & 3)) << 4);
+            const uint32_t addr = pb + rr * 64 + ((kq ^ ((rr >> 1) & 3)) << 4);
             st_shared_v4(addr, cw[0], cw[1], cw[2], cw[3]);
-            // the two scale bytes of this chunk's 16-key groups
-            const uint32_t sfa = pb + L::P4_BYTES + (c >> 1) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + 2 * (c & 1);
+            const uint32_t sfa = pb + L::P4_BYTES + (kq >> 1) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + 2 * (kq & 1);
             asm volatile("st.shared.b16 [%0], %1;" ::"r"(sfa), "h"((uint16_t)sfw) : "memory");
           }
         }
@@ -808,15 +800,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && have_pend) ok = merge(g - 1);
       if (!ok) break;
       mbar_arrive(&bars->list_empty[lb]);
-      // combine the two halves' partial denominators
-      const float l_tot = l_run + exchange(l_run);
+      // combine the four warps' partial denominators
+      const float l_tot = exchange(l_run, false);
       if (!ok) break;
       // epilogue: O / l in FP16, lse in natural-log units of the tau-scaled scores
       const float inv_l = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
       const int64_t orow = (int64_t)(ui.b * p.Hq + ui.h) * p.N + row;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D + hh * DH);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D + kq * DW);
 #pragma unroll
-      for (int c = 0; c < DH / 8; ++c) {
+      for (int c = 0; c < DW / 8; ++c) {
         uint4 v;
         v.x = pack_half2(O[8 * c] * inv_l, O[8 * c + 1] * inv_l);
         v.y = pack_half2(O[8 * c + 2] * inv_l, O[8 * c + 3] * inv_l);
@@ -824,7 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         v.w = pack_half2(O[8 * c + 6] * inv_l, O[8 * c + 7] * inv_l);
         dst[c] = v;
       }
-      if (p.lse && hh == 0) p.lse[orow] = (m_ref + __log2f(l_tot)) * kLn2;
+      if (p.lse && kq == 0) p.lse[orow] = (m_ref + __log2f(l_tot)) * kLn2;
     }
   }
 
