@@ -1,21 +1,29 @@
 // Fused selective mixed-precision attention forward for sm_100a (ThriftAttention technical
 // summary, "Gemengd-Precisie Berekening & Samenvoeging" and the paragraph on its fused kernel).
 //
-// One persistent CTA per SM walks (batch, query head, 128-row query tile) units.  For each unit
-// the key blocks form a list of entries: first every key block that some row of the tile computes
-// in NVFP4, then every key block it computes in FP16 (the order the pages' kernel uses; the FP16
-// query tile is fetched only when the first FP16 entry comes up).  Warp roles:
-//   warp 0      TMA producer: the unit's NVFP4 query tile, the FP16 query tile on demand, and for
-//               every entry its K and V tiles (NVFP4 codes + scales, or FP16) into a slot ring.
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of two TMEM score buffers, then the
-//               previous entry's PV into the TMEM PV buffer.  NVFP4 products use
-//               tcgen05.mma.kind::mxf4nvf4.block_scale.block16 with the E4M3 scale vectors copied
-//               into TMEM by tcgen05.cp; FP16 products use tcgen05.mma.kind::f16.
-//   warps 2-5   one thread per query row: read S from TMEM, causal mask, the row maximum M of the
-//               key block, P^ = exp(S - M); NVFP4 entries re-quantise P' = 2688 P^ with one E4M3
-//               scale per 16 keys into shared memory (the PV MMA's A operand), FP16 entries round
-//               P^ to FP16; then merge the previous entry's PV into the row's FP32 output with
-//               weight exp(M - m) (m = running maximum), and sum the unquantised P^ into l.
+// One persistent CTA per SM walks (batch, query head, 128-row query tile) units, heaviest causal
+// tiles first.  For each unit the key blocks form a list of entries: first every key block that
+// some row of the tile computes in NVFP4, then every key block it computes in FP16 (the order the
+// pages' kernel uses; the FP16 query tile is fetched only when the first FP16 entry comes up).
+// Warp roles:
+//   warp 0      TMA producer: builds the unit's entry list, loads the NVFP4 query tile, the FP16
+//               query tile on demand, and for every entry its K and V tiles into a page ring (one
+//               page holds an NVFP4 entry's K and V, an FP16 entry takes two pages).
+//   warp 1      QK^T issuer: S = Q K^T of each entry into one of two TMEM score buffers;
+//               tcgen05.mma.kind::mxf4nvf4.block_scale.block16 for NVFP4 pairs (E4M3 scale
+//               vectors copied into TMEM by tcgen05.cp), kind::f16 for FP16 pairs.
+//   warp 2      PV issuer: the entry's probability block times V into a TMEM PV buffer.
+//   warps 4-11  two softmax warpgroups; a thread of warp w owns query row 32 (w % 4) + lane of the
+//               tile for one half of the keys and one half of the output columns.  Per entry both
+//               read the whole score row from TMEM (so each has the row maximum M of the key block
+//               without any exchange), compute P^ = exp(S - M) for their half of the keys: NVFP4
+//               entries re-quantise P' = 2688 P^ with one E4M3 scale per 16 keys into shared
+//               memory (the PV MMA's A operand), FP16 entries round P^ to FP16.  Then each folds
+//               the previous entry's PV into its half of the row's FP32 output (registers) with
+//               weight exp(M - m) and adds its half of the unquantised sum of P^ into the
+//               denominator.  Part of the exponentials run as a polynomial on the FMA pipe, the
+//               rest on the MUFU unit, so that neither pipe alone limits.
+// Registers move from the producer warpgroup to the softmax warpgroups with setmaxnreg.
 // Every wait is bounded; on timeout the CTA records THRIFT_ERR_TIMEOUT and unwinds.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -27,66 +35,81 @@ namespace thrift {
 
 namespace {
 
-constexpr int kThreads = 608;  // warp 0 producer, 1 QK^T issuer, 2 PV issuer, 3-18 softmax (four per TMEM lane quarter)
-constexpr int kSoftmaxThreads = 512;
-constexpr int kFirstSoftmaxWarp = 3;
 constexpr int kBQ = 128;
 constexpr long long kWaitLimit = 1ll << 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kSW128 = 2, kSW64 = 4, kSW32 = 6;
+constexpr int kMaxPages = 8;
+constexpr int kSmemLimit = 232448;  // largest dynamic shared memory of one CTA on sm_100
+constexpr int kProducerRegs = 56, kSoftmaxRegs = 224;  // setmaxnreg split (384 threads x 168 at launch)
+constexpr float kNegInf = -__builtin_huge_valf();
+constexpr float kRescale = 8.0f;  // log2 units: rescale O only when the block max grows past 256x
+constexpr int kPolyPerGroup = 4;  // exponentials per 16 keys evaluated by the polynomial
 
 __host__ __device__ constexpr int round1024(int x) { return (x + 1023) & ~1023; }
 __host__ __device__ constexpr int swz_for_row_bytes(int b) { return b == 128 ? kSW128 : (b == 64 ? kSW64 : kSW32); }
+__host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
 template <int D, int BK>
 struct Layout {
+  // TMEM columns: PV result buffers, two score buffers, scale vectors of Q, K (x2), V (x2), P (x2)
+  static constexpr int SFQ = 4 * (D / 64);
+  static constexpr int SFV = 4 * (BK / 64);
+  static constexpr int SF_COLS = 3 * SFQ + 4 * SFV;
+  static constexpr int NPV = 2 * D + 2 * BK + SF_COLS <= 512 ? 2 : 1;  // PV buffers
+  static constexpr int COL_PV = 0;
+  static constexpr int COL_S = NPV * D;
+  static constexpr int COL_SFQ = COL_S + 2 * BK;
+  static constexpr int COL_SFK = COL_SFQ + SFQ;
+  static constexpr int COL_SFV = COL_SFK + 2 * SFQ;
+  static constexpr int COL_SFP = COL_SFV + 2 * SFV;
+  static constexpr int TMEM_COLS = COL_SFP + 2 * SFV;
+  static_assert(TMEM_COLS <= 512, "TMEM budget");
+  static constexpr int THREADS = 384;
+  static constexpr int KH = BK / 2;  // keys of a row per softmax warpgroup
+  static constexpr int DH = D / 2;   // output columns of a row per softmax warpgroup
+
+  // shared memory: NVFP4 query tile + its scales, FP16 query tile, two PV operand buffers
   static constexpr int Q4_BYTES = kBQ * D / 2;
   static constexpr int QSF_BYTES = (D / 64) * 512;
+  static constexpr int Q4_REGION = round1024(Q4_BYTES + QSF_BYTES);
   static constexpr int Q16_BYTES = kBQ * D * 2;
-  static constexpr int SLOT_BYTES = BK * D * 2;
-  static constexpr int NSLOT = BK == 128 ? 3 : 6;
-  static constexpr int P16_BYTES = kBQ * BK * 2;
   static constexpr int P4_BYTES = kBQ * BK / 2;
   static constexpr int PSF_BYTES = (BK / 64) * 512;
-  static constexpr int PBUF_BYTES = round1024(P16_BYTES > P4_BYTES + PSF_BYTES ? P16_BYTES : P4_BYTES + PSF_BYTES);
+  static constexpr int P16_BYTES = kBQ * BK * 2;
+  static constexpr int PBUF = round1024(cmax(P16_BYTES, P4_BYTES + PSF_BYTES));
+  // one page: an NVFP4 entry (K codes, K scales, V codes, V scales) or one FP16 K or V tile
+  static constexpr int K16_BYTES = BK * D * 2;
+  static constexpr int K4_BYTES = BK * D / 2;
+  static constexpr int KSF_BYTES = (D / 64) * 512;  // the 128-row scale block(s) holding the tile's rows
+  static constexpr int V4_OFF = round1024(K4_BYTES + KSF_BYTES);
+  static constexpr int V4_BYTES = D * BK / 2;
+  static constexpr int VSF_BYTES = (BK / 64) * 512;
+  static constexpr int FP4_ENTRY = V4_OFF + V4_BYTES + VSF_BYTES;
+  static constexpr int PAGE = round1024(cmax(K16_BYTES, FP4_ENTRY));
+
   static constexpr int OFF_Q4 = 0;
-  static constexpr int OFF_QSF = Q4_BYTES;
-  static constexpr int OFF_Q16 = round1024(OFF_QSF + QSF_BYTES);
-  static constexpr int OFF_SLOTS = OFF_Q16 + Q16_BYTES;
-  static constexpr int OFF_P = OFF_SLOTS + NSLOT * SLOT_BYTES;
-  static constexpr int MAXE = 4096;  // entries per unit (two phases of at most 2048 key blocks)
-  static constexpr int OFF_LIST = OFF_P + 2 * PBUF_BYTES;
-  static constexpr int OFF_BAR = OFF_LIST + 2 * MAXE * 2;
-  static constexpr int BYTES = OFF_BAR + 6144 + 1024;  // barriers + alignment slack
-  // TMEM columns
-  static constexpr int COL_S = 0;  // two buffers of BK columns
-  static constexpr int COL_PV = 2 * BK;
-  static constexpr int COL_SFQ = COL_PV + D;
-  static constexpr int SFK_COLS = 4 * (D / 64);
-  static constexpr int SFKV_COLS = 4 * (BK / 64);
-  static constexpr int COL_SFK = COL_SFQ + SFK_COLS;        // two buffers
-  static constexpr int COL_SFV = COL_SFK + 2 * SFK_COLS;    // two buffers
-  static constexpr int COL_SFP = COL_SFV + 2 * SFKV_COLS;   // two buffers
-  static constexpr int TMEM_COLS_USED = COL_SFP + 2 * SFKV_COLS;
-  static_assert(TMEM_COLS_USED <= 512, "TMEM budget");
-  static_assert(BYTES <= 232448, "shared memory budget");
+  static constexpr int OFF_Q16 = OFF_Q4 + Q4_REGION;
+  static constexpr int OFF_P = OFF_Q16 + Q16_BYTES;
+  static constexpr int OFF_PAGES = OFF_P + 2 * PBUF;
+  static constexpr int BAR_BYTES = 3072;
+  // + npage pages, then the barrier block, then the entry lists (sizes chosen at launch)
+  static constexpr int fixed_bytes() { return OFF_PAGES + BAR_BYTES + 1024 /* alignment slack */; }
 };
 
 struct Bars {
-  uint64_t q_full, q_empty, q16_full, q16_empty;
-  uint64_t s_full[2], s_free[2], p_full[2];
-  uint64_t pv_full, pv_free;
-  uint64_t kv_full[6], kv_empty[6];
-  uint64_t list_full[2], list_empty[2];  // per-unit entry lists, double-buffered by unit parity
+  uint64_t q4_full, q4_empty, q16_full, q16_empty;
+  uint64_t s_full[2], s_free[2], p_full[2], pv_full[2], pv_free[2];
+  uint64_t list_full[2], list_empty[2];  // by unit parity
+  uint64_t lx_bar[2];                    // the two softmax warpgroups swap their denominators
+  uint64_t page_full[kMaxPages], page_empty[kMaxPages];
   int list_count[2];
   uint32_t tmem_base;
   int abort_flag;
-  uint64_t pair[4];         // the four softmax warps of each TMEM lane quarter exchange values
-  float xch[2][4][128];     // exchange buffers of the four warps of each lane quarter: [parity][warp][row]
+  float lx[2][2][128];  // [unit parity][warpgroup][row] partial denominators
 };
-
-static_assert(sizeof(Bars) <= 6144, "barrier block");
+static_assert(sizeof(Bars) <= 3072, "barrier block");
 
 struct AttnParams {
   const uint32_t* mask;
@@ -99,44 +122,12 @@ struct AttnParams {
   __half* out;
   float* lse;
   int* status;
-  float* dbg;  // optional dump of one entry (S, P bytes, PV) of the first unit of CTA 0
+  float* dbg;  // optional dump of one entry (S, P bytes, PV) of tile 0 of the first unit of CTA 0
   int dbg_entry;
   int B, Hq, Hkv, N, bq, causal, mode, nqb, nkb, mask_words, n_units;
+  int npage, maxe, off_bar, off_list;
   float tau;
   long long wait_limit;
-};
-
-// The entry list of one unit, regenerated identically by every role.
-struct EntryIter {
-  const uint32_t* m0;
-  const uint32_t* m1;
-  int jmax0, jmax1, jmax, two, mode, phase, j;
-
-  __device__ __forceinline__ int sel(const uint32_t* m, int jj) const {
-    if (mode == 2) return 1;
-    if (mode == 1) return 0;
-    return (int)((__ldg(m + (jj >> 5)) >> (jj & 31)) & 1u);
-  }
-  __device__ __forceinline__ bool next(int& j_out, int& f16_out, int& rm_out) {
-    while (phase < 2) {
-      while (j < jmax) {
-        int jj = j++;
-        int want = phase;
-        int rm = 0;
-        if (jj < jmax0 && sel(m0, jj) == want) rm |= 1;
-        if (two && jj < jmax1 && sel(m1, jj) == want) rm |= 2;
-        if (rm) {
-          j_out = jj;
-          f16_out = want;
-          rm_out = two ? rm : 3;
-          return true;
-        }
-      }
-      ++phase;
-      j = 0;
-    }
-    return false;
-  }
 };
 
 struct UnitInfo {
@@ -144,65 +135,129 @@ struct UnitInfo {
 };
 
 __device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, int u) {
-  int bh_count = p.B * p.Hq;
-  int ntiles = p.N / kBQ;
+  const int bh_count = p.B * p.Hq;
   UnitInfo ui;
-  ui.t = ntiles - 1 - u / bh_count;
-  int bh = u % bh_count;
+  ui.t = p.N / kBQ - 1 - u / bh_count;  // heaviest (longest causal rows) first
+  const int bh = u % bh_count;
   ui.b = bh / p.Hq;
   ui.h = bh % p.Hq;
   ui.hk = ui.h / (p.Hq / p.Hkv);
   return ui;
 }
 
+// The entry list of one 128-row tile of query head h, built by a whole warp: NVFP4 entries, then
+// FP16 entries, each as j | fp16 << 13 | row-half mask << 14 (with 64-row query blocks a key
+// block can be NVFP4 for one half of the tile and FP16 for the other).  Returns the number of
+// entries (same in every lane).
 template <int BK>
-__device__ __forceinline__ EntryIter make_iter(const AttnParams& p, const UnitInfo& ui) {
-  EntryIter it;
-  it.mode = p.mode;
-  it.two = p.bq == 64;
-  int i0 = it.two ? 2 * ui.t : ui.t;
-  int i1 = i0 + 1;
-  const uint32_t* base = p.mask ? p.mask + ((int64_t)(ui.b * p.Hq + ui.h) * p.nqb) * p.mask_words : nullptr;
-  it.m0 = base ? base + (int64_t)i0 * p.mask_words : nullptr;
-  it.m1 = (base && it.two) ? base + (int64_t)i1 * p.mask_words : nullptr;
+__device__ int build_list(const AttnParams& p, int b, int h, int t, uint16_t* list, int lane) {
+  const bool two = p.bq == 64;
+  const int i0 = two ? 2 * t : t, i1 = i0 + 1;
+  const uint32_t* base = p.mask ? p.mask + ((int64_t)(b * p.Hq + h) * p.nqb) * p.mask_words : nullptr;
+  const uint32_t* m0 = base ? base + (int64_t)i0 * p.mask_words : nullptr;
+  const uint32_t* m1 = (base && two) ? base + (int64_t)i1 * p.mask_words : nullptr;
+  int jmax0, jmax1;
   if (p.causal) {
-    it.jmax0 = ((i0 + 1) * p.bq - 1) / BK + 1;
-    it.jmax1 = it.two ? ((i1 + 1) * p.bq - 1) / BK + 1 : 0;
+    jmax0 = ((i0 + 1) * p.bq - 1) / BK + 1;
+    jmax1 = two ? ((i1 + 1) * p.bq - 1) / BK + 1 : 0;
   } else {
-    it.jmax0 = p.nkb;
-    it.jmax1 = it.two ? p.nkb : 0;
+    jmax0 = p.nkb;
+    jmax1 = two ? p.nkb : 0;
   }
-  it.jmax = it.jmax0 > it.jmax1 ? it.jmax0 : it.jmax1;
-  it.phase = 0;
-  it.j = 0;
-  return it;
-}
-
-// The unit's entry list, built once by a whole warp: NVFP4 entries, then FP16 entries, each as
-// j | fp16 << 13 | row-half mask << 14.  Returns the number of entries (same in every lane).
-template <int BK>
-__device__ int build_list(const AttnParams& p, const UnitInfo& ui, uint16_t* list, int lane) {
-  EntryIter it = make_iter<BK>(p, ui);
+  const int jmax = jmax0 > jmax1 ? jmax0 : jmax1;
+  auto sel = [&](const uint32_t* m, int jj) -> int {
+    if (p.mode == 2) return 1;
+    if (p.mode == 1) return 0;
+    return (int)((__ldg(m + (jj >> 5)) >> (jj & 31)) & 1u);
+  };
   int n = 0;
   for (int phase = 0; phase < 2; ++phase) {
-    for (int jb = 0; jb < it.jmax; jb += 32) {
+    for (int jb = 0; jb < jmax; jb += 32) {
       const int jj = jb + lane;
       int rm = 0;
-      if (jj < it.jmax0 && it.sel(it.m0, jj) == phase) rm |= 1;
-      if (it.two && jj < it.jmax1 && it.sel(it.m1, jj) == phase) rm |= 2;
-      if (!it.two && rm) rm = 3;
-      const unsigned b = __ballot_sync(0xffffffffu, rm != 0);
-      if (rm) list[n + __popc(b & ((1u << lane) - 1u))] = (uint16_t)(jj | (phase << 13) | (rm << 14));
-      n += __popc(b);
+      if (jj < jmax0 && sel(m0, jj) == phase) rm |= 1;
+      if (two && jj < jmax1 && sel(m1, jj) == phase) rm |= 2;
+      if (!two && rm) rm = 3;
+      const unsigned bal = __ballot_sync(0xffffffffu, rm != 0);
+      if (rm) list[n + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)(jj | (phase << 13) | (rm << 14));
+      n += __popc(bal);
     }
   }
   return n;
+}
+
+// Page ring position shared by the producer and both issuers (same sequence of pages).
+struct PageRing {
+  int idx, phase, n;
+  __device__ __forceinline__ void next(int& i, int& ph) {
+    i = idx;
+    ph = phase;
+    if (++idx == n) {
+      idx = 0;
+      phase ^= 1;
+    }
+  }
+};
+
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+}
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
 }
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x for a pair of values on the FMA pipe: x = n + f with n = round(x) (by the 1.5 * 2^23
+// rounding constant) and f in [-1/2, 1/2]; 2^f by a degree-5 polynomial (a relative-error minimax
+// fit on [-1/2, 1/2]; relative error below 2.2e-7 including FP32 rounding, about that of the
+// MUFU ex2 approximation, so the E2M1 code decisions of the two paths agree as often); n is added
+// to the exponent field.  Inputs are clamped at -125 so that the result stays a normal number
+// (2^-125 is far below anything that can change a sum or a code).
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+  float2 q = __ffma2_rn(make_float2(0.0013276473619043827f, 0.0013276473619043827f), f,
+                        make_float2(0.009675541892647743f, 0.009675541892647743f));
+  q = __ffma2_rn(q, f, make_float2(0.05550713092088699f, 0.05550713092088699f));
+  q = __ffma2_rn(q, f, make_float2(0.24022120237350464f, 0.24022120237350464f));
+  q = __ffma2_rn(q, f, make_float2(0.6931469440460205f, 0.6931469440460205f));
+  q = __ffma2_rn(q, f, make_float2(1.0000001192092896f, 1.0000001192092896f));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
+// exp2 of a pair of keys; `pair` is the pair's index within its 16-key group (a constant after
+// unrolling): pairs at or past (16 - kPolyPerGroup) / 2 use the polynomial, the others MUFU.
+__device__ __forceinline__ float ex2_poly1(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float n = t - 12582912.0f;
+  const float f = x - n;
+  float q = fmaf(0.0013276473619043827f, f, 0.009675541892647743f);
+  q = fmaf(q, f, 0.05550713092088699f);
+  q = fmaf(q, f, 0.24022120237350464f);
+  q = fmaf(q, f, 0.6931469440460205f);
+  q = fmaf(q, f, 1.0000001192092896f);
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+}
+
+__device__ __forceinline__ float2 ex2_pair(float2 x, int pair) {
+  if (2 * pair >= 16 - kPolyPerGroup) return make_float2(ex2_poly1(x.x), ex2_poly1(x.y));
+  return make_float2(ex2(x.x), ex2(x.y));
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
@@ -214,74 +269,10 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t a) {
-  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
-}
-
-
-constexpr float kNegInf = -__builtin_huge_valf();
-constexpr float kRescale = 8.0f;  // log2 units: rescale O only when the block max grows past 256x
-
-// Rows that do not take part in this block, and keys above the query (causal), become -inf.
-template <int n>
-__device__ __forceinline__ void mask_s(float (&s)[n], bool part, bool diag, int key0, int row) {
-  if (!part) {
-#pragma unroll
-    for (int i = 0; i < n; ++i) s[i] = kNegInf;
-  } else if (diag) {
-#pragma unroll
-    for (int i = 0; i < n; ++i) s[i] = (key0 + i > row) ? kNegInf : s[i];
-  }
-}
-
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-template <int n>
-__device__ __forceinline__ void group_max(const float (&s)[n], float* gm) {
-#pragma unroll
-  for (int q = 0; q < n / 16; ++q) {
-    const float* x = s + 16 * q;
-    float a = max3(x[0], x[1], x[2]), b = max3(x[3], x[4], x[5]), c = max3(x[6], x[7], x[8]);
-    float d = max3(x[9], x[10], x[11]), e = max3(x[12], x[13], x[14]);
-    gm[q] = max3(max3(a, b, c), max3(d, e, x[15]), kNegInf);
-  }
-}
-
-// N consecutive 32-bit TMEM columns of this thread's lane (N = 16 or 32).
-template <int N>
-__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]);
-template <>
-__device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, uint32_t (&r)[32]) {
-  tmem_ld32(taddr, r);
-}
-template <>
-__device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-
-// FP16 probabilities of N keys: exp2(s * sl2 - Ms) rounded to FP16 pairs; returns their FP32 sum.
-template <int N>
-__device__ __forceinline__ float probs_fp16(const float (&s)[N], float sl2, float Ms, uint32_t (&hw)[N / 2]) {
-  const float2 a2 = make_float2(sl2, sl2), b2 = make_float2(-Ms, -Ms);
-  float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-  for (int i = 0; i < N; i += 2) {
-    float2 x = __ffma2_rn(make_float2(s[i], s[i + 1]), a2, b2);
-    float2 pr = make_float2(ex2(x.x), ex2(x.y));
-    acc[(i >> 1) & 1] = __fadd2_rn(acc[(i >> 1) & 1], pr);
-    hw[i >> 1] = pack_half2(pr.x, pr.y);
-  }
-  float2 t = __fadd2_rn(acc[0], acc[1]);
-  return t.x + t.y;
 }
 
 // Eight FP32 values to eight E2M1 codes packed in one word (element 0 in the low nibble).
@@ -298,87 +289,144 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float* y) {
   return out;
 }
 
-// NVFP4 re-quantisation of NG 16-key groups of one row:
-//   P^ = exp2(s*sl2 - Ms); per group s_b = E4M3(2688 max(P^) / 6); codes = E2M1(2688 P^ / s_b).
-// 2688 / s_b is folded into the exponent, so each key costs one FMA and one exp2.  A group whose
-// scale underflows to 0 gets all-zero codes (its values are below 2688 * 2^-10 / 6 / 448).
-// Returns the FP32 sum of the unquantised P^; writes 2*NG code words and NG scale bytes (sfw).
-template <int NG>
-__device__ __forceinline__ float probs_nvfp4(const float (&s)[16 * NG], const float* gm, float sl2, float Ms,
-                                             uint32_t (&cw)[2 * NG], uint32_t& sfw) {
-  float sum = 0.0f;
-  sfw = 0u;
-  const float2 a2 = make_float2(sl2, sl2);
+// Two non-negative FP32 values to E4M3 (round to nearest even, saturating): lo in bits 0-7, hi in 8-15.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(hi), "f"(lo));
+  return out;
+}
+
+// Two E4M3 codes (bits 0-7, 8-15) back to FP32, exactly (through FP16).
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t c2) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(h2) : "r"(c2));
+  __half2 h = *reinterpret_cast<__half2*>(&h2);
+  return __half22float2(h);
+}
+
+// Keys above the query become -inf (causal, on a diagonal block).
+template <int n>
+__device__ __forceinline__ void mask_causal(float (&s)[n], int key0, int row) {
 #pragma unroll
-  for (int q = 0; q < NG; ++q) {
-    const bool live = gm[q] != kNegInf;
-    const float pmax = live ? 2688.0f * ex2(fmaf(gm[q], sl2, -Ms)) : 0.0f;
-    const uint32_t sb = cvt_e4m3(pmax * (1.0f / 6.0f));
-    const float sbf = e4m3_to_f32(sb);
+  for (int i = 0; i < n; ++i) s[i] = (key0 + i > row) ? kNegInf : s[i];
+}
+
+template <int n>
+__device__ __forceinline__ void group_max(const float (&s)[n], float* gm) {
+#pragma unroll
+  for (int q = 0; q < n / 16; ++q) {
+    const float* x = s + 16 * q;
+    const float a = max3(x[0], x[1], x[2]), b = max3(x[3], x[4], x[5]), c = max3(x[6], x[7], x[8]);
+    const float d = max3(x[9], x[10], x[11]), e = max3(x[12], x[13], x[14]);
+    gm[q] = max3(max3(a, b, c), max3(d, e, x[15]), kNegInf);
+  }
+}
+
+// NVFP4 re-quantisation of 32 keys (two 16-key groups) of one row:
+//   P^ = exp2(s*sl2 - Ms); per group s_b = E4M3(2688 max(P^) / 6); codes = E2M1(2688 P^ / s_b).
+// log2(2688 / s_b) is folded into the exponent, so each key costs one FMA and one exp2.  A group
+// whose scale underflows to 0 gets all-zero codes (its values are below 2688 * 2^-10 / 6 / 448).
+// Returns the FP32 sum of the unquantised P^; writes 4 code words and the 2 scale bytes (sf2).
+__device__ __forceinline__ float probs_nvfp4_32(const float (&s)[32], const float* gm, float sl2, float Ms,
+                                                uint32_t (&cw)[4], uint32_t& sf2) {
+  const float pm0 = gm[0] != kNegInf ? 448.0f * ex2(fmaf(gm[0], sl2, -Ms)) : 0.0f;
+  const float pm1 = gm[1] != kNegInf ? 448.0f * ex2(fmaf(gm[1], sl2, -Ms)) : 0.0f;
+  sf2 = cvt_e4m3x2(pm0, pm1);
+  const float2 sbd = e4m3x2_to_f32(sf2);
+  float sum = 0.0f;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const float sbf = q ? sbd.y : sbd.x;
     const float sbe = sbf > 0.0f ? sbf : 448.0f;
-    const float bias = live ? (11.392317422778761f - __log2f(sbe)) - Ms : kNegInf;  // log2(2688 / s_b) - Ms
-    const float2 b2 = make_float2(bias, bias);
+    const float bias = gm[q] != kNegInf ? (11.392317422778761f - lg2(sbe)) - Ms : kNegInf;  // log2(2688/s_b) - Ms
     float y[16];
     float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int t = 0; t < 16; t += 2) {
-      float2 x = __ffma2_rn(make_float2(s[16 * q + t], s[16 * q + t + 1]), a2, b2);
-      y[t] = ex2(x.x);
-      y[t + 1] = ex2(x.y);
-      if (t & 2)
-        acc1 = __fadd2_rn(acc1, make_float2(y[t], y[t + 1]));
-      else
-        acc0 = __fadd2_rn(acc0, make_float2(y[t], y[t + 1]));
+      const float2 x = make_float2(fmaf(s[16 * q + t], sl2, bias), fmaf(s[16 * q + t + 1], sl2, bias));
+      const float2 e = ex2_pair(x, t >> 1);
+      y[t] = e.x;
+      y[t + 1] = e.y;
+      if (t & 2) { acc1.x += e.x; acc1.y += e.y; } else { acc0.x += e.x; acc0.y += e.y; }
     }
     cw[2 * q] = cvt_e2m1x8(y);
     cw[2 * q + 1] = cvt_e2m1x8(y + 8);
-    const float2 t2 = __fadd2_rn(acc0, acc1);
-    sum = fmaf(t2.x + t2.y, sbe * (1.0f / 2688.0f), sum);
-    sfw |= sb << (8 * q);
+    sum = fmaf((acc0.x + acc1.x) + (acc0.y + acc1.y), sbe * (1.0f / 2688.0f), sum);
   }
   return sum;
 }
 
+// FP16 probabilities of 32 keys: exp2(s * sl2 - Ms) rounded to FP16 pairs, written straight into
+// the SW128 PV operand row at `rowaddr` (16-byte chunk c8 at ((c8 ^ swz) << 4), chunks c0..c0+3);
+// returns their FP32 sum.  `dbg` (may be null) receives the 16 words as well.
+__device__ __forceinline__ float probs_fp16_32(const float (&s)[32], float sl2, float Ms, uint32_t rowaddr, int c0,
+                                               int swz, uint32_t* dbg) {
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c8 = 0; c8 < 4; ++c8) {
+    uint32_t hw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = 8 * c8 + 2 * k;
+      const float2 x = make_float2(fmaf(s[i], sl2, -Ms), fmaf(s[i + 1], sl2, -Ms));
+      const float2 pr = ex2_pair(x, (4 * c8 + k) & 7);
+      acc[k & 1] += pr.x;
+      acc[2 + (k & 1)] += pr.y;
+      hw[k] = pack_half2(pr.x, pr.y);
+    }
+    st_shared_v4(rowaddr + (((c0 + c8) ^ swz) << 4), hw[0], hw[1], hw[2], hw[3]);
+    if (dbg)
+      for (int k = 0; k < 4; ++k) dbg[4 * c8 + k] = hw[k];
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// Maximum of n values.
+template <int n>
+__device__ __forceinline__ float row_max(const float* x) {
+  float m = kNegInf;
+#pragma unroll
+  for (int i = 0; i + 2 < n; i += 3) m = max3(m, x[i], fmaxf(x[i + 1], x[i + 2]));
+#pragma unroll
+  for (int i = n - n % 3; i < n; ++i) m = fmaxf(m, x[i]);
+  return m;
+}
+
 template <int D, int BK, bool DBG>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q4, const __grid_constant__ CUtensorMap tm_k4,
                 const __grid_constant__ CUtensorMap tm_v4, const __grid_constant__ CUtensorMap tm_q16,
                 const __grid_constant__ CUtensorMap tm_k16, const __grid_constant__ CUtensorMap tm_v16,
                 const __grid_constant__ AttnParams p) {
   using L = Layout<D, BK>;
+  constexpr int KH = L::KH, DH = L::DH;
   extern __shared__ uint8_t smem_raw[];
-  uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023) & ~1023u) - raw_addr);
-  uint8_t* sQ4 = smem + L::OFF_Q4;
-  uint8_t* sQSF = smem + L::OFF_QSF;
-  uint8_t* sQ16 = smem + L::OFF_Q16;
-  uint8_t* sSlots = smem + L::OFF_SLOTS;
-  uint8_t* sP = smem + L::OFF_P;
-  Bars* bars = reinterpret_cast<Bars*>(smem + L::OFF_BAR);
+  Bars* bars = reinterpret_cast<Bars*>(smem + p.off_bar);
+  uint16_t* lists = reinterpret_cast<uint16_t*>(smem + p.off_list);  // [unit parity][maxe]
   volatile int* abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
+    mbar_init(&bars->q4_full, 1);
+    mbar_init(&bars->q4_empty, 1);
     mbar_init(&bars->q16_full, 1);
     mbar_init(&bars->q16_empty, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->s_free[i], kSoftmaxThreads);
-      mbar_init(&bars->p_full[i], kSoftmaxThreads);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->s_free[x], 256);
+      mbar_init(&bars->p_full[x], 256);
+      mbar_init(&bars->pv_full[x], 1);
+      mbar_init(&bars->pv_free[x], 256);
+      mbar_init(&bars->list_full[x], 1);
+      mbar_init(&bars->list_empty[x], 2 + 256);
+      mbar_init(&bars->lx_bar[x], 256);
     }
-    mbar_init(&bars->pv_full, 1);
-    mbar_init(&bars->pv_free, kSoftmaxThreads);
-    for (int i = 0; i < 4; ++i) mbar_init(&bars->pair[i], 128);
-    for (int i = 0; i < L::NSLOT; ++i) {
-      mbar_init(&bars->kv_full[i], 1);
-      mbar_init(&bars->kv_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->list_full[i], 1);
-      mbar_init(&bars->list_empty[i], 2 + kSoftmaxThreads);
+    for (int i = 0; i < kMaxPages; ++i) {
+      mbar_init(&bars->page_full[i], 1);
+      mbar_init(&bars->page_empty[i], 2);
     }
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -393,422 +441,438 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
   const long long lim = p.wait_limit;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ producer
-    // The whole warp builds each unit's entry list; lane 0 then issues the unit's loads.
-    uint16_t* lists = reinterpret_cast<uint16_t*>(smem + L::OFF_LIST);
-    if (lane == 0) {
-      if (p.mode != 2) {
-        prefetch_tmap(&tm_q4);
-        prefetch_tmap(&tm_k4);
-        prefetch_tmap(&tm_v4);
+  if (warp < 4) {
+    setmaxnreg_dec();
+    if (warp == 0) {
+      // ---------------------------------------------------------------- producer
+      if (lane == 0) {
+        if (p.mode != 2) {
+          prefetch_tmap(&tm_q4);
+          prefetch_tmap(&tm_k4);
+          prefetch_tmap(&tm_v4);
+        }
+        if (p.mode != 1) {
+          prefetch_tmap(&tm_q16);
+          prefetch_tmap(&tm_k16);
+          prefetch_tmap(&tm_v16);
+        }
       }
-      if (p.mode != 1) {
-        prefetch_tmap(&tm_q16);
-        prefetch_tmap(&tm_k16);
-        prefetch_tmap(&tm_v16);
-      }
-    }
-    {
-      uint32_t slot_ctr = 0, unit_ctr = 0, u16_ctr = 0;
+      PageRing ring{0, 0, p.npage};
+      uint32_t uc = 0, u16c = 0;
       bool ok = true;
-      // lane 0: every load of one unit (returns false after a timeout)
-      auto issue_unit = [&](const UnitInfo& ui, const uint16_t* list, int n_entries) -> bool {
-          const int qrow0 = (ui.b * p.Hq + ui.h) * p.N + ui.t * kBQ;
-          const int kvh = ui.b * p.Hkv + ui.hk;
-          if (!mbar_wait(&bars->q_empty, (unit_ctr & 1) ^ 1, abort_flag, p.status, lim)) return false;
-          if (p.mode != 2) {
-            mbar_arrive_expect_tx(&bars->q_full, L::Q4_BYTES + L::QSF_BYTES);
-            tma_load_2d(sQ4, &tm_q4, &bars->q_full, 0, qrow0);
-            bulk_load(sQSF, p.q_sf + (size_t)(qrow0 / 128) * L::QSF_BYTES, L::QSF_BYTES, &bars->q_full);
-          } else {
-            mbar_arrive(&bars->q_full);
-          }
-          bool q16_loaded = false;
-          for (int e = 0; e < n_entries; ++e) {
-            const uint32_t x = list[e];
-            const int j = x & 0x1fff, f16 = (x >> 13) & 1;
-            if (f16 && !q16_loaded) {
-              if (!(ok = mbar_wait(&bars->q16_empty, (u16_ctr & 1) ^ 1, abort_flag, p.status, lim))) break;
-              mbar_arrive_expect_tx(&bars->q16_full, L::Q16_BYTES);
-  #pragma unroll
-              for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(sQ16 + cb * kBQ * 128, &tm_q16, &bars->q16_full, cb * 64, qrow0);
-              q16_loaded = true;
-            }
-            const int krow0 = kvh * p.N + j * BK;
-            // K tile
-            {
-              uint32_t s = slot_ctr % L::NSLOT, ph = (slot_ctr / L::NSLOT) & 1;
-              ++slot_ctr;
-              if (!(ok = mbar_wait(&bars->kv_empty[s], ph ^ 1, abort_flag, p.status, lim))) break;
-              uint8_t* dst = sSlots + s * L::SLOT_BYTES;
-              if (f16) {
-                mbar_arrive_expect_tx(&bars->kv_full[s], BK * D * 2);
-  #pragma unroll
-                for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(dst + cb * BK * 128, &tm_k16, &bars->kv_full[s], cb * 64, krow0);
-              } else {
-                mbar_arrive_expect_tx(&bars->kv_full[s], BK * D / 2 + L::QSF_BYTES);
-                tma_load_2d(dst, &tm_k4, &bars->kv_full[s], 0, krow0);
-                bulk_load(dst + BK * D / 2, p.k_sf + (size_t)(krow0 / 128) * L::QSF_BYTES, L::QSF_BYTES, &bars->kv_full[s]);
-              }
-            }
-            // V tile
-            {
-              uint32_t s = slot_ctr % L::NSLOT, ph = (slot_ctr / L::NSLOT) & 1;
-              ++slot_ctr;
-              if (!(ok = mbar_wait(&bars->kv_empty[s], ph ^ 1, abort_flag, p.status, lim))) break;
-              uint8_t* dst = sSlots + s * L::SLOT_BYTES;
-              if (f16) {
-                mbar_arrive_expect_tx(&bars->kv_full[s], BK * D * 2);
-  #pragma unroll
-                for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(dst + cb * BK * 128, &tm_v16, &bars->kv_full[s], cb * 64, krow0);
-              } else {
-                const int vrow0 = kvh * D;
-                mbar_arrive_expect_tx(&bars->kv_full[s], D * BK / 2 + L::PSF_BYTES);
-                tma_load_2d(dst, &tm_v4, &bars->kv_full[s], j * (BK / 2), vrow0);
-                size_t sf_off = ((size_t)(vrow0 / 128) * (p.N / 64) + (size_t)j * (BK / 64)) * 512;
-                bulk_load(dst + D * BK / 2, p.v_sf + sf_off, L::PSF_BYTES, &bars->kv_full[s]);
-              }
-            }
-          }
-          if (q16_loaded) ++u16_ctr;
-          return ok;
-      };
-      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x, ++unit_ctr) {
-        UnitInfo ui = decode_unit(p, u);
-        const uint32_t lb = unit_ctr & 1;
-        uint16_t* list = lists + lb * L::MAXE;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
+        const UnitInfo ui = decode_unit(p, u);
+        const uint32_t lb = uc & 1, lph = (uc >> 1) & 1;
         // the warp is converged here: every exit below is taken by all 32 lanes together
-        const bool free_ok = mbar_wait(&bars->list_empty[lb], ((unit_ctr >> 1) & 1) ^ 1, abort_flag, p.status, lim);
+        const bool free_ok = mbar_wait(&bars->list_empty[lb], lph ^ 1, abort_flag, p.status, lim);
         if (!__all_sync(0xffffffffu, free_ok)) break;
-        const int n_entries = build_list<BK>(p, ui, list, lane);
+        uint16_t* list = lists + lb * p.maxe;
+        const int n = build_list<BK>(p, ui.b, ui.h, ui.t, list, lane);
         __syncwarp();
         if (lane == 0) {
-          bars->list_count[lb] = n_entries;
+          bars->list_count[lb] = n;
           mbar_arrive(&bars->list_full[lb]);
-          ok = issue_unit(ui, list, n_entries);
+          const int kvh = ui.b * p.Hkv + ui.hk;
+          const int qrow0 = (ui.b * p.Hq + ui.h) * p.N + ui.t * kBQ;
+          if ((ok = mbar_wait(&bars->q4_empty, (uc & 1) ^ 1, abort_flag, p.status, lim))) {
+            uint8_t* sq = smem + L::OFF_Q4;
+            if (p.mode != 2) {
+              mbar_arrive_expect_tx(&bars->q4_full, L::Q4_BYTES + L::QSF_BYTES);
+              tma_load_2d(sq, &tm_q4, &bars->q4_full, 0, qrow0);
+              bulk_load(sq + L::Q4_BYTES, p.q_sf + (size_t)(qrow0 / 128) * L::QSF_BYTES, L::QSF_BYTES, &bars->q4_full);
+            } else {
+              mbar_arrive(&bars->q4_full);
+            }
+          }
+          bool q16_loaded = false;
+          for (int e = 0; e < n && ok; ++e) {
+            const uint32_t xe = list[e];
+            const int j = xe & 0x1fff, f16 = (xe >> 13) & 1;
+            const int krow0 = kvh * p.N + j * BK;
+            if (f16 && !q16_loaded) {
+              if (!(ok = mbar_wait(&bars->q16_empty, (u16c & 1) ^ 1, abort_flag, p.status, lim))) break;
+              ++u16c;
+              uint8_t* sq = smem + L::OFF_Q16;
+              mbar_arrive_expect_tx(&bars->q16_full, L::Q16_BYTES);
+#pragma unroll
+              for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(sq + cb * kBQ * 128, &tm_q16, &bars->q16_full, cb * 64, qrow0);
+              q16_loaded = true;
+            }
+            int pg, ph;
+            if (f16) {
+              for (int kv = 0; kv < 2 && ok; ++kv) {
+                ring.next(pg, ph);
+                if (!(ok = mbar_wait(&bars->page_empty[pg], ph ^ 1, abort_flag, p.status, lim))) break;
+                uint8_t* dst = smem + L::OFF_PAGES + pg * L::PAGE;
+                mbar_arrive_expect_tx(&bars->page_full[pg], L::K16_BYTES);
+#pragma unroll
+                for (int cb = 0; cb < D / 64; ++cb)
+                  tma_load_2d(dst + cb * BK * 128, kv ? &tm_v16 : &tm_k16, &bars->page_full[pg], cb * 64, krow0);
+              }
+            } else {
+              ring.next(pg, ph);
+              if (!(ok = mbar_wait(&bars->page_empty[pg], ph ^ 1, abort_flag, p.status, lim))) break;
+              uint8_t* dst = smem + L::OFF_PAGES + pg * L::PAGE;
+              mbar_arrive_expect_tx(&bars->page_full[pg], L::K4_BYTES + L::KSF_BYTES + L::V4_BYTES + L::VSF_BYTES);
+              tma_load_2d(dst, &tm_k4, &bars->page_full[pg], 0, krow0);
+              bulk_load(dst + L::K4_BYTES, p.k_sf + (size_t)(krow0 / 128) * L::KSF_BYTES, L::KSF_BYTES,
+                        &bars->page_full[pg]);
+              const int vrow0 = kvh * D;
+              tma_load_2d(dst + L::V4_OFF, &tm_v4, &bars->page_full[pg], j * (BK / 2), vrow0);
+              const size_t sf_off = ((size_t)(vrow0 / 128) * (p.N / 64) + (size_t)j * (BK / 64)) * 512;
+              bulk_load(dst + L::V4_OFF + L::V4_BYTES, p.v_sf + sf_off, L::VSF_BYTES, &bars->page_full[pg]);
+            }
+          }
         }
         __syncwarp();
-        if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
+        ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ QK^T issuer
-    if (lane == 0) {
-      const uint32_t idesc_qk4 = idesc_nvf4(kBQ, BK);
-      const uint32_t idesc_qk16 = idesc_f16(kBQ, BK, 0, 0);
-      constexpr int SWQ = swz_for_row_bytes(D / 2);
-      const uint32_t qb4 = smem_u32(sQ4), qb16 = smem_u32(sQ16);
-      uint32_t slot_ctr = 0, unit_ctr = 0, u16_ctr = 0, g = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_ctr) {
-        UnitInfo ui = decode_unit(p, u);
-        const int kvh = ui.b * p.Hkv + ui.hk;
-        if (!(ok = mbar_wait(&bars->q_full, unit_ctr & 1, abort_flag, p.status, lim))) break;
-        tc_fence_after();
-        if (p.mode != 2) {
-#pragma unroll
-          for (int kk = 0; kk < D / 64; ++kk)
-            tc_copy_sf(tmem + L::COL_SFQ + 4 * kk, make_sdesc(smem_u32(sQSF) + kk * 512, 16, 128, 0));
-        }
-        bool any16 = false;
-        const uint32_t lb = unit_ctr & 1;
-        const uint16_t* list = reinterpret_cast<const uint16_t*>(smem + L::OFF_LIST) + lb * L::MAXE;
-        if (!(ok = mbar_wait(&bars->list_full[lb], (unit_ctr >> 1) & 1, abort_flag, p.status, lim))) break;
-        const int n_entries = bars->list_count[lb];
-        for (int e = 0; ok && e < n_entries; ++e) {
-          const uint32_t x = list[e];
-          const int j = x & 0x1fff, f16 = (x >> 13) & 1;
-          const uint32_t kslot = slot_ctr % L::NSLOT, kph = (slot_ctr / L::NSLOT) & 1;
-          slot_ctr += 2;  // this entry's V tile takes the next slot (the PV issuer consumes it)
-          if (f16 && !any16) {
-            if (!(ok = mbar_wait(&bars->q16_full, u16_ctr & 1, abort_flag, p.status, lim))) break;
-            any16 = true;
-          }
-          const uint32_t buf = g & 1;
-          if (!(ok = mbar_wait(&bars->kv_full[kslot], kph, abort_flag, p.status, lim))) break;
-          if (!(ok = mbar_wait(&bars->s_free[buf], ((g >> 1) & 1) ^ 1, abort_flag, p.status, lim))) break;
+    } else if (warp == 1) {
+      // ---------------------------------------------------------------- QK^T issuer
+      if (lane == 0) {
+        const uint32_t idesc_qk4 = idesc_nvf4(kBQ, BK);
+        const uint32_t idesc_qk16 = idesc_f16(kBQ, BK, 0, 0);
+        constexpr int SWQ = swz_for_row_bytes(D / 2);
+        const uint32_t qb4 = smem_u32(smem + L::OFF_Q4), qb16 = smem_u32(smem + L::OFF_Q16);
+        PageRing ring{0, 0, p.npage};
+        uint32_t uc = 0, u16c = 0, g = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
+          const UnitInfo ui = decode_unit(p, u);
+          const int kvh = ui.b * p.Hkv + ui.hk;
+          const uint32_t lb = uc & 1, lph = (uc >> 1) & 1;
+          if (!(ok = mbar_wait(&bars->list_full[lb], lph, abort_flag, p.status, lim))) break;
+          const int n = bars->list_count[lb];
+          const uint16_t* list = lists + lb * p.maxe;
+          if (!(ok = mbar_wait(&bars->q4_full, uc & 1, abort_flag, p.status, lim))) break;
           tc_fence_after();
-          const uint32_t kbuf = smem_u32(sSlots + kslot * L::SLOT_BYTES);
-          const uint32_t dS = tmem + L::COL_S + buf * BK;
-          if (f16) {
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              uint64_t ad = make_sdesc(qb16 + (kk >> 2) * kBQ * 128 + (kk & 3) * 32, 16, 1024, kSW128);
-              uint64_t bd = make_sdesc(kbuf + (kk >> 2) * BK * 128 + (kk & 3) * 32, 16, 1024, kSW128);
-              mma_f16(dS, ad, bd, idesc_qk16, kk > 0);
-            }
-          } else {
-            const int krow0 = kvh * p.N + j * BK;
-            const int sfk_off = (krow0 & 127) >> 5;
-            const uint32_t sfk = tmem + L::COL_SFK + buf * L::SFK_COLS;
+          if (p.mode != 2) {
 #pragma unroll
             for (int kk = 0; kk < D / 64; ++kk)
-              tc_copy_sf(sfk + 4 * kk, make_sdesc(kbuf + BK * D / 2 + kk * 512, 16, 128, 0));
-#pragma unroll
-            for (int kk = 0; kk < D / 64; ++kk) {
-              uint64_t ad = make_sdesc(qb4 + kk * 32, 16, 8 * (D / 2), SWQ);
-              uint64_t bd = make_sdesc(kbuf + kk * 32, 16, 8 * (D / 2), SWQ);
-              mma_nvf4(dS, ad, bd, idesc_qk4, tmem + L::COL_SFQ + 4 * kk, sfk + 4 * kk + sfk_off, kk > 0);
-            }
+              tc_copy_sf(tmem + L::COL_SFQ + 4 * kk, make_sdesc(qb4 + L::Q4_BYTES + kk * 512, 16, 128, 0));
           }
-          tc_commit(&bars->s_full[buf]);
-          tc_commit(&bars->kv_empty[kslot]);
-          ++g;
-        }
-        if (!ok) break;
-        mbar_arrive(&bars->list_empty[lb]);
-        tc_commit(&bars->q_empty);
-        if (any16) {
-          tc_commit(&bars->q16_empty);
-          ++u16_ctr;
+          bool released4 = false, any16 = false;
+          for (int e = 0; e < n && ok; ++e) {
+            const uint32_t xe = list[e];
+            const int j = xe & 0x1fff, f16 = (xe >> 13) & 1;
+            if (f16 && !released4) {
+              tc_commit(&bars->q4_empty);  // every NVFP4 product of this unit has been issued
+              released4 = true;
+            }
+            if (f16 && !any16) {
+              if (!(ok = mbar_wait(&bars->q16_full, u16c & 1, abort_flag, p.status, lim))) break;
+              ++u16c;
+              any16 = true;
+            }
+            int pk, phk, pv = 0, phv = 0;
+            ring.next(pk, phk);
+            if (f16) ring.next(pv, phv);
+            const uint32_t buf = g & 1;
+            if (!(ok = mbar_wait(&bars->page_full[pk], phk, abort_flag, p.status, lim))) break;
+            if (!(ok = mbar_wait(&bars->s_free[buf], ((g >> 1) & 1) ^ 1, abort_flag, p.status, lim))) break;
+            tc_fence_after();
+            const uint32_t kbuf = smem_u32(smem + L::OFF_PAGES + pk * L::PAGE);
+            const uint32_t dS = tmem + L::COL_S + buf * BK;
+            if (f16) {
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t ad = make_sdesc(qb16 + (kk >> 2) * kBQ * 128 + (kk & 3) * 32, 16, 1024, kSW128);
+                const uint64_t bd = make_sdesc(kbuf + (kk >> 2) * BK * 128 + (kk & 3) * 32, 16, 1024, kSW128);
+                mma_f16(dS, ad, bd, idesc_qk16, kk > 0);
+              }
+            } else {
+              const int sfk_off = ((kvh * p.N + j * BK) & 127) >> 5;
+              const uint32_t sfk = tmem + L::COL_SFK + buf * L::SFQ;
+#pragma unroll
+              for (int kk = 0; kk < D / 64; ++kk)
+                tc_copy_sf(sfk + 4 * kk, make_sdesc(kbuf + L::K4_BYTES + kk * 512, 16, 128, 0));
+#pragma unroll
+              for (int kk = 0; kk < D / 64; ++kk) {
+                const uint64_t ad = make_sdesc(qb4 + kk * 32, 16, 8 * (D / 2), SWQ);
+                const uint64_t bd = make_sdesc(kbuf + kk * 32, 16, 8 * (D / 2), SWQ);
+                mma_nvf4(dS, ad, bd, idesc_qk4, tmem + L::COL_SFQ + 4 * kk, sfk + 4 * kk + sfk_off, kk > 0);
+              }
+            }
+            tc_commit(&bars->s_full[buf]);
+            tc_commit(&bars->page_empty[pk]);  // the V page of an FP16 entry is the PV issuer's
+            ++g;
+          }
+          if (!ok) break;
+          if (!released4) tc_commit(&bars->q4_empty);
+          if (any16) tc_commit(&bars->q16_empty);
+          mbar_arrive(&bars->list_empty[lb]);
         }
       }
-    }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------------ PV issuer
-    if (lane == 0) {
-      const uint32_t idesc_pv4 = idesc_nvf4(kBQ, D);
-      const uint32_t idesc_pv16 = idesc_f16(kBQ, D, 0, 1);
-      constexpr int SWP = swz_for_row_bytes(BK / 2);
-      uint32_t slot_ctr = 0, unit_ctr = 0, g = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_ctr) {
-        UnitInfo ui = decode_unit(p, u);
-        const int sfv_off = (((ui.b * p.Hkv + ui.hk) * D) & 127) >> 5;
-        const uint32_t lb = unit_ctr & 1;
-        const uint16_t* list = reinterpret_cast<const uint16_t*>(smem + L::OFF_LIST) + lb * L::MAXE;
-        if (!(ok = mbar_wait(&bars->list_full[lb], (unit_ctr >> 1) & 1, abort_flag, p.status, lim))) break;
-        const int n_entries = bars->list_count[lb];
-        for (int e = 0; ok && e < n_entries; ++e) {
-          const int f16 = (list[e] >> 13) & 1;
-          const uint32_t vslot = (slot_ctr + 1) % L::NSLOT, vph = ((slot_ctr + 1) / L::NSLOT) & 1;
-          slot_ctr += 2;
-          const uint32_t buf = g & 1;
-          if (!(ok = mbar_wait(&bars->p_full[buf], (g >> 1) & 1, abort_flag, p.status, lim))) break;
-          if (!(ok = mbar_wait(&bars->pv_free, (g & 1) ^ 1, abort_flag, p.status, lim))) break;
-          if (!(ok = mbar_wait(&bars->kv_full[vslot], vph, abort_flag, p.status, lim))) break;
-          tc_fence_after();
-          const uint32_t pbuf = smem_u32(sP + buf * L::PBUF_BYTES);
-          const uint32_t vbuf = smem_u32(sSlots + vslot * L::SLOT_BYTES);
-          if (f16) {
+    } else if (warp == 2) {
+      // ---------------------------------------------------------------- PV issuer
+      if (lane == 0) {
+        const uint32_t idesc_pv4 = idesc_nvf4(kBQ, D);
+        const uint32_t idesc_pv16 = idesc_f16(kBQ, D, 0, 1);
+        constexpr int SWP = swz_for_row_bytes(BK / 2);
+        PageRing ring{0, 0, p.npage};
+        uint32_t uc = 0, g = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
+          const UnitInfo ui = decode_unit(p, u);
+          const int sfv_off = (((ui.b * p.Hkv + ui.hk) * D) & 127) >> 5;
+          const uint32_t lb = uc & 1, lph = (uc >> 1) & 1;
+          if (!(ok = mbar_wait(&bars->list_full[lb], lph, abort_flag, p.status, lim))) break;
+          const int n = bars->list_count[lb];
+          const uint16_t* list = lists + lb * p.maxe;
+          for (int e = 0; e < n && ok; ++e) {
+            const int f16 = (list[e] >> 13) & 1;
+            int pk, phk, pv = 0, phv = 0;
+            ring.next(pk, phk);
+            if (f16) ring.next(pv, phv);
+            const int pgv = f16 ? pv : pk, phv_ = f16 ? phv : phk;
+            const uint32_t buf = g & 1;
+            const uint32_t pvb = L::NPV == 2 ? buf : 0;
+            const uint32_t pv_par = L::NPV == 2 ? (((g >> 1) & 1) ^ 1) : ((g & 1) ^ 1);
+            if (!(ok = mbar_wait(&bars->p_full[buf], (g >> 1) & 1, abort_flag, p.status, lim))) break;
+            if (!(ok = mbar_wait(&bars->pv_free[pvb], pv_par, abort_flag, p.status, lim))) break;
+            if (!(ok = mbar_wait(&bars->page_full[pgv], phv_, abort_flag, p.status, lim))) break;
+            tc_fence_after();
+            const uint32_t pbuf = smem_u32(smem + L::OFF_P + buf * L::PBUF);
+            const uint32_t vpage = smem_u32(smem + L::OFF_PAGES + pgv * L::PAGE);
+            const uint32_t dPV = tmem + L::COL_PV + pvb * D;
+            if (f16) {
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              uint64_t ad = make_sdesc(pbuf + (kk >> 2) * kBQ * 128 + (kk & 3) * 32, 16, 1024, kSW128);
-              uint64_t bd = make_sdesc(vbuf + kk * 16 * 128, BK * 128, 1024, kSW128);
-              mma_f16(tmem + L::COL_PV, ad, bd, idesc_pv16, kk > 0);
-            }
-          } else {
-            const uint32_t sfv = tmem + L::COL_SFV + buf * L::SFKV_COLS;
-            const uint32_t sfp = tmem + L::COL_SFP + buf * L::SFKV_COLS;
+              for (int kk = 0; kk < BK / 16; ++kk) {
+                const uint64_t ad = make_sdesc(pbuf + (kk >> 2) * kBQ * 128 + (kk & 3) * 32, 16, 1024, kSW128);
+                const uint64_t bd = make_sdesc(vpage + kk * 16 * 128, BK * 128, 1024, kSW128);
+                mma_f16(dPV, ad, bd, idesc_pv16, kk > 0);
+              }
+            } else {
+              const uint32_t vbuf = vpage + L::V4_OFF;
+              const uint32_t sfv = tmem + L::COL_SFV + buf * L::SFV, sfp = tmem + L::COL_SFP + buf * L::SFV;
 #pragma unroll
-            for (int kb = 0; kb < BK / 64; ++kb) {
-              tc_copy_sf(sfv + 4 * kb, make_sdesc(vbuf + D * BK / 2 + kb * 512, 16, 128, 0));
-              tc_copy_sf(sfp + 4 * kb, make_sdesc(pbuf + L::P4_BYTES + kb * 512, 16, 128, 0));
-            }
+              for (int kb = 0; kb < BK / 64; ++kb) {
+                tc_copy_sf(sfv + 4 * kb, make_sdesc(vbuf + L::V4_BYTES + kb * 512, 16, 128, 0));
+                tc_copy_sf(sfp + 4 * kb, make_sdesc(pbuf + L::P4_BYTES + kb * 512, 16, 128, 0));
+              }
 #pragma unroll
-            for (int kb = 0; kb < BK / 64; ++kb) {
-              uint64_t ad = make_sdesc(pbuf + kb * 32, 16, 8 * (BK / 2), SWP);
-              uint64_t bd = make_sdesc(vbuf + kb * 32, 16, 8 * (BK / 2), SWP);
-              mma_nvf4(tmem + L::COL_PV, ad, bd, idesc_pv4, sfp + 4 * kb, sfv + 4 * kb + sfv_off, kb > 0);
+              for (int kb = 0; kb < BK / 64; ++kb) {
+                const uint64_t ad = make_sdesc(pbuf + kb * 32, 16, 8 * (BK / 2), SWP);
+                const uint64_t bd = make_sdesc(vbuf + kb * 32, 16, 8 * (BK / 2), SWP);
+                mma_nvf4(dPV, ad, bd, idesc_pv4, sfp + 4 * kb, sfv + 4 * kb + sfv_off, kb > 0);
+              }
             }
+            tc_commit(&bars->pv_full[pvb]);
+            if (f16) {
+              // Both arrivals of the V page come from here, after its page_full wait: an arrival
+              // issued before the page holds this entry's tile could complete the phase of the
+              // page's previous use.  The K page gets the QK^T issuer's commit and this arrival.
+              mbar_arrive(&bars->page_empty[pk]);
+              mbar_arrive(&bars->page_empty[pv]);
+              tc_commit(&bars->page_empty[pv]);
+            } else {
+              tc_commit(&bars->page_empty[pk]);
+            }
+            ++g;
           }
-          tc_commit(&bars->pv_full);
-          tc_commit(&bars->kv_empty[vslot]);
-          ++g;
+          if (!ok) break;
+          mbar_arrive(&bars->list_empty[lb]);
         }
-        if (!ok) break;
-        mbar_arrive(&bars->list_empty[lb]);
       }
     }
   } else {
     // ------------------------------------------------------------------ softmax / merge
-    // Four warps share each TMEM lane quarter (the same 32 query rows).  Warp `kq` of the quarter
-    // reads keys [kq*BK/4, (kq+1)*BK/4) of the score row, the four swap their maxima to get the
-    // row maximum M of the key block, and each produces its keys' probabilities and accumulates
-    // output columns [kq*D/4, (kq+1)*D/4).
+    setmaxnreg_inc();
+    const int wg = (warp - 4) >> 2;  // which half of the keys and of the output columns
     const int quarter = warp & 3;
-    const int kq = (warp - kFirstSoftmaxWarp) >> 2;
     const int rr = quarter * 32 + lane;  // row of the tile = TMEM lane
-    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    constexpr int DW = D / 4, KW = BK / 4;
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const float q_ts = (p.mode != 2) ? __ldg(p.q_ts) : 1.0f;
     const float k_ts = (p.mode != 2) ? __ldg(p.k_ts) : 1.0f;
     const float v_ts = (p.mode != 2) ? __ldg(p.v_ts) : 1.0f;
     const float sl2_4 = q_ts * k_ts * p.tau * kLog2e;
     const float sl2_16 = p.tau * kLog2e;
     const float pv4_scale = v_ts * (1.0f / 2688.0f);
-    uint32_t g = 0, unit_ctr = 0, xk = 0;
+    uint32_t g = 0, uc = 0;
     bool ok = true;
-    // combine a value over the four warps of this lane quarter (max or sum; bounded wait)
-    auto exchange = [&](float v, bool take_max) -> float {
-      const uint32_t par = xk & 1;
-      bars->xch[par][kq][rr] = v;
-      mbar_arrive(&bars->pair[quarter]);
-      const bool got = mbar_wait(&bars->pair[quarter], par, abort_flag, p.status, lim);
-      ++xk;
-      if (!got) {
-        ok = false;
-        return v;
-      }
-      const float a = bars->xch[par][0][rr], b = bars->xch[par][1][rr];
-      const float c = bars->xch[par][2][rr], d = bars->xch[par][3][rr];
-      return take_max ? max3(a, b, fmaxf(c, d)) : (a + b) + (c + d);
-    };
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_ctr) {
-      UnitInfo ui = decode_unit(p, u);
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
+      const UnitInfo ui = decode_unit(p, u);
+      const uint32_t lb = uc & 1, lph = (uc >> 1) & 1;
+      if (!(ok = mbar_wait(&bars->list_full[lb], lph, abort_flag, p.status, lim))) break;
+      const int n_entries = bars->list_count[lb];
+      const uint16_t* list = lists + lb * p.maxe;
       const int row = ui.t * kBQ + rr;
       const int half = (p.bq == 64) ? (rr >> 6) : 0;
-      float O[DW];
+      float O[DH];
 #pragma unroll
-      for (int c = 0; c < DW; ++c) O[c] = 0.0f;
+      for (int c = 0; c < DH; ++c) O[c] = 0.0f;
       // running state: O and l are relative to exp2(m_ref); m_ref moves only when a block's
-      // maximum exceeds it by more than 2^kRescale (the final O / l does not depend on m_ref)
+      // maximum exceeds it by more than 2^kRescale (the final O / l does not depend on m_ref).
+      // Both warpgroups see the same block maxima, so they take the same decisions.
       float m_ref = kNegInf, l_run = 0.0f;
       float pend_M = kNegInf, pend_sum = 0.0f;
       int pend_f16 = 0;
-      bool have_pend = false;
       const bool dbg_unit = DBG && p.dbg && blockIdx.x == 0 && u == (int)blockIdx.x;
-      int local_e = 0;
+      const uint32_t g0 = g;
 
-      auto merge = [&](uint32_t ge) -> bool {
-        if (!mbar_wait(&bars->pv_full, ge & 1, abort_flag, p.status, lim)) return false;
-        tc_fence_after();
-        const bool need = pend_M != kNegInf && (m_ref == kNegInf || pend_M > m_ref + kRescale);
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? (m_ref == kNegInf ? 0.0f : ex2(m_ref - pend_M)) : 1.0f;
-          const float2 a2 = make_float2(alpha, alpha);
-          l_run *= alpha;
+      // iteration e: the softmax of entry e (if any), then the merge of entry e - 1 (if any)
+      for (int e = 0; e <= n_entries; ++e) {
+        float cur_M = kNegInf, cur_sum = 0.0f;
+        int cur_f16 = 0;
+        if (e < n_entries) {
+          const uint32_t xe = list[e];
+          const int j = xe & 0x1fff, f16 = (xe >> 13) & 1, rm = xe >> 14;
+          const bool part = (rm >> half) & 1;
+          const bool diag = p.causal && (j * BK + BK - 1 > ui.t * kBQ);
+          const float sl2 = f16 ? sl2_16 : sl2_4;
+          const bool dumpP = dbg_unit && e == p.dbg_entry;
+          const uint32_t gv = g0 + e, buf = gv & 1;
+          if (!(ok = mbar_wait(&bars->s_full[buf], (gv >> 1) & 1, abort_flag, p.status, lim))) break;
+          tc_fence_after();
+          const uint32_t tS = tl + L::COL_S + buf * BK;
+          const int k_mine = wg * KH, k_other = KH - k_mine;
+          // the other warpgroup's keys only contribute to the block maximum
+          float M;
+          float sm[KH];
+          {
+            float so[KH];
 #pragma unroll
-          for (int c = 0; c < DW; c += 2) {
-            float2 o = __fmul2_rn(make_float2(O[c], O[c + 1]), a2);
-            O[c] = o.x;
-            O[c + 1] = o.y;
-          }
-          if (need) m_ref = pend_M;
-        }
-        const float gs = (pend_M == kNegInf) ? 0.0f : ex2(pend_M - m_ref);
-        l_run = fmaf(gs, pend_sum, l_run);
-        const float gpv = pend_f16 ? gs : gs * pv4_scale;
-        const float2 g2 = make_float2(gpv, gpv);
-        uint32_t r[DW];
-        tmem_ld<DW>(tmem + lane_base + L::COL_PV + kq * DW, r);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&bars->pv_free);
+            for (int c = 0; c < KH; c += 32)
+              tmem_ld32(tS + k_other + c, *reinterpret_cast<uint32_t(*)[32]>(&so[c]));
+            if constexpr (BK == 128) {
+              tmem_wait_ld();
+              if (diag) mask_causal(so, j * BK + k_other, row);
+              M = row_max<KH>(so);
+            }
 #pragma unroll
-        for (int i = 0; i < DW; i += 2) {
-          float2 o = __ffma2_rn(g2, make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])),
-                                make_float2(O[i], O[i + 1]));
-          O[i] = o.x;
-          O[i + 1] = o.y;
-        }
-        if constexpr (DBG) {
-          if (dbg_unit && (local_e - 1) == p.dbg_entry)
-            for (int i = 0; i < DW; ++i) p.dbg[kBQ * BK + kBQ * (BK / 2) + rr * D + kq * DW + i] = __uint_as_float(r[i]);
-        }
-        return true;
-      };
-
-      const uint32_t lb = unit_ctr & 1;
-      const uint16_t* list = reinterpret_cast<const uint16_t*>(smem + L::OFF_LIST) + lb * L::MAXE;
-      if (!(ok = mbar_wait(&bars->list_full[lb], (unit_ctr >> 1) & 1, abort_flag, p.status, lim))) break;
-      const int n_entries = bars->list_count[lb];
-      for (int e = 0; e < n_entries; ++e) {
-        const uint32_t x = list[e];
-        const int j = x & 0x1fff, f16 = (x >> 13) & 1, rm = x >> 14;
-        const uint32_t buf = g & 1;
-        if (!(ok = mbar_wait(&bars->s_full[buf], (g >> 1) & 1, abort_flag, p.status, lim))) break;
-        tc_fence_after();
-        const bool part = (rm >> half) & 1;
-        const bool diag = p.causal && (j * BK + BK - 1 > ui.t * kBQ);
-        const int key0 = j * BK + kq * KW;  // first key of this warp's columns
-        const float sl2 = f16 ? sl2_16 : sl2_4;
-        const bool dumpP = dbg_unit && local_e == p.dbg_entry;
-        const uint32_t pb = smem_u32(sP + buf * L::PBUF_BYTES);
-
-        // this warp's KW scores of the row: one TMEM round trip, then the buffer goes back
-        float sv[KW];
-        tmem_ld<KW>(tmem + lane_base + L::COL_S + buf * BK + kq * KW, *reinterpret_cast<uint32_t(*)[KW]>(sv));
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&bars->s_free[buf]);
-        if constexpr (DBG) {
-          if (dumpP)
-            for (int i = 0; i < KW; ++i) p.dbg[rr * BK + kq * KW + i] = sv[i];
-        }
-        mask_s(sv, part, diag, key0, row);
-        float gmax[KW / 16];
-        group_max<KW>(sv, gmax);
-        float Mh = gmax[0];
-#pragma unroll
-        for (int q = 1; q < KW / 16; ++q) Mh = fmaxf(Mh, gmax[q]);
-        const float M = exchange(Mh, true);  // the block maximum over the four warps
-        if (!ok) break;
-        const bool valid = M != kNegInf;     // false when every key of the block is masked for this row
-        const float Ms = valid ? M * sl2 : 0.0f;
-
-        // this warp's probabilities, their partial sum, and its part of the PV operand
-        float sum;
-        if (f16) {
-          uint32_t hw[KW / 2];
-          sum = probs_fp16<KW>(sv, sl2, Ms, hw);
-          if constexpr (DBG) {
-            if (dumpP)
-              for (int i = 0; i < KW / 2; ++i) reinterpret_cast<uint32_t*>(p.dbg + kBQ * BK + rr * (BK / 2))[kq * (KW / 2) + i] = hw[i];
-          }
-#pragma unroll
-          for (int q = 0; q < KW / 8; ++q) {
-            const int chunk = kq * (KW / 8) + q;  // 16-byte chunk of the row (8 keys)
-            const int cb = chunk >> 3, c8 = chunk & 7;
-            st_shared_v4(pb + cb * kBQ * 128 + rr * 128 + ((c8 ^ (rr & 7)) << 4), hw[4 * q], hw[4 * q + 1],
-                         hw[4 * q + 2], hw[4 * q + 3]);
-          }
-        } else {
-          uint32_t cw[KW / 8], sfw = 0u;
-          sum = probs_nvfp4<KW / 16>(sv, gmax, sl2, Ms, cw, sfw);
-          if constexpr (DBG) {
-            if (dumpP) {
-              uint8_t* db = reinterpret_cast<uint8_t*>(p.dbg + kBQ * BK + rr * (BK / 2));
-              for (int i = 0; i < KW / 8; ++i) reinterpret_cast<uint32_t*>(db + kq * (KW / 2))[i] = cw[i];
-              for (int q = 0; q < KW / 16; ++q) db[BK / 2 + kq * (KW / 16) + q] = (uint8_t)(sfw >> (8 * q));
+            for (int c = 0; c < KH; c += 32)
+              tmem_ld32(tS + k_mine + c, *reinterpret_cast<uint32_t(*)[32]>(&sm[c]));
+            tmem_wait_ld();
+            if constexpr (BK == 64) {
+              if (diag) mask_causal(so, j * BK + k_other, row);
+              M = row_max<KH>(so);
             }
           }
-          if constexpr (BK == 64) {
-            // 8 code bytes: half of the row's 16-byte chunk kq/2
-            const uint32_t addr = pb + rr * 32 + (((kq >> 1) ^ ((rr >> 2) & 1)) << 4) + 8 * (kq & 1);
-            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(cw[0]), "r"(cw[1]) : "memory");
-            const uint32_t sfa = pb + L::P4_BYTES + (rr & 31) * 16 + (rr >> 5) * 4 + kq;
-            asm volatile("st.shared.b8 [%0], %1;" ::"r"(sfa), "r"(sfw) : "memory");
-          } else {
-            const uint32_t addr = pb + rr * 64 + ((kq ^ ((rr >> 1) & 3)) << 4);
-            st_shared_v4(addr, cw[0], cw[1], cw[2], cw[3]);
-            const uint32_t sfa = pb + L::P4_BYTES + (kq >> 1) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + 2 * (kq & 1);
-            asm volatile("st.shared.b16 [%0], %1;" ::"r"(sfa), "h"((uint16_t)sfw) : "memory");
+          tc_fence_before();
+          mbar_arrive(&bars->s_free[buf]);
+          if constexpr (DBG) {
+            if (dumpP)  // raw scores before masking; the other half comes from the other warpgroup
+              for (int i = 0; i < KH; ++i) p.dbg[rr * BK + k_mine + i] = sm[i];
+          }
+          if (diag) mask_causal(sm, j * BK + k_mine, row);
+          float gm[KH / 16];
+          group_max(sm, gm);
+#pragma unroll
+          for (int q = 0; q < KH / 16; ++q) M = fmaxf(M, gm[q]);
+          // a row outside the entry's query block (64-row query blocks) takes no part: all of its
+          // group maxima become -inf, which zeroes its codes, its FP16 probabilities and its sum
+          if (!part) {
+            M = kNegInf;
+#pragma unroll
+            for (int q = 0; q < KH / 16; ++q) gm[q] = kNegInf;
+          }
+          const bool valid = M != kNegInf;  // false when every key of the block is masked for this row
+          const float Ms = valid ? M * sl2 : __builtin_huge_valf();
+
+          // this warpgroup's probabilities, 32 keys at a time, into PV operand buffer `buf`; its
+          // previous reader, the PV product of entry e - 2, finished before that entry's merge
+          const uint32_t pb = smem_u32(smem + L::OFF_P + buf * L::PBUF);
+          float sum = 0.0f;
+#pragma unroll
+          for (int c = 0; c < KH; c += 32) {
+            const int k0 = k_mine + c;  // first key of this chunk within the block
+            const float(&sc)[32] = *reinterpret_cast<const float(*)[32]>(&sm[c]);
+            if (f16) {
+              uint32_t* dbw = nullptr;
+              if constexpr (DBG) {
+                if (dumpP) dbw = reinterpret_cast<uint32_t*>(p.dbg + kBQ * BK + rr * (BK / 2)) + k0 / 2;
+              }
+              sum += probs_fp16_32(sc, sl2, Ms, pb + (k0 >> 6) * kBQ * 128 + rr * 128, (k0 & 63) >> 3, rr & 7, dbw);
+            } else {
+              uint32_t cw[4], sf2 = 0u;
+              sum += probs_nvfp4_32(sc, gm + c / 16, sl2, Ms, cw, sf2);
+              const int q = k0 >> 5;  // 16-byte chunk of the row's codes
+              const uint32_t addr = BK == 64 ? pb + rr * 32 + ((q ^ ((rr >> 2) & 1)) << 4)
+                                             : pb + rr * 64 + ((q ^ ((rr >> 1) & 3)) << 4);
+              st_shared_v4(addr, cw[0], cw[1], cw[2], cw[3]);
+              const int g16 = k0 >> 4;  // first 16-key group of the chunk
+              asm volatile("st.shared.b16 [%0], %1;" ::"r"(pb + L::P4_BYTES + (g16 >> 2) * 512 + (rr & 31) * 16 +
+                                                            (rr >> 5) * 4 + (g16 & 3)),
+                           "h"((uint16_t)sf2)
+                           : "memory");
+              if constexpr (DBG) {
+                if (dumpP) {
+                  uint8_t* db = reinterpret_cast<uint8_t*>(p.dbg + kBQ * BK + rr * (BK / 2));
+                  for (int i = 0; i < 4; ++i) reinterpret_cast<uint32_t*>(db)[(k0 >> 3) + i] = cw[i];
+                  db[BK / 2 + g16] = (uint8_t)sf2;
+                  db[BK / 2 + g16 + 1] = (uint8_t)(sf2 >> 8);
+                }
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&bars->p_full[buf]);
+          cur_M = valid ? Ms : kNegInf;
+          cur_sum = sum;
+          cur_f16 = f16;
+        }
+        if (e > 0) {
+          // merge entry e - 1: its PV product into this warpgroup's output columns with weight
+          // exp2(pend_M - m_ref)
+          const uint32_t v = g0 + e - 1;
+          const uint32_t pvb = L::NPV == 2 ? (v & 1) : 0;
+          const uint32_t par = L::NPV == 2 ? ((v >> 1) & 1) : (v & 1);
+          if (!(ok = mbar_wait(&bars->pv_full[pvb], par, abort_flag, p.status, lim))) break;
+          tc_fence_after();
+          const bool need = pend_M != kNegInf && (m_ref == kNegInf || pend_M > m_ref + kRescale);
+          if (__any_sync(0xffffffffu, need)) {
+            const float alpha = need ? (m_ref == kNegInf ? 0.0f : ex2(m_ref - pend_M)) : 1.0f;
+            const float2 a2 = make_float2(alpha, alpha);
+            l_run *= alpha;
+#pragma unroll
+            for (int c = 0; c < DH; c += 2) {
+              const float2 o = __fmul2_rn(make_float2(O[c], O[c + 1]), a2);
+              O[c] = o.x;
+              O[c + 1] = o.y;
+            }
+            if (need) m_ref = pend_M;
+          }
+          const float gs = (pend_M == kNegInf) ? 0.0f : ex2(pend_M - m_ref);
+          l_run = fmaf(gs, pend_sum, l_run);
+          const float gpv = pend_f16 ? gs : gs * pv4_scale;
+          const float2 g2 = make_float2(gpv, gpv);
+          uint32_t r[DH];
+#pragma unroll
+          for (int c = 0; c < DH; c += 32)
+            tmem_ld32(tl + L::COL_PV + pvb * D + wg * DH + c, *reinterpret_cast<uint32_t(*)[32]>(&r[c]));
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(&bars->pv_free[pvb]);
+#pragma unroll
+          for (int i = 0; i < DH; i += 2) {
+            const float2 o = __ffma2_rn(g2, make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])),
+                                        make_float2(O[i], O[i + 1]));
+            O[i] = o.x;
+            O[i + 1] = o.y;
+          }
+          if constexpr (DBG) {
+            if (dbg_unit && e - 1 == p.dbg_entry)
+              for (int i = 0; i < DH; ++i) p.dbg[kBQ * BK + kBQ * (BK / 2) + rr * D + wg * DH + i] = __uint_as_float(r[i]);
           }
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&bars->p_full[buf]);
-        if (have_pend && !(ok = merge(g - 1))) break;
-        pend_M = valid ? Ms : kNegInf;
-        pend_sum = sum;
-        pend_f16 = f16;
-        have_pend = true;
-        ++g;
-        ++local_e;
+        pend_M = cur_M;
+        pend_sum = cur_sum;
+        pend_f16 = cur_f16;
       }
-      if (ok && have_pend) ok = merge(g - 1);
       if (!ok) break;
+      g = g0 + n_entries;
       mbar_arrive(&bars->list_empty[lb]);
-      // combine the four warps' partial denominators
-      const float l_tot = exchange(l_run, false);
-      if (!ok) break;
-      // epilogue: O / l in FP16, lse in natural-log units of the tau-scaled scores
+      // the two warpgroups' partial denominators (same m_ref in both), then the epilogue:
+      // O / l in FP16, lse in natural-log units of the tau-scaled scores
+      bars->lx[lb][wg][rr] = l_run;
+      mbar_arrive(&bars->lx_bar[lb]);
+      if (!(ok = mbar_wait(&bars->lx_bar[lb], lph, abort_flag, p.status, lim))) break;
+      const float l_tot = bars->lx[lb][0][rr] + bars->lx[lb][1][rr];
       const float inv_l = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
       const int64_t orow = (int64_t)(ui.b * p.Hq + ui.h) * p.N + row;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D + kq * DW);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D + wg * DH);
 #pragma unroll
-      for (int c = 0; c < DW / 8; ++c) {
+      for (int c = 0; c < DH / 8; ++c) {
         uint4 v;
         v.x = pack_half2(O[8 * c] * inv_l, O[8 * c + 1] * inv_l);
         v.y = pack_half2(O[8 * c + 2] * inv_l, O[8 * c + 3] * inv_l);
@@ -816,7 +880,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         v.w = pack_half2(O[8 * c + 6] * inv_l, O[8 * c + 7] * inv_l);
         dst[c] = v;
       }
-      if (p.lse && kq == 0) p.lse[orow] = (m_ref + __log2f(l_tot)) * kLn2;
+      if (p.lse && wg == 0) p.lse[orow] = (m_ref + __log2f(l_tot)) * kLn2;
     }
   }
 
@@ -868,6 +932,19 @@ template <int D, int BK>
 thrift_status launch_t(const void* q, const void* k, const void* v, const thrift_nvfp4* q4, const thrift_nvfp4* k4,
                        const thrift_nvfp4* v4, AttnParams& prm, cudaStream_t stream) {
   using L = Layout<D, BK>;
+  // entry lists: [unit parity][maxe] u16 after the barrier block; the rest goes to pages
+  prm.maxe = (prm.bq == 64 ? 2 : 1) * prm.nkb;
+  const int list_bytes = (2 * prm.maxe * 2 + 1023) & ~1023;
+  const int room = kSmemLimit - L::fixed_bytes() - list_bytes;
+  int npage = room / L::PAGE;
+  if (npage > kMaxPages) npage = kMaxPages;
+  if (npage < 3) return THRIFT_ERR_UNSUPPORTED;
+  prm.npage = npage;
+  prm.off_bar = L::OFF_PAGES + npage * L::PAGE;
+  prm.off_list = prm.off_bar + L::BAR_BYTES;
+  const int smem_bytes = prm.off_list + list_bytes + 1024;
+  prm.n_units = prm.B * prm.Hq * (prm.N / kBQ);
+
   CUtensorMap maps[6];
   memset(maps, 0, sizeof(maps));
   const uint64_t qrows = (uint64_t)prm.B * prm.Hq * prm.N, krows = (uint64_t)prm.B * prm.Hkv * prm.N;
@@ -885,11 +962,18 @@ thrift_status launch_t(const void* q, const void* k, const void* v, const thrift
   }
   if (!ok) return THRIFT_ERR_CUDA;
   auto kern = prm.dbg ? attn_kernel<D, BK, true> : attn_kernel<D, BK, false>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES) != cudaSuccess)
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
     return THRIFT_ERR_CUDA;
+  {
+    // setmaxnreg.inc waits until the registers it asks for are free in the CTA's launch
+    // allocation; refuse to launch unless the split fits that allocation.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return THRIFT_ERR_CUDA;
+    if ((long)fa.numRegs * L::THREADS < 128L * kProducerRegs + 256L * kSoftmaxRegs) return THRIFT_ERR_UNSUPPORTED;
+  }
   int grid = num_sms();
   if (grid > prm.n_units) grid = prm.n_units;
-  kern<<<grid, kThreads, L::BYTES, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], prm);
+  kern<<<grid, L::THREADS, smem_bytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], prm);
   return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 
@@ -938,9 +1022,8 @@ thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const
   prm.nqb = c.N / c.block_q;
   prm.nkb = c.N / c.block_k;
   prm.mask_words = (prm.nkb + 31) / 32;
-  prm.n_units = c.B * c.Hq * (c.N / kBQ);
   prm.tau = c.softmax_scale > 0.0f ? c.softmax_scale : 1.0f / sqrtf((float)c.d);
-  if (2 * prm.nkb > 4096) return THRIFT_ERR_UNSUPPORTED;  // the per-unit entry list holds 4096 entries
+  if (prm.nkb > 8191) return THRIFT_ERR_UNSUPPORTED;  // key-block index field of an entry
   prm.wait_limit = kWaitLimit;
   if (c.d == 128 && c.block_k == 64) return launch_t<128, 64>(q, k, v, q4, k4, v4, prm, stream);
   if (c.d == 128 && c.block_k == 128) return launch_t<128, 128>(q, k, v, q4, k4, v4, prm, stream);

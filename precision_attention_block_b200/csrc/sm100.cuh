@@ -59,7 +59,8 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 }
 
 // Bounded wait for the phase with the given parity.  Gives up after `limit` clock cycles,
-// records the timeout in the global status word and raises the CTA's abort flag (a shared flag:
+// records the timeout in the global status word (and, in the word after it, which wait gave up
+// first) and raises the CTA's abort flag (a shared flag:
 // once any wait of the CTA gives up, every later wait returns at once, so that all warps reach
 // the kernel's end, release TMEM and exit).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -71,7 +72,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
     if (clock64() - t0 > limit) {
       *abort_flag = 1;
-      if (status) atomicOr(status, kStatusTimeout);
+      if (status) {
+        atomicOr(status, kStatusTimeout);
+        // the first wait to give up: warp, parity and shared-memory address of its barrier
+        atomicCAS(status + 1, 0, (int)(((threadIdx.x >> 5) << 24) | (parity << 23) | (smem_u32(bar) & 0x7FFFFF)));
+      }
       return false;
     }
   }
