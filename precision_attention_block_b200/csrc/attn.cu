@@ -100,7 +100,9 @@ struct Layout {
 
 struct Bars {
   uint64_t q4_full, q4_empty, q16_full, q16_empty;
-  uint64_t s_full[2], s_free[2], p_full[2], pv_full[2], pv_free[2];
+  uint64_t ready[2];  // visit v: S(v) = Q K^T and the PV product of visit v - LAG are in TMEM (one
+                      // commit from each issuer)
+  uint64_t s_free[2], p_full[2];  // score buffer read, PV operand written (both softmax warpgroups)
   uint64_t list_full[2], list_empty[2];  // by unit parity
   uint64_t lx_bar[2];                    // the two softmax warpgroups swap their denominators
   uint64_t page_full[kMaxPages], page_empty[kMaxPages];
@@ -212,36 +214,12 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-__device__ __forceinline__ float lg2(float x) {
-  float y;
-  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// 2^x for a pair of values on the FMA pipe: x = n + f with n = round(x) (by the 1.5 * 2^23
-// rounding constant) and f in [-1/2, 1/2]; 2^f by a degree-5 polynomial (a relative-error minimax
-// fit on [-1/2, 1/2]; relative error below 2.2e-7 including FP32 rounding, about that of the
-// MUFU ex2 approximation, so the E2M1 code decisions of the two paths agree as often); n is added
-// to the exponent field.  Inputs are clamped at -125 so that the result stays a normal number
-// (2^-125 is far below anything that can change a sum or a code).
-__device__ __forceinline__ float2 ex2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
-  const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
-  const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
-  float2 q = __ffma2_rn(make_float2(0.0013276473619043827f, 0.0013276473619043827f), f,
-                        make_float2(0.009675541892647743f, 0.009675541892647743f));
-  q = __ffma2_rn(q, f, make_float2(0.05550713092088699f, 0.05550713092088699f));
-  q = __ffma2_rn(q, f, make_float2(0.24022120237350464f, 0.24022120237350464f));
-  q = __ffma2_rn(q, f, make_float2(0.6931469440460205f, 0.6931469440460205f));
-  q = __ffma2_rn(q, f, make_float2(1.0000001192092896f, 1.0000001192092896f));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
-}
-
-// exp2 of a pair of keys; `pair` is the pair's index within its 16-key group (a constant after
-// unrolling): pairs at or past (16 - kPolyPerGroup) / 2 use the polynomial, the others MUFU.
+// 2^x on the FMA pipe: x = n + f with n = round(x) (by the 1.5 * 2^23 rounding constant) and f in
+// [-1/2, 1/2]; 2^f by a degree-5 polynomial (a relative-error minimax fit on [-1/2, 1/2]; relative
+// error below 2.2e-7 including FP32 rounding, about that of the MUFU ex2 approximation, so the
+// E2M1 code decisions of the two paths agree as often); n is added to the exponent field.  Inputs
+// are clamped at -125 so that the result stays a normal number (2^-125 is far below anything that
+// can change a sum or a code).
 __device__ __forceinline__ float ex2_poly1(float x) {
   x = fmaxf(x, -125.0f);
   const float t = x + 12582912.0f;
@@ -258,6 +236,12 @@ __device__ __forceinline__ float ex2_poly1(float x) {
 __device__ __forceinline__ float2 ex2_pair(float2 x, int pair) {
   if (2 * pair >= 16 - kPolyPerGroup) return make_float2(ex2_poly1(x.x), ex2_poly1(x.y));
   return make_float2(ex2(x.x), ex2(x.y));
+}
+
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
@@ -415,11 +399,9 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&bars->q16_full, 1);
     mbar_init(&bars->q16_empty, 1);
     for (int x = 0; x < 2; ++x) {
-      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->ready[x], 2);
       mbar_init(&bars->s_free[x], 256);
       mbar_init(&bars->p_full[x], 256);
-      mbar_init(&bars->pv_full[x], 1);
-      mbar_init(&bars->pv_free[x], 256);
       mbar_init(&bars->list_full[x], 1);
       mbar_init(&bars->list_empty[x], 2 + 256);
       mbar_init(&bars->lx_bar[x], 256);
@@ -529,13 +511,15 @@ __global__ void __launch_bounds__(384, 1)
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------------- QK^T issuer
+      // S = Q K^T of every visit v (a global visit counter over this CTA's units), then its commit
+      // to ready[v & 1]; the PV issuer makes the other arrival.
       if (lane == 0) {
         const uint32_t idesc_qk4 = idesc_nvf4(kBQ, BK);
         const uint32_t idesc_qk16 = idesc_f16(kBQ, BK, 0, 0);
         constexpr int SWQ = swz_for_row_bytes(D / 2);
         const uint32_t qb4 = smem_u32(smem + L::OFF_Q4), qb16 = smem_u32(smem + L::OFF_Q16);
         PageRing ring{0, 0, p.npage};
-        uint32_t uc = 0, u16c = 0, g = 0;
+        uint32_t uc = 0, u16c = 0, v = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
           const UnitInfo ui = decode_unit(p, u);
@@ -552,7 +536,7 @@ __global__ void __launch_bounds__(384, 1)
               tc_copy_sf(tmem + L::COL_SFQ + 4 * kk, make_sdesc(qb4 + L::Q4_BYTES + kk * 512, 16, 128, 0));
           }
           bool released4 = false, any16 = false;
-          for (int e = 0; e < n && ok; ++e) {
+          for (int e = 0; e < n && ok; ++e, ++v) {
             const uint32_t xe = list[e];
             const int j = xe & 0x1fff, f16 = (xe >> 13) & 1;
             if (f16 && !released4) {
@@ -564,12 +548,12 @@ __global__ void __launch_bounds__(384, 1)
               ++u16c;
               any16 = true;
             }
-            int pk, phk, pv = 0, phv = 0;
+            int pk, phk, pv, phv;
             ring.next(pk, phk);
             if (f16) ring.next(pv, phv);
-            const uint32_t buf = g & 1;
+            const uint32_t buf = v & 1;
             if (!(ok = mbar_wait(&bars->page_full[pk], phk, abort_flag, p.status, lim))) break;
-            if (!(ok = mbar_wait(&bars->s_free[buf], ((g >> 1) & 1) ^ 1, abort_flag, p.status, lim))) break;
+            if (!(ok = mbar_wait(&bars->s_free[buf], ((v >> 1) & 1) ^ 1, abort_flag, p.status, lim))) break;
             tc_fence_after();
             const uint32_t kbuf = smem_u32(smem + L::OFF_PAGES + pk * L::PAGE);
             const uint32_t dS = tmem + L::COL_S + buf * BK;
@@ -593,25 +577,79 @@ __global__ void __launch_bounds__(384, 1)
                 mma_nvf4(dS, ad, bd, idesc_qk4, tmem + L::COL_SFQ + 4 * kk, sfk + 4 * kk + sfk_off, kk > 0);
               }
             }
-            tc_commit(&bars->s_full[buf]);
             tc_commit(&bars->page_empty[pk]);  // the V page of an FP16 entry is the PV issuer's
-            ++g;
+            tc_commit(&bars->ready[buf]);
           }
           if (!ok) break;
           if (!released4) tc_commit(&bars->q4_empty);
           if (any16) tc_commit(&bars->q16_empty);
           mbar_arrive(&bars->list_empty[lb]);
         }
+        // the ready phases of the visits after the last one (the softmax warpgroups' last merges);
+        // each arrival waits for the barrier's previous phase, so that it cannot complete that one
+        for (int d = 0; d < L::NPV && ok; ++d, ++v) {
+          if (!(ok = mbar_wait(&bars->ready[v & 1], ((v >> 1) & 1) ^ 1, abort_flag, p.status, lim))) break;
+          mbar_arrive(&bars->ready[v & 1]);
+        }
       }
     } else if (warp == 2) {
       // ---------------------------------------------------------------- PV issuer
+      // For every visit v: the PV product of visit v - LAG, then its commit to ready[v & 1].  The
+      // product lags LAG visits behind S so that the softmax warpgroups merge it one iteration
+      // after it was issued.  LAG more iterations after the last unit issue the remaining ones.
       if (lane == 0) {
+        constexpr int LAG = L::NPV;
         const uint32_t idesc_pv4 = idesc_nvf4(kBQ, D);
         const uint32_t idesc_pv16 = idesc_f16(kBQ, D, 0, 1);
         constexpr int SWP = swz_for_row_bytes(BK / 2);
+        // entry parameters of the visits whose products are still to be issued, by visit parity
+        int pf16[2] = {0, 0}, ppk[2] = {0, 0}, ppv[2] = {0, 0}, pphv[2] = {0, 0}, psfv[2] = {0, 0};
         PageRing ring{0, 0, p.npage};
-        uint32_t uc = 0, g = 0;
+        uint32_t uc = 0, v = 0;
         bool ok = true;
+        auto issue_pv = [&](uint32_t w) -> bool {
+          const uint32_t buf = w & 1;
+          const int f16 = buf ? pf16[1] : pf16[0];
+          const int pk = buf ? ppk[1] : ppk[0], pv = buf ? ppv[1] : ppv[0];
+          const int phv = buf ? pphv[1] : pphv[0], sfv_off = buf ? psfv[1] : psfv[0];
+          const uint32_t pvb = LAG == 2 ? buf : 0;
+          if (!mbar_wait(&bars->p_full[buf], (w >> 1) & 1, abort_flag, p.status, lim)) return false;
+          if (!mbar_wait(&bars->page_full[pv], phv, abort_flag, p.status, lim)) return false;
+          tc_fence_after();
+          const uint32_t pbuf = smem_u32(smem + L::OFF_P + buf * L::PBUF);
+          const uint32_t vpage = smem_u32(smem + L::OFF_PAGES + pv * L::PAGE);
+          const uint32_t dPV = tmem + L::COL_PV + pvb * D;
+          if (f16) {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = make_sdesc(pbuf + (kk >> 2) * kBQ * 128 + (kk & 3) * 32, 16, 1024, kSW128);
+              const uint64_t bd = make_sdesc(vpage + kk * 16 * 128, BK * 128, 1024, kSW128);
+              mma_f16(dPV, ad, bd, idesc_pv16, kk > 0);
+            }
+            // Both arrivals of the V page come from here, after its page_full wait: an arrival
+            // issued before the page holds this entry's tile could complete the phase of the
+            // page's previous use.  The K page gets the QK^T commit and this arrival.
+            mbar_arrive(&bars->page_empty[pk]);
+            mbar_arrive(&bars->page_empty[pv]);
+            tc_commit(&bars->page_empty[pv]);
+          } else {
+            const uint32_t vbuf = vpage + L::V4_OFF;
+            const uint32_t sfv = tmem + L::COL_SFV + buf * L::SFV, sfp = tmem + L::COL_SFP + buf * L::SFV;
+#pragma unroll
+            for (int kb = 0; kb < BK / 64; ++kb) {
+              tc_copy_sf(sfv + 4 * kb, make_sdesc(vbuf + L::V4_BYTES + kb * 512, 16, 128, 0));
+              tc_copy_sf(sfp + 4 * kb, make_sdesc(pbuf + L::P4_BYTES + kb * 512, 16, 128, 0));
+            }
+#pragma unroll
+            for (int kb = 0; kb < BK / 64; ++kb) {
+              const uint64_t ad = make_sdesc(pbuf + kb * 32, 16, 8 * (BK / 2), SWP);
+              const uint64_t bd = make_sdesc(vbuf + kb * 32, 16, 8 * (BK / 2), SWP);
+              mma_nvf4(dPV, ad, bd, idesc_pv4, sfp + 4 * kb, sfv + 4 * kb + sfv_off, kb > 0);
+            }
+            tc_commit(&bars->page_empty[pv]);  // the QK^T commit was the page's other arrival
+          }
+          return true;
+        };
         for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
           const UnitInfo ui = decode_unit(p, u);
           const int sfv_off = (((ui.b * p.Hkv + ui.hk) * D) & 127) >> 5;
@@ -619,59 +657,29 @@ __global__ void __launch_bounds__(384, 1)
           if (!(ok = mbar_wait(&bars->list_full[lb], lph, abort_flag, p.status, lim))) break;
           const int n = bars->list_count[lb];
           const uint16_t* list = lists + lb * p.maxe;
-          for (int e = 0; e < n && ok; ++e) {
+          for (int e = 0; e < n && ok; ++e, ++v) {
+            if (v >= (uint32_t)LAG && !(ok = issue_pv(v - LAG))) break;
+            tc_commit(&bars->ready[v & 1]);
             const int f16 = (list[e] >> 13) & 1;
-            int pk, phk, pv = 0, phv = 0;
+            int pk, phk, pv, phv;
             ring.next(pk, phk);
+            pv = pk;
+            phv = phk;
             if (f16) ring.next(pv, phv);
-            const int pgv = f16 ? pv : pk, phv_ = f16 ? phv : phk;
-            const uint32_t buf = g & 1;
-            const uint32_t pvb = L::NPV == 2 ? buf : 0;
-            const uint32_t pv_par = L::NPV == 2 ? (((g >> 1) & 1) ^ 1) : ((g & 1) ^ 1);
-            if (!(ok = mbar_wait(&bars->p_full[buf], (g >> 1) & 1, abort_flag, p.status, lim))) break;
-            if (!(ok = mbar_wait(&bars->pv_free[pvb], pv_par, abort_flag, p.status, lim))) break;
-            if (!(ok = mbar_wait(&bars->page_full[pgv], phv_, abort_flag, p.status, lim))) break;
-            tc_fence_after();
-            const uint32_t pbuf = smem_u32(smem + L::OFF_P + buf * L::PBUF);
-            const uint32_t vpage = smem_u32(smem + L::OFF_PAGES + pgv * L::PAGE);
-            const uint32_t dPV = tmem + L::COL_PV + pvb * D;
-            if (f16) {
-#pragma unroll
-              for (int kk = 0; kk < BK / 16; ++kk) {
-                const uint64_t ad = make_sdesc(pbuf + (kk >> 2) * kBQ * 128 + (kk & 3) * 32, 16, 1024, kSW128);
-                const uint64_t bd = make_sdesc(vpage + kk * 16 * 128, BK * 128, 1024, kSW128);
-                mma_f16(dPV, ad, bd, idesc_pv16, kk > 0);
-              }
+            const int k = v & 1;
+            if (k) {
+              pf16[1] = f16; ppk[1] = pk; ppv[1] = pv; pphv[1] = phv; psfv[1] = sfv_off;
             } else {
-              const uint32_t vbuf = vpage + L::V4_OFF;
-              const uint32_t sfv = tmem + L::COL_SFV + buf * L::SFV, sfp = tmem + L::COL_SFP + buf * L::SFV;
-#pragma unroll
-              for (int kb = 0; kb < BK / 64; ++kb) {
-                tc_copy_sf(sfv + 4 * kb, make_sdesc(vbuf + L::V4_BYTES + kb * 512, 16, 128, 0));
-                tc_copy_sf(sfp + 4 * kb, make_sdesc(pbuf + L::P4_BYTES + kb * 512, 16, 128, 0));
-              }
-#pragma unroll
-              for (int kb = 0; kb < BK / 64; ++kb) {
-                const uint64_t ad = make_sdesc(pbuf + kb * 32, 16, 8 * (BK / 2), SWP);
-                const uint64_t bd = make_sdesc(vbuf + kb * 32, 16, 8 * (BK / 2), SWP);
-                mma_nvf4(dPV, ad, bd, idesc_pv4, sfp + 4 * kb, sfv + 4 * kb + sfv_off, kb > 0);
-              }
+              pf16[0] = f16; ppk[0] = pk; ppv[0] = pv; pphv[0] = phv; psfv[0] = sfv_off;
             }
-            tc_commit(&bars->pv_full[pvb]);
-            if (f16) {
-              // Both arrivals of the V page come from here, after its page_full wait: an arrival
-              // issued before the page holds this entry's tile could complete the phase of the
-              // page's previous use.  The K page gets the QK^T issuer's commit and this arrival.
-              mbar_arrive(&bars->page_empty[pk]);
-              mbar_arrive(&bars->page_empty[pv]);
-              tc_commit(&bars->page_empty[pv]);
-            } else {
-              tc_commit(&bars->page_empty[pk]);
-            }
-            ++g;
           }
           if (!ok) break;
           mbar_arrive(&bars->list_empty[lb]);
+        }
+        // the last LAG PV products (and the ready phases the softmax warpgroups wait for)
+        for (int d = 0; d < LAG && ok; ++d, ++v) {
+          if (v >= (uint32_t)LAG && !(ok = issue_pv(v - LAG))) break;
+          tc_commit(&bars->ready[v & 1]);
         }
       }
     }
@@ -705,15 +713,60 @@ __global__ void __launch_bounds__(384, 1)
       // maximum exceeds it by more than 2^kRescale (the final O / l does not depend on m_ref).
       // Both warpgroups see the same block maxima, so they take the same decisions.
       float m_ref = kNegInf, l_run = 0.0f;
-      float pend_M = kNegInf, pend_sum = 0.0f;
-      int pend_f16 = 0;
+      // block maximum (log2 units; -inf: the row took no part), unquantised sum and precision of
+      // the entries whose PV products are still to be merged, by entry parity
+      float pend_M[2] = {kNegInf, kNegInf}, pend_sum[2] = {0.0f, 0.0f};
+      int pend_f16[2] = {0, 0};
       const bool dbg_unit = DBG && p.dbg && blockIdx.x == 0 && u == (int)blockIdx.x;
       const uint32_t g0 = g;
+      constexpr int LAG = L::NPV;
 
-      // iteration e: the softmax of entry e (if any), then the merge of entry e - 1 (if any)
-      for (int e = 0; e <= n_entries; ++e) {
-        float cur_M = kNegInf, cur_sum = 0.0f;
-        int cur_f16 = 0;
+      // iteration e: wait for ready(v) (S of entry e and the PV product of entry e - LAG), merge
+      // that PV product, then the softmax of entry e; LAG more iterations merge the last entries
+      for (int e = 0; e < n_entries + LAG; ++e) {
+        const uint32_t v = g0 + e, buf = v & 1;
+        if (!(ok = mbar_wait(&bars->ready[buf], (v >> 1) & 1, abort_flag, p.status, lim))) break;
+        tc_fence_after();
+        if (e >= LAG) {
+          // merge entry e - LAG: its PV product into this warpgroup's output columns with weight
+          // exp2(pend_M - m_ref)
+          const int pe = (e - LAG) & 1;
+          const float pM = pend_M[pe];
+          const uint32_t pvb = LAG == 2 ? buf : 0;
+          const bool need = pM != kNegInf && (m_ref == kNegInf || pM > m_ref + kRescale);
+          if (__any_sync(0xffffffffu, need)) {
+            const float alpha = need ? (m_ref == kNegInf ? 0.0f : ex2(m_ref - pM)) : 1.0f;
+            const float2 a2 = make_float2(alpha, alpha);
+            l_run *= alpha;
+#pragma unroll
+            for (int c = 0; c < DH; c += 2) {
+              const float2 o = __fmul2_rn(make_float2(O[c], O[c + 1]), a2);
+              O[c] = o.x;
+              O[c + 1] = o.y;
+            }
+            if (need) m_ref = pM;
+          }
+          const float gs = (pM == kNegInf) ? 0.0f : ex2(pM - m_ref);
+          l_run = fmaf(gs, pend_sum[pe], l_run);
+          const float gpv = pend_f16[pe] ? gs : gs * pv4_scale;
+          const float2 g2 = make_float2(gpv, gpv);
+          uint32_t r[DH];
+#pragma unroll
+          for (int c = 0; c < DH; c += 32)
+            tmem_ld32(tl + L::COL_PV + pvb * D + wg * DH + c, *reinterpret_cast<uint32_t(*)[32]>(&r[c]));
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < DH; i += 2) {
+            const float2 o = __ffma2_rn(g2, make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])),
+                                        make_float2(O[i], O[i + 1]));
+            O[i] = o.x;
+            O[i + 1] = o.y;
+          }
+          if constexpr (DBG) {
+            if (dbg_unit && e - LAG == p.dbg_entry)
+              for (int i = 0; i < DH; ++i) p.dbg[kBQ * BK + kBQ * (BK / 2) + rr * D + wg * DH + i] = __uint_as_float(r[i]);
+          }
+        }
         if (e < n_entries) {
           const uint32_t xe = list[e];
           const int j = xe & 0x1fff, f16 = (xe >> 13) & 1, rm = xe >> 14;
@@ -721,9 +774,6 @@ __global__ void __launch_bounds__(384, 1)
           const bool diag = p.causal && (j * BK + BK - 1 > ui.t * kBQ);
           const float sl2 = f16 ? sl2_16 : sl2_4;
           const bool dumpP = dbg_unit && e == p.dbg_entry;
-          const uint32_t gv = g0 + e, buf = gv & 1;
-          if (!(ok = mbar_wait(&bars->s_full[buf], (gv >> 1) & 1, abort_flag, p.status, lim))) break;
-          tc_fence_after();
           const uint32_t tS = tl + L::COL_S + buf * BK;
           const int k_mine = wg * KH, k_other = KH - k_mine;
           // the other warpgroup's keys only contribute to the block maximum
@@ -767,10 +817,10 @@ __global__ void __launch_bounds__(384, 1)
             for (int q = 0; q < KH / 16; ++q) gm[q] = kNegInf;
           }
           const bool valid = M != kNegInf;  // false when every key of the block is masked for this row
-          const float Ms = valid ? M * sl2 : __builtin_huge_valf();
+          const float Ms = valid ? M * sl2 : __builtin_huge_valf();  // +inf zeroes every probability
 
           // this warpgroup's probabilities, 32 keys at a time, into PV operand buffer `buf`; its
-          // previous reader, the PV product of entry e - 2, finished before that entry's merge
+          // previous reader, the PV product of entry e - 2, has completed (ready(v) covers it)
           const uint32_t pb = smem_u32(smem + L::OFF_P + buf * L::PBUF);
           float sum = 0.0f;
 #pragma unroll
@@ -805,59 +855,15 @@ __global__ void __launch_bounds__(384, 1)
               }
             }
           }
+          // the TMEM reads of this iteration's merge are complete (tcgen05.wait::ld above), so
+          // this arrival also releases the PV buffer for the product of entry e
+          tc_fence_before();
           fence_proxy_async_smem();
           mbar_arrive(&bars->p_full[buf]);
-          cur_M = valid ? Ms : kNegInf;
-          cur_sum = sum;
-          cur_f16 = f16;
+          pend_M[e & 1] = valid ? Ms : kNegInf;
+          pend_sum[e & 1] = sum;
+          pend_f16[e & 1] = f16;
         }
-        if (e > 0) {
-          // merge entry e - 1: its PV product into this warpgroup's output columns with weight
-          // exp2(pend_M - m_ref)
-          const uint32_t v = g0 + e - 1;
-          const uint32_t pvb = L::NPV == 2 ? (v & 1) : 0;
-          const uint32_t par = L::NPV == 2 ? ((v >> 1) & 1) : (v & 1);
-          if (!(ok = mbar_wait(&bars->pv_full[pvb], par, abort_flag, p.status, lim))) break;
-          tc_fence_after();
-          const bool need = pend_M != kNegInf && (m_ref == kNegInf || pend_M > m_ref + kRescale);
-          if (__any_sync(0xffffffffu, need)) {
-            const float alpha = need ? (m_ref == kNegInf ? 0.0f : ex2(m_ref - pend_M)) : 1.0f;
-            const float2 a2 = make_float2(alpha, alpha);
-            l_run *= alpha;
-#pragma unroll
-            for (int c = 0; c < DH; c += 2) {
-              const float2 o = __fmul2_rn(make_float2(O[c], O[c + 1]), a2);
-              O[c] = o.x;
-              O[c + 1] = o.y;
-            }
-            if (need) m_ref = pend_M;
-          }
-          const float gs = (pend_M == kNegInf) ? 0.0f : ex2(pend_M - m_ref);
-          l_run = fmaf(gs, pend_sum, l_run);
-          const float gpv = pend_f16 ? gs : gs * pv4_scale;
-          const float2 g2 = make_float2(gpv, gpv);
-          uint32_t r[DH];
-#pragma unroll
-          for (int c = 0; c < DH; c += 32)
-            tmem_ld32(tl + L::COL_PV + pvb * D + wg * DH + c, *reinterpret_cast<uint32_t(*)[32]>(&r[c]));
-          tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(&bars->pv_free[pvb]);
-#pragma unroll
-          for (int i = 0; i < DH; i += 2) {
-            const float2 o = __ffma2_rn(g2, make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])),
-                                        make_float2(O[i], O[i + 1]));
-            O[i] = o.x;
-            O[i + 1] = o.y;
-          }
-          if constexpr (DBG) {
-            if (dbg_unit && e - 1 == p.dbg_entry)
-              for (int i = 0; i < DH; ++i) p.dbg[kBQ * BK + kBQ * (BK / 2) + rr * D + wg * DH + i] = __uint_as_float(r[i]);
-          }
-        }
-        pend_M = cur_M;
-        pend_sum = cur_sum;
-        pend_f16 = cur_f16;
       }
       if (!ok) break;
       g = g0 + n_entries;
