@@ -44,7 +44,11 @@ constexpr int kMaxPages = 8;
 constexpr int kSmemLimit = 232448;  // largest dynamic shared memory of one CTA on sm_100
 constexpr int kProducerRegs = 56, kSoftmaxRegs = 224;  // setmaxnreg split (384 threads x 168 at launch)
 constexpr float kNegInf = -__builtin_huge_valf();
-constexpr float kRescale = 8.0f;  // log2 units: rescale O only when the block max grows past 256x
+// log2 units: O and l are rescaled only when a block maximum exceeds the reference maximum by more
+// than 2^32.  Until then every weight exp2(M - m_ref) is at most 2^32, so with at most 2^13 key
+// blocks of at most 128 keys and |V| < 2^16 the FP32 sums stay below 2^68, far from overflow, and
+// FP32 keeps its relative precision at any scale.
+constexpr float kRescale = 32.0f;
 constexpr int kPolyPerGroup = 4;  // exponentials per 16 keys evaluated by the polynomial
 
 __host__ __device__ constexpr int round1024(int x) { return (x + 1023) & ~1023; }
@@ -714,9 +718,9 @@ __global__ void __launch_bounds__(384, 1)
       // Both warpgroups see the same block maxima, so they take the same decisions.
       float m_ref = kNegInf, l_run = 0.0f;
       // block maximum (log2 units; -inf: the row took no part), unquantised sum and precision of
-      // the entries whose PV products are still to be merged, by entry parity
-      float pend_M[2] = {kNegInf, kNegInf}, pend_sum[2] = {0.0f, 0.0f};
-      int pend_f16[2] = {0, 0};
+      // the entries whose PV products are still to be merged: entry e - 1 (p1) and e - 2 (p2)
+      float p1_M = kNegInf, p1_sum = 0.0f, p2_M = kNegInf, p2_sum = 0.0f;
+      int p1_f16 = 0, p2_f16 = 0;
       const bool dbg_unit = DBG && p.dbg && blockIdx.x == 0 && u == (int)blockIdx.x;
       const uint32_t g0 = g;
       constexpr int LAG = L::NPV;
@@ -725,13 +729,16 @@ __global__ void __launch_bounds__(384, 1)
       // that PV product, then the softmax of entry e; LAG more iterations merge the last entries
       for (int e = 0; e < n_entries + LAG; ++e) {
         const uint32_t v = g0 + e, buf = v & 1;
+        float cur_M = kNegInf, cur_sum = 0.0f;
+        int cur_f16 = 0;
         if (!(ok = mbar_wait(&bars->ready[buf], (v >> 1) & 1, abort_flag, p.status, lim))) break;
         tc_fence_after();
         if (e >= LAG) {
           // merge entry e - LAG: its PV product into this warpgroup's output columns with weight
           // exp2(pend_M - m_ref)
-          const int pe = (e - LAG) & 1;
-          const float pM = pend_M[pe];
+          const float pM = LAG == 2 ? p2_M : p1_M;
+          const float pSum = LAG == 2 ? p2_sum : p1_sum;
+          const int pF16 = LAG == 2 ? p2_f16 : p1_f16;
           const uint32_t pvb = LAG == 2 ? buf : 0;
           const bool need = pM != kNegInf && (m_ref == kNegInf || pM > m_ref + kRescale);
           if (__any_sync(0xffffffffu, need)) {
@@ -747,8 +754,8 @@ __global__ void __launch_bounds__(384, 1)
             if (need) m_ref = pM;
           }
           const float gs = (pM == kNegInf) ? 0.0f : ex2(pM - m_ref);
-          l_run = fmaf(gs, pend_sum[pe], l_run);
-          const float gpv = pend_f16[pe] ? gs : gs * pv4_scale;
+          l_run = fmaf(gs, pSum, l_run);
+          const float gpv = pF16 ? gs : gs * pv4_scale;
           const float2 g2 = make_float2(gpv, gpv);
           uint32_t r[DH];
 #pragma unroll
@@ -860,10 +867,16 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_before();
           fence_proxy_async_smem();
           mbar_arrive(&bars->p_full[buf]);
-          pend_M[e & 1] = valid ? Ms : kNegInf;
-          pend_sum[e & 1] = sum;
-          pend_f16[e & 1] = f16;
+          cur_M = valid ? Ms : kNegInf;
+          cur_sum = sum;
+          cur_f16 = f16;
         }
+        p2_M = p1_M;
+        p2_sum = p1_sum;
+        p2_f16 = p1_f16;
+        p1_M = cur_M;
+        p1_sum = cur_sum;
+        p1_f16 = cur_f16;
       }
       if (!ok) break;
       g = g0 + n_entries;
