@@ -49,7 +49,7 @@ constexpr float kNegInf = -__builtin_huge_valf();
 // blocks of at most 128 keys and |V| < 2^16 the FP32 sums stay below 2^68, far from overflow, and
 // FP32 keeps its relative precision at any scale.
 constexpr float kRescale = 32.0f;
-constexpr int kPolyPerGroup = 4;  // exponentials per 16 keys evaluated by the polynomial
+constexpr int kPolyPerGroup = 6;  // exponentials per 16 keys evaluated by the polynomial (measured best)
 
 __host__ __device__ constexpr int round1024(int x) { return (x + 1023) & ~1023; }
 __host__ __device__ constexpr int swz_for_row_bytes(int b) { return b == 128 ? kSW128 : (b == 64 ? kSW64 : kSW32); }
@@ -139,6 +139,13 @@ struct AttnParams {
 struct UnitInfo {
   int b, h, hk, t;
 };
+
+// The unit a CTA takes in its round r: units are ordered heaviest first (longest causal rows), and
+// the CTAs take them in a snake order (CTA c takes unit r * G + c in even rounds and
+// r * G + G - 1 - c in odd ones), which evens out the work per CTA.
+__device__ __forceinline__ int unit_of(int r) {
+  return r * (int)gridDim.x + ((r & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+}
 
 __device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, int u) {
   const int bh_count = p.B * p.Hq;
@@ -446,7 +453,7 @@ __global__ void __launch_bounds__(384, 1)
       PageRing ring{0, 0, p.npage};
       uint32_t uc = 0, u16c = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
+      for (int r = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++r), ++uc) {
         const UnitInfo ui = decode_unit(p, u);
         const uint32_t lb = uc & 1, lph = (uc >> 1) & 1;
         // the warp is converged here: every exit below is taken by all 32 lanes together
@@ -525,7 +532,7 @@ __global__ void __launch_bounds__(384, 1)
         PageRing ring{0, 0, p.npage};
         uint32_t uc = 0, u16c = 0, v = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
+        for (int r = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++r), ++uc) {
           const UnitInfo ui = decode_unit(p, u);
           const int kvh = ui.b * p.Hkv + ui.hk;
           const uint32_t lb = uc & 1, lph = (uc >> 1) & 1;
@@ -654,7 +661,7 @@ __global__ void __launch_bounds__(384, 1)
           }
           return true;
         };
-        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
+        for (int r = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++r), ++uc) {
           const UnitInfo ui = decode_unit(p, u);
           const int sfv_off = (((ui.b * p.Hkv + ui.hk) * D) & 127) >> 5;
           const uint32_t lb = uc & 1, lph = (uc >> 1) & 1;
@@ -702,7 +709,7 @@ __global__ void __launch_bounds__(384, 1)
     const float pv4_scale = v_ts * (1.0f / 2688.0f);
     uint32_t g = 0, uc = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
+    for (int r = 0, u = unit_of(0); u < p.n_units && ok; u = unit_of(++r), ++uc) {
       const UnitInfo ui = decode_unit(p, u);
       const uint32_t lb = uc & 1, lph = (uc >> 1) & 1;
       if (!(ok = mbar_wait(&bars->list_full[lb], lph, abort_flag, p.status, lim))) break;
