@@ -67,6 +67,7 @@ def lib():
         L.orc_quantize_nvfp4.restype = ctypes.c_float
         L.orc_quantize_nvfp4.argtypes = [_u16p, _i64, _i32, _i32, _i32, _u8p, _u8p]
         L.orc_block_scores.argtypes = [_u16p, _u16p] + [_int] * 8 + [_f64p]
+        L.orc_block_scores_qk.argtypes = [_u16p, _u16p] + [_int] * 9 + [_f64p]
         L.orc_topk_count.restype = _i64
         L.orc_topk_count.argtypes = [_i64, _int, _int]
         L.orc_select.argtypes = [_f64p, _i64, _i64, _int, _int, _u8p, _f64p, _i64p]
@@ -78,6 +79,10 @@ def lib():
         L.orc_attn.argtypes = (
             [_u16p, _u16p, _u16p, _u8p, _u8p, ctypes.c_float, _u8p, _u8p, ctypes.c_float,
              _u8p, _u8p, ctypes.c_float, _u8p] + [_int] * 8 + [ctypes.c_float, _i32p, _int, _int,
+             ctypes.c_void_p, _u16p, _f32p, ctypes.c_void_p, _int])
+        L.orc_attn_qk.argtypes = (
+            [_u16p, _u16p, _u16p, _u8p, _u8p, ctypes.c_float, _u8p, _u8p, ctypes.c_float,
+             _u8p, _u8p, ctypes.c_float, _u8p] + [_int] * 9 + [ctypes.c_float, _i32p, _int, _int,
              ctypes.c_void_p, _u16p, _f32p, ctypes.c_void_p, _int])
         L.orc_tile_scores.argtypes = (
             [_u16p, _u16p, _u8p, _u8p, ctypes.c_float, _u8p, _u8p, ctypes.c_float] + [_int] * 8
@@ -275,5 +280,63 @@ def forward(w, q, k, v, units=None, want_f64=False, threads=None):
     sel, kth, kc = select(scores, w)
     out, lse, out64 = attn(q, k, v, q4, k4, v4, sel, w, units=units, want_f64=want_f64,
                            threads=threads)
+    return dict(q4=q4, k4=k4, v4=v4, scores=scores, sel=sel, kth=kth, k=kc, out=out, lse=lse,
+                out64=out64)
+
+
+# ------------------------------------------------------------------ decode
+
+def decode_block_scores(q: np.ndarray, k: np.ndarray, block_k: int, causal: bool) -> np.ndarray:
+    """Decode selection scores (reading R-decode): the Nq query rows of each (batch, query head)
+    form one query block; S^_j = qbar . kbar_j over the key blocks of the cache, float64
+    [B, Hq, 1, Nk/block_k]."""
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    out = np.empty((B, Hq, 1, Nk // block_k), np.float64)
+    lib().orc_block_scores_qk(_u16(q).reshape(-1), _u16(k).reshape(-1), B, Hq, Hkv, Nq, Nk, d, Nq,
+                              block_k, int(causal), out.reshape(-1))
+    return out
+
+
+def decode_attn(q, k, v, q4: NVFP4, k4: NVFP4, v4: NVFP4, sel, block_k: int, causal: bool, tau=None,
+                want_f64=False, threads=None):
+    """Decode attention (reading R-decode): the Nq rows of q [B,Hq,Nq,d] are the newest
+    positions of the cache k, v [B,Hkv,Nk,d]; sel [B,Hq,1,Nk/block_k] marks the FP16 key blocks.
+    The same mixed-precision computation as `attn`.  Returns (out fp16 [B,Hq,Nq,d],
+    lse f32 [B,Hq,Nq], out64 or None)."""
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if tau is None:
+        tau = softmax_scale(d)
+    units = [(b, h, 0) for b in range(B) for h in range(Hq)]
+    u = np.ascontiguousarray(np.array(units, np.int32).reshape(-1))
+    out = np.zeros((B, Hq, Nq, d), np.uint16)
+    lse = np.zeros((B, Hq, Nq), np.float32)
+    out64 = np.zeros((B, Hq, Nq, d), np.float64) if want_f64 else None
+    if threads is None:
+        threads = os.cpu_count() or 1
+    lib().orc_attn_qk(_u16(q).reshape(-1), _u16(k).reshape(-1), _u16(v).reshape(-1),
+                      q4.codes.reshape(-1), q4.scales.reshape(-1), q4.tensor_scale,
+                      k4.codes.reshape(-1), k4.scales.reshape(-1), k4.tensor_scale,
+                      v4.codes.reshape(-1), v4.scales.reshape(-1), v4.tensor_scale,
+                      np.ascontiguousarray(sel, np.uint8).reshape(-1),
+                      B, Hq, Hkv, Nq, Nk, d, Nq, block_k, int(causal), np.float32(tau),
+                      u, len(units), 0, None, out.reshape(-1), lse.reshape(-1),
+                      None if out64 is None else out64.ctypes.data, int(threads))
+    return out.view(np.float16), lse, out64
+
+
+def decode_forward(w, q, k, v, k4=None, v4=None, want_f64=False, threads=None):
+    """One decode step: quantise the query rows, score and select key blocks, attend.
+    k4, v4: the cache's NVFP4 copies (computed here when None).  Returns a dict."""
+    q4 = quantize_nvfp4(q, 0)
+    if k4 is None:
+        k4 = quantize_nvfp4(k, 0)
+    if v4 is None:
+        v4 = quantize_nvfp4(v, 1)
+    scores = decode_block_scores(q, k, w.block_k, w.causal)
+    sel, kth, kc = select(scores, w)
+    out, lse, out64 = decode_attn(q, k, v, q4, k4, v4, sel, w.block_k, w.causal, want_f64=want_f64,
+                                  threads=threads)
     return dict(q4=q4, k4=k4, v4=v4, scores=scores, sel=sel, kth=kth, k=kc, out=out, lse=lse,
                 out64=out64)

@@ -37,6 +37,14 @@
  *            exp(M - m) (m = row maximum over all valid keys); the softmax
  *            denominator sums the unquantised FP32 exp(S - M).
  *   R-fp16   the FP16 pairs use P rounded to FP16 and the FP16 V.
+ *   R-decode decode (Nq query rows against a cache of Nk >= Nq keys): the
+ *            query rows are the newest Nq positions Nk-Nq .. Nk-1, so causal
+ *            masking is aligned bottom-right (key t visible to query row r
+ *            when t <= Nk - Nq + r); the Nq rows form one query block, so the
+ *            selection is one top-k per (batch, query head) over the key
+ *            blocks with qbar the mean of the Nq rows; the query rows are
+ *            quantised as their own tensor (their own FP32 tensor scale).
+ *            Prefill is the case Nq = Nk.
  */
 #include <math.h>
 #include <pthread.h>
@@ -202,23 +210,27 @@ double orc_nvfp4_elem(const uint8_t* codes, const uint8_t* scales, int64_t row, 
 
 /* ---------------------------------------------------------- block select */
 
-static inline int pair_valid(int causal, int i, int j, int bq, int bk) {
-  return !causal || (int64_t)j * bk <= (int64_t)(i + 1) * bq - 1;
+/* Pair (query block i, key block j) is valid when some key of block j is visible to some
+ * row of block i; with the causal offset qoff, query row r sits at position qoff + r. */
+static inline int pair_valid(int causal, int64_t qoff, int i, int j, int bq, int bk) {
+  return !causal || (int64_t)j * bk <= qoff + (int64_t)(i + 1) * bq - 1;
 }
 
-int orc_pair_valid(int causal, int i, int j, int bq, int bk) { return pair_valid(causal, i, j, bq, bk); }
+int orc_pair_valid(int causal, int i, int j, int bq, int bk) { return pair_valid(causal, 0, i, j, bq, bk); }
 
 /* S^_ij = qbar_i . kbar_j per (batch, query head); -inf for invalid pairs.
- * q [B,Hq,N,d], k [B,Hkv,N,d] FP16; scores [B,Hq,nQb,nKb] float64. */
-void orc_block_scores(const uint16_t* q, const uint16_t* k, int B, int Hq, int Hkv, int N, int d, int bq,
-                      int bk, int causal, double* scores) {
-  int nqb = N / bq, nkb = N / bk, grp = Hq / Hkv;
+ * q [B,Hq,Nq,d], k [B,Hkv,Nk,d] FP16 (query row r at position Nk - Nq + r);
+ * scores [B,Hq,Nq/bq,Nk/bk] float64. */
+void orc_block_scores_qk(const uint16_t* q, const uint16_t* k, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                         int bq, int bk, int causal, double* scores) {
+  int nqb = Nq / bq, nkb = Nk / bk, grp = Hq / Hkv;
+  int64_t qoff = (int64_t)Nk - Nq;
   double* kbar = (double*)malloc(sizeof(double) * (size_t)nkb * d);
   double* qbar = (double*)malloc(sizeof(double) * (size_t)d);
   for (int b = 0; b < B; ++b)
     for (int h = 0; h < Hq; ++h) {
-      const uint16_t* kh = k + ((int64_t)b * Hkv + h / grp) * (int64_t)N * d;
-      const uint16_t* qh = q + ((int64_t)b * Hq + h) * (int64_t)N * d;
+      const uint16_t* kh = k + ((int64_t)b * Hkv + h / grp) * (int64_t)Nk * d;
+      const uint16_t* qh = q + ((int64_t)b * Hq + h) * (int64_t)Nq * d;
       for (int j = 0; j < nkb; ++j)
         for (int c = 0; c < d; ++c) {
           double s = 0.0;
@@ -233,7 +245,7 @@ void orc_block_scores(const uint16_t* q, const uint16_t* k, int B, int Hq, int H
         }
         double* row = scores + (((int64_t)b * Hq + h) * nqb + i) * nkb;
         for (int j = 0; j < nkb; ++j) {
-          if (!pair_valid(causal, i, j, bq, bk)) { row[j] = -INFINITY; continue; }
+          if (!pair_valid(causal, qoff, i, j, bq, bk)) { row[j] = -INFINITY; continue; }
           double s = 0.0;
           for (int c = 0; c < d; ++c) s += qbar[c] * kbar[(int64_t)j * d + c];
           row[j] = s;
@@ -242,6 +254,12 @@ void orc_block_scores(const uint16_t* q, const uint16_t* k, int B, int Hq, int H
     }
   free(kbar);
   free(qbar);
+}
+
+/* Prefill form: q and k both [.., N, d]. */
+void orc_block_scores(const uint16_t* q, const uint16_t* k, int B, int Hq, int Hkv, int N, int d, int bq,
+                      int bk, int causal, double* scores) {
+  orc_block_scores_qk(q, k, B, Hq, Hkv, N, N, d, bq, bk, causal, scores);
 }
 
 int64_t orc_topk_count(int64_t n_valid, int topk_abs, int topk_bp) {
@@ -285,12 +303,15 @@ typedef struct {
   const uint8_t *q4c, *q4s, *k4c, *k4s, *v4c, *v4s;
   float q4t, k4t, v4t;
   const uint8_t* sel;
-  int B, Hq, Hkv, N, d, bq, bk, causal;
+  int B, Hq, Hkv, Nq, Nk, d, bq, bk, causal;
   double tau;
 } attn_problem;
 
+/* position of query row 0 among the keys (bottom-right causal alignment) */
+static inline int64_t qoff_of(const attn_problem* P) { return (int64_t)P->Nk - P->Nq; }
+
 static int pair_is_fp16(const attn_problem* P, int b, int h, int i, int j) {
-  int nqb = P->N / P->bq, nkb = P->N / P->bk;
+  int nqb = P->Nq / P->bq, nkb = P->Nk / P->bk;
   return P->sel[(((int64_t)b * P->Hq + h) * nqb + i) * nkb + j] != 0;
 }
 
@@ -302,8 +323,8 @@ static int pair_is_fp16(const attn_problem* P, int b, int h, int i, int j) {
 static void block_scores(const attn_problem* P, int b, int h, int i, int j, int fp16, double* qd, double* kd,
                          double* S, int64_t ldS) {
   int d = P->d, hk = h / (P->Hq / P->Hkv);
-  int64_t qbase = ((int64_t)b * P->Hq + h) * P->N + (int64_t)i * P->bq;
-  int64_t kbase = ((int64_t)b * P->Hkv + hk) * P->N + (int64_t)j * P->bk;
+  int64_t qbase = ((int64_t)b * P->Hq + h) * P->Nq + (int64_t)i * P->bq;
+  int64_t kbase = ((int64_t)b * P->Hkv + hk) * P->Nk + (int64_t)j * P->bk;
   for (int t = 0; t < P->bk; ++t)
     for (int c = 0; c < d; ++c)
       kd[t * d + c] = fp16 ? orc_half_to_double(P->k[(kbase + t) * d + c])
@@ -312,9 +333,9 @@ static void block_scores(const attn_problem* P, int b, int h, int i, int j, int 
   for (int r = 0; r < P->bq; ++r) {
     for (int c = 0; c < d; ++c)
       qd[c] = fp16 ? orc_half_to_double(P->q[(qbase + r) * d + c]) : nvfp4_elem(P->q4c, P->q4s, qbase + r, d, c);
-    int row = i * P->bq + r;
+    int64_t row = qoff_of(P) + (int64_t)i * P->bq + r;
     for (int t = 0; t < P->bk; ++t) {
-      int key = j * P->bk + t;
+      int64_t key = (int64_t)j * P->bk + t;
       if (P->causal && key > row) { S[r * ldS + t] = -INFINITY; continue; }
       double s = 0.0;
       for (int c = 0; c < d; ++c) s += qd[c] * kd[t * d + c];
@@ -369,8 +390,8 @@ static void block_values(const attn_problem* P, int b, int h, int j, int fp16, d
   for (int t = 0; t < P->bk; ++t) {
     int key = j * P->bk + t;
     for (int c = 0; c < d; ++c)
-      vd[t * d + c] = fp16 ? orc_half_to_double(P->v[(vb * P->N + key) * d + c])
-                           : nvfp4_elem(P->v4c, P->v4s, vb * d + c, P->N, key) * (double)P->v4t;
+      vd[t * d + c] = fp16 ? orc_half_to_double(P->v[(vb * P->Nk + key) * d + c])
+                           : nvfp4_elem(P->v4c, P->v4s, vb * d + c, P->Nk, key) * (double)P->v4t;
   }
 }
 
@@ -381,9 +402,9 @@ static void block_values(const attn_problem* P, int b, int h, int j, int fp16, d
  * running sums by exp(m_old - m_new) whenever it grows. */
 static void attn_unit(const attn_problem* P, int b, int h, int i, int online, const int32_t* order,
                       uint16_t* out, float* lse, double* out64) {
-  int nkb = P->N / P->bk, d = P->d, bq = P->bq, bk = P->bk;
-  int64_t ldS = (int64_t)P->N;
-  double* S = (double*)malloc(sizeof(double) * (size_t)bq * (size_t)P->N);
+  int nkb = P->Nk / P->bk, d = P->d, bq = P->bq, bk = P->bk;
+  int64_t ldS = (int64_t)P->Nk, qoff = qoff_of(P);
+  double* S = (double*)malloc(sizeof(double) * (size_t)bq * (size_t)P->Nk);
   double* qd = (double*)malloc(sizeof(double) * (size_t)d);
   double* kd = (double*)malloc(sizeof(double) * (size_t)bk * d);
   double* vd = (double*)malloc(sizeof(double) * (size_t)bk * d);
@@ -394,7 +415,7 @@ static void attn_unit(const attn_problem* P, int b, int h, int i, int online, co
   for (int r = 0; r < bq; ++r) m[r] = -INFINITY;
 
   for (int j = 0; j < nkb; ++j) {
-    if (!pair_valid(P->causal, i, j, bq, bk)) {
+    if (!pair_valid(P->causal, qoff, i, j, bq, bk)) {
       for (int r = 0; r < bq; ++r)
         for (int t = 0; t < bk; ++t) S[r * ldS + (int64_t)j * bk + t] = -INFINITY;
       continue;
@@ -403,11 +424,11 @@ static void attn_unit(const attn_problem* P, int b, int h, int i, int online, co
   }
   if (!online)
     for (int r = 0; r < bq; ++r)
-      for (int64_t t = 0; t < P->N; ++t) if (S[r * ldS + t] > m[r]) m[r] = S[r * ldS + t];
+      for (int64_t t = 0; t < P->Nk; ++t) if (S[r * ldS + t] > m[r]) m[r] = S[r * ldS + t];
 
   for (int jj = 0; jj < nkb; ++jj) {
     int j = order ? order[jj] : jj;
-    if (!pair_valid(P->causal, i, j, bq, bk)) continue;
+    if (!pair_valid(P->causal, qoff, i, j, bq, bk)) continue;
     int fp16 = pair_is_fp16(P, b, h, i, j);
     block_values(P, b, h, j, fp16, vd);
     for (int r = 0; r < bq; ++r) {
@@ -431,7 +452,7 @@ static void attn_unit(const attn_problem* P, int b, int h, int i, int online, co
     }
   }
   for (int r = 0; r < bq; ++r) {
-    int64_t orow = ((int64_t)b * P->Hq + h) * P->N + (int64_t)i * bq + r;
+    int64_t orow = ((int64_t)b * P->Hq + h) * P->Nq + (int64_t)i * bq + r;
     for (int c = 0; c < d; ++c) {
       double o = acc[(int64_t)r * d + c] / l[r];
       out[orow * d + c] = orc_double_to_half(o);
@@ -468,18 +489,18 @@ static void* attn_worker(void* arg) {
   return NULL;
 }
 
-/* Attention forward over the listed (b, h, i) units.  Inputs: FP16 q [B,Hq,N,d], k, v
- * [B,Hkv,N,d]; NVFP4 codes/scales of q, k (grouped along d) and v (grouped along tokens,
- * [B,Hkv,d,N/2]) with their tensor scales; sel [B,Hq,nQb,nKb] (1 = FP16 pair).
- * Writes O (FP16, and float64 when out64 != NULL) and lse (natural log, tau-scaled
- * scores) for the rows of the listed units only. */
-void orc_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint8_t* q4c, const uint8_t* q4s,
-              float q4t, const uint8_t* k4c, const uint8_t* k4s, float k4t, const uint8_t* v4c,
-              const uint8_t* v4s, float v4t, const uint8_t* sel, int B, int Hq, int Hkv, int N, int d, int bq,
-              int bk, int causal, float tau, const int32_t* units, int n_units, int online,
-              const int32_t* order, uint16_t* out, float* lse, double* out64, int n_threads) {
+/* Attention forward over the listed (b, h, i) units.  Inputs: FP16 q [B,Hq,Nq,d], k, v
+ * [B,Hkv,Nk,d] (query row r at position Nk - Nq + r); NVFP4 codes/scales of q, k (grouped
+ * along d) and v (grouped along tokens, [B,Hkv,d,Nk/2]) with their tensor scales;
+ * sel [B,Hq,Nq/bq,Nk/bk] (1 = FP16 pair).  Writes O (FP16 [B,Hq,Nq,d], and float64 when
+ * out64 != NULL) and lse (natural log, tau-scaled scores) for the rows of the listed units. */
+void orc_attn_qk(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint8_t* q4c, const uint8_t* q4s,
+                 float q4t, const uint8_t* k4c, const uint8_t* k4s, float k4t, const uint8_t* v4c,
+                 const uint8_t* v4s, float v4t, const uint8_t* sel, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                 int bq, int bk, int causal, float tau, const int32_t* units, int n_units, int online,
+                 const int32_t* order, uint16_t* out, float* lse, double* out64, int n_threads) {
   attn_problem P = {q, k, v, q4c, q4s, k4c, k4s, v4c, v4s, q4t, k4t, v4t, sel,
-                    B, Hq, Hkv, N, d, bq, bk, causal, (double)tau};
+                    B, Hq, Hkv, Nq, Nk, d, bq, bk, causal, (double)tau};
   attn_job J;
   J.P = &P; J.units = units; J.n_units = n_units; J.online = online; J.order = order;
   J.out = out; J.lse = lse; J.out64 = out64; J.next = 0;
@@ -492,13 +513,23 @@ void orc_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uin
   pthread_mutex_destroy(&J.mu);
 }
 
+/* Prefill form: q, k, v all [.., N, d]. */
+void orc_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint8_t* q4c, const uint8_t* q4s,
+              float q4t, const uint8_t* k4c, const uint8_t* k4s, float k4t, const uint8_t* v4c,
+              const uint8_t* v4s, float v4t, const uint8_t* sel, int B, int Hq, int Hkv, int N, int d, int bq,
+              int bk, int causal, float tau, const int32_t* units, int n_units, int online,
+              const int32_t* order, uint16_t* out, float* lse, double* out64, int n_threads) {
+  orc_attn_qk(q, k, v, q4c, q4s, q4t, k4c, k4s, k4t, v4c, v4s, v4t, sel, B, Hq, Hkv, N, N, d, bq, bk, causal, tau,
+              units, n_units, online, order, out, lse, out64, n_threads);
+}
+
 /* The tau-scaled scores of one (b, h, query block i, key block j) tile, [bq, bk] float64,
  * in the given precision (fp16 = 1: FP16 inputs; 0: NVFP4 inputs).  For the pins. */
 void orc_tile_scores(const uint16_t* q, const uint16_t* k, const uint8_t* q4c, const uint8_t* q4s, float q4t,
                      const uint8_t* k4c, const uint8_t* k4s, float k4t, int B, int Hq, int Hkv, int N, int d,
                      int bq, int bk, int causal, float tau, int b, int h, int i, int j, int fp16, double* S) {
   attn_problem P = {q, k, NULL, q4c, q4s, k4c, k4s, NULL, NULL, q4t, k4t, 0.0f, NULL,
-                    B, Hq, Hkv, N, d, bq, bk, causal, (double)tau};
+                    B, Hq, Hkv, N, N, d, bq, bk, causal, (double)tau};
   double* qd = (double*)malloc(sizeof(double) * (size_t)d);
   double* kd = (double*)malloc(sizeof(double) * (size_t)bk * d);
   block_scores(&P, b, h, i, j, fp16, qd, kd, S, bk);

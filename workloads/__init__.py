@@ -48,6 +48,7 @@ STREAM_Q, STREAM_K, STREAM_V = 1, 2, 3
 STREAM_KBIAS = 4
 STREAM_QOUT, STREAM_KOUT, STREAM_VOUT = 5, 6, 7
 STREAM_QROW, STREAM_KROW, STREAM_VROW = 8, 9, 10
+STREAM_QDEC = 11  # the query rows of a decode step
 
 _f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
 _u64 = ctypes.c_uint64
@@ -113,6 +114,7 @@ class Workload:
     topk_abs: int  # >= 0: absolute k per head; -1: use topk_bp
     topk_bp: int   # budget in basis points of the valid pairs
     dist: str      # "normal" | "heavy_bias" | "student_t" | "row_lognormal"
+    n_query: int = 0  # > 0: a decode step, n_query query rows against a cache of N keys
 
     @property
     def seed(self) -> int:
@@ -125,6 +127,10 @@ class Workload:
     @property
     def n_kb(self) -> int:
         return self.N // self.block_k
+
+    @property
+    def is_decode(self) -> bool:
+        return self.n_query > 0
 
     def with_budget(self, topk_bp: int, topk_abs: int = -1) -> "Workload":
         return dataclasses.replace(self, topk_bp=topk_bp, topk_abs=topk_abs)
@@ -145,6 +151,14 @@ WORKLOADS = {
                          "student_t"),
     "diffusion": Workload("diffusion", 4, 2, 24, 24, 16384, 64, False, 128, 64, -1, 500,
                           "row_lognormal"),
+    # decode steps: n_query new query rows (the newest positions) against a cache of N keys;
+    # block_q is unused (the query rows form one block)
+    "decode_tiny": Workload("decode_tiny", 6, 1, 4, 2, 1024, 64, True, 128, 64, -1, 1000, "normal",
+                            n_query=2),
+    "decode32k": Workload("decode32k", 7, 1, 32, 8, 32768, 128, True, 128, 64, -1, 500, "heavy_bias",
+                          n_query=1),
+    "decode131k": Workload("decode131k", 8, 1, 32, 8, 131072, 128, True, 128, 128, -1, 200,
+                           "student_t", n_query=1),
 }
 DIFFUSION_BUDGETS_BP = (0, 100, 500, 2000, 10000)
 
@@ -194,8 +208,12 @@ def _tensor(w: Workload, stream: int, shape, which: str) -> np.ndarray:
 
 
 def make_qkv(w: Workload):
-    """Seeded FP16 Q [B,Hq,N,d], K [B,Hkv,N,d], V [B,Hkv,N,d] as numpy arrays."""
-    q = _tensor(w, STREAM_Q, (w.B, w.Hq, w.N, w.d), "q")
+    """Seeded FP16 Q [B,Hq,N,d] (decode: [B,Hq,n_query,d]), K [B,Hkv,N,d], V [B,Hkv,N,d] as
+    numpy arrays."""
+    if w.is_decode:
+        q = _tensor(w, STREAM_QDEC, (w.B, w.Hq, w.n_query, w.d), "q")
+    else:
+        q = _tensor(w, STREAM_Q, (w.B, w.Hq, w.N, w.d), "q")
     k = _tensor(w, STREAM_K, (w.B, w.Hkv, w.N, w.d), "k")
     v = _tensor(w, STREAM_V, (w.B, w.Hkv, w.N, w.d), "v")
     return q, k, v
