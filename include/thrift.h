@@ -153,6 +153,71 @@ thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, 
                                    float* lse, const thrift_cfg* cfg, void* ws,
                                    size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------ decode
+ *
+ * Decode form of the same method (ThriftAttention technical summary, "Methodologie" for the
+ * computation; "Resultaten" for its decode use against a KV cache held in FP16 and NVFP4).
+ * A step has Nq new query rows per query head; they are the newest Nq positions of a cache of
+ * Nk keys (the rows of this step already appended), so with causal = 1 key t is visible to
+ * query row r (0-based among the Nq) when t <= Nk - Nq + r.  The Nq rows of a head form one
+ * query block: selection picks the k key blocks with the largest qbar . kbar_j per (batch,
+ * query head), qbar the mean of the Nq rows, k = topk_abs or ceil(topk_bp * nKb / 10000).
+ * The query rows are quantised to NVFP4 as one tensor (their own FP32 tensor scale).  Every
+ * other step -- NVFP4 scores on the other blocks, two-level re-quantisation of the probability
+ * blocks, FP16 on the selected blocks, one softmax -- is the prefill computation.
+ *
+ * The cache: k, v FP16 [B,Hkv,Nk,d]; k4 = thrift_quantize_nvfp4(k, group_axis 0), v4 =
+ * thrift_quantize_nvfp4(v, group_axis 1); kbar = thrift_kv_block_means(k).  All owned by the
+ * caller and only read. */
+typedef struct {
+  int32_t B, Hq, Hkv;  /* batch, query heads, key/value heads (Hq % Hkv == 0) */
+  int32_t Nq;          /* query rows per head in this step, 1 <= Nq, (Hq/Hkv) * Nq <= 16 */
+  int32_t Nk;          /* cache length, Nq <= Nk, a multiple of 128 and of block_k */
+  int32_t d;           /* head dim, 64 or 128 */
+  int32_t causal;      /* 0 or 1 (bottom-right aligned, see above) */
+  int32_t block_k;     /* key block size, 64 or 128 */
+  int32_t topk_abs;    /* >= 0: FP16 key blocks per (batch, query head); -1: use topk_bp */
+  int32_t topk_bp;     /* budget in basis points of the nKb = Nk/block_k key blocks
+                          (0 = every block NVFP4, 10000 = every block FP16) */
+  float softmax_scale; /* tau; 0 selects 1/sqrt(d) rounded to FP32 */
+} thrift_decode_cfg;
+
+/* Block means of the cache's keys: kbar [outer, Nk/block_k, d] float64, the exact FP16 sum of
+ * each column over the block's tokens divided by block_k (k: device FP16 [outer, Nk, d]).
+ * Computed once per cache (and per appended block); thrift_decode_select reads it. */
+thrift_status thrift_kv_block_means(const void* k, int64_t outer, int32_t Nk, int32_t d, int32_t block_k,
+                                    double* kbar, void* stream);
+
+/* Workspace bytes of thrift_decode_select, thrift_decode_attn and thrift_decode_fwd (the
+ * query rows' NVFP4 copy, the selection of thrift_decode_fwd and the splits' partial sums).
+ * 0 for an unsupported configuration. */
+size_t thrift_decode_workspace_bytes(const thrift_decode_cfg* cfg);
+
+/* Decode selection.  q: device FP16 [B,Hq,Nq,d]; kbar: device [B,Hkv,nKb,d] float64.
+ * Outputs (device): mask [B,Hq,ceil(nKb/32)] u32 (bit j%32 of word j/32: key block j in FP16),
+ * counts [B,Hq] i32, lists [B,Hq,nKb] i16 (ascending, -1 past counts), scores [B,Hq,nKb]
+ * float64 S^_j (may be NULL).  Ties in S^ go to the smaller j. */
+thrift_status thrift_decode_select(const void* q, const double* kbar, const thrift_decode_cfg* cfg,
+                                   uint32_t* mask, int32_t* counts, int16_t* lists, double* scores,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/* Decode attention.  q: device FP16 [B,Hq,Nq,d]; k, v: the FP16 cache (may be NULL when the
+ * budget is 0); k4, v4: its NVFP4 copies (may be NULL when the budget is 10000); mask: the
+ * selection of thrift_decode_select (may be NULL for budgets 0 and 10000).
+ * out: device FP16 [B,Hq,Nq,d]; lse: device float [B,Hq,Nq] (may be NULL).
+ * Launches: the query rows' NVFP4 quantisation, a split-over-key-blocks kernel (m16n8k16
+ * tensor-core tiles, bulk/tensor copies into shared memory, bounded waits) and a kernel that
+ * combines the splits. */
+thrift_status thrift_decode_attn(const void* q, const void* k, const void* v, const thrift_nvfp4* k4,
+                                 const thrift_nvfp4* v4, const uint32_t* mask, void* out, float* lse,
+                                 const thrift_decode_cfg* cfg, void* ws, size_t ws_bytes, void* stream);
+
+/* One decode step: thrift_decode_select (selection kept in the workspace), then
+ * thrift_decode_attn. */
+thrift_status thrift_decode_fwd(const void* q, const void* k, const void* v, const thrift_nvfp4* k4,
+                                const thrift_nvfp4* v4, const double* kbar, void* out, float* lse,
+                                const thrift_decode_cfg* cfg, void* ws, size_t ws_bytes, void* stream);
+
 /* Zero the device status word at the start of the workspace (enqueued on stream). */
 thrift_status thrift_reset_device_status(void* ws, void* stream);
 

@@ -23,7 +23,8 @@ from . import _lib
 from ._lib import ThriftError, check, load
 
 __all__ = ["Config", "NVFP4Tensor", "Selection", "Workspace", "quantize_nvfp4", "quantize_qkv",
-           "block_select", "attn_fwd", "attn_fwd_auto", "device_status", "reset_device_status",
+           "block_select", "attn_fwd", "attn_fwd_auto", "DecodeConfig", "KVCache", "kv_block_means",
+           "decode_select", "decode_attn", "decode_fwd", "device_status", "reset_device_status",
            "ThriftError", "load"]
 
 
@@ -250,3 +251,132 @@ def device_status(ws: Workspace) -> int:
     v = ctypes.c_int32(0)
     check(load().thrift_get_device_status(ws.ptr, _stream(), ctypes.byref(v)), "thrift_get_device_status")
     return int(v.value)
+
+
+# ------------------------------------------------------------------ decode
+
+@dataclasses.dataclass
+class DecodeConfig:
+    """Decode step description (thrift_decode_cfg): Nq new query rows per head, the newest
+    positions of a cache of Nk keys."""
+
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool = True
+    block_k: int = 64
+    topk_abs: int = -1
+    topk_bp: int = 500
+    softmax_scale: float = 0.0
+
+    @classmethod
+    def from_workload(cls, w) -> "DecodeConfig":
+        return cls(w.B, w.Hq, w.Hkv, w.n_query, w.N, w.d, bool(w.causal), w.block_k, w.topk_abs,
+                   w.topk_bp)
+
+    def c(self) -> _lib.CDecodeCfg:
+        return _lib.CDecodeCfg(self.B, self.Hq, self.Hkv, self.Nq, self.Nk, self.d, int(self.causal),
+                               self.block_k, self.topk_abs, self.topk_bp, self.softmax_scale)
+
+    @property
+    def n_kb(self) -> int:
+        return self.Nk // self.block_k
+
+    @property
+    def mask_words(self) -> int:
+        return (self.n_kb + 31) // 32
+
+    def workspace(self, device) -> Workspace:
+        c = self.c()
+        n = load().thrift_decode_workspace_bytes(ctypes.byref(c))
+        if n == 0:
+            raise ThriftError(_lib.THRIFT_ERR_UNSUPPORTED, "decode workspace size")
+        return Workspace(n, device)
+
+
+def kv_block_means(k: torch.Tensor, block_k: int) -> torch.Tensor:
+    """Block means of the cache's keys, float64 [.., Nk/block_k, d] (thrift_kv_block_means)."""
+    assert k.is_cuda and k.dtype == torch.float16 and k.is_contiguous()
+    *lead, Nk, d = k.shape
+    outer = 1
+    for s in lead:
+        outer *= s
+    kbar = torch.empty((*lead, Nk // block_k, d), dtype=torch.float64, device=k.device)
+    check(load().thrift_kv_block_means(_ptr(k), outer, Nk, d, block_k, _ptr(kbar), _stream()),
+          "thrift_kv_block_means")
+    return kbar
+
+
+@dataclasses.dataclass
+class KVCache:
+    """A KV cache held twice, FP16 and NVFP4, with the key block means the selection reads."""
+
+    k: torch.Tensor
+    v: torch.Tensor
+    k4: NVFP4Tensor
+    v4: NVFP4Tensor
+    kbar: torch.Tensor
+    block_k: int
+
+    @classmethod
+    def build(cls, k: torch.Tensor, v: torch.Tensor, block_k: int, ws: Optional[Workspace] = None) -> "KVCache":
+        return cls(k, v, quantize_nvfp4(k, 0, ws=ws), quantize_nvfp4(v, 1, ws=ws), kv_block_means(k, block_k),
+                   block_k)
+
+
+def decode_select(q: torch.Tensor, cache: KVCache, cfg: DecodeConfig, ws: Optional[Workspace] = None,
+                  want_scores: bool = False) -> Selection:
+    """Per-head top-k key blocks of one decode step (thrift_decode_select); the Selection's
+    tensors have a query-block axis of length 1."""
+    dev = q.device
+    sel = Selection(
+        torch.empty((cfg.B, cfg.Hq, 1, cfg.mask_words), dtype=torch.int32, device=dev),
+        torch.empty((cfg.B, cfg.Hq, 1), dtype=torch.int32, device=dev),
+        torch.empty((cfg.B, cfg.Hq, 1, cfg.n_kb), dtype=torch.int16, device=dev),
+        torch.empty((cfg.B, cfg.Hq, 1, cfg.n_kb), dtype=torch.float64, device=dev) if want_scores else None)
+    if ws is None:
+        ws = cfg.workspace(dev)
+    c = cfg.c()
+    check(load().thrift_decode_select(_ptr(q), _ptr(cache.kbar), ctypes.byref(c), _ptr(sel.mask),
+                                      _ptr(sel.counts), _ptr(sel.lists), _ptr(sel.scores), ws.ptr, ws.nbytes,
+                                      _stream()), "thrift_decode_select")
+    return sel
+
+
+def _decode_out(q, cfg, out, lse, want_lse):
+    if out is None:
+        out = torch.empty((cfg.B, cfg.Hq, cfg.Nq, cfg.d), dtype=torch.float16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((cfg.B, cfg.Hq, cfg.Nq), dtype=torch.float32, device=q.device)
+    return out, lse
+
+
+def decode_attn(q: torch.Tensor, cache: KVCache, sel: Optional[Selection], cfg: DecodeConfig,
+                out=None, lse=None, ws: Optional[Workspace] = None, want_lse: bool = True):
+    """Decode attention with a given selection (thrift_decode_attn).  Returns (out, lse)."""
+    out, lse = _decode_out(q, cfg, out, lse, want_lse)
+    if ws is None:
+        ws = cfg.workspace(q.device)
+    c = cfg.c()
+    k4, v4 = cache.k4.c(), cache.v4.c()
+    check(load().thrift_decode_attn(_ptr(q), _ptr(cache.k), _ptr(cache.v), ctypes.byref(k4), ctypes.byref(v4),
+                                    None if sel is None else _ptr(sel.mask), _ptr(out), _ptr(lse),
+                                    ctypes.byref(c), ws.ptr, ws.nbytes, _stream()), "thrift_decode_attn")
+    return out, lse
+
+
+def decode_fwd(q: torch.Tensor, cache: KVCache, cfg: DecodeConfig, out=None, lse=None,
+               ws: Optional[Workspace] = None, want_lse: bool = True):
+    """One decode step, selection and attention (thrift_decode_fwd).  Returns (out, lse)."""
+    out, lse = _decode_out(q, cfg, out, lse, want_lse)
+    if ws is None:
+        ws = cfg.workspace(q.device)
+    c = cfg.c()
+    k4, v4 = cache.k4.c(), cache.v4.c()
+    check(load().thrift_decode_fwd(_ptr(q), _ptr(cache.k), _ptr(cache.v), ctypes.byref(k4), ctypes.byref(v4),
+                                   _ptr(cache.kbar), _ptr(out), _ptr(lse), ctypes.byref(c), ws.ptr, ws.nbytes,
+                                   _stream()), "thrift_decode_fwd")
+    return out, lse

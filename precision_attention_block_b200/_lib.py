@@ -35,6 +35,14 @@ class CCfg(ctypes.Structure):
                 ("softmax_scale", ctypes.c_float)]
 
 
+class CDecodeCfg(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("Nq", ctypes.c_int32), ("Nk", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("causal", ctypes.c_int32), ("block_k", ctypes.c_int32),
+                ("topk_abs", ctypes.c_int32), ("topk_bp", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float)]
+
+
 class CNVFP4(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("scales_mma", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p),
@@ -50,6 +58,7 @@ _i32 = ctypes.c_int32
 _i64 = ctypes.c_int64
 _cfgp = ctypes.POINTER(CCfg)
 _nvp = ctypes.POINTER(CNVFP4)
+_dcfgp = ctypes.POINTER(CDecodeCfg)
 
 SIGNATURES = {
     "thrift_nvfp4_scales_mma_bytes": (_sz, [_i64, _i32, _i32, _i32]),
@@ -61,6 +70,11 @@ SIGNATURES = {
     "thrift_attn_fwd": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _nvp, _vp, _vp, _vp, _vp, _vp, _cfgp,
                                        _vp, _sz, _vp]),
     "thrift_attn_fwd_auto": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _cfgp, _vp, _sz, _vp]),
+    "thrift_kv_block_means": (ctypes.c_int, [_vp, _i64, _i32, _i32, _i32, _vp, _vp]),
+    "thrift_decode_workspace_bytes": (_sz, [_dcfgp]),
+    "thrift_decode_select": (ctypes.c_int, [_vp, _vp, _dcfgp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "thrift_decode_attn": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _vp, _vp, _vp, _dcfgp, _vp, _sz, _vp]),
+    "thrift_decode_fwd": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _vp, _vp, _vp, _dcfgp, _vp, _sz, _vp]),
     "thrift_reset_device_status": (ctypes.c_int, [_vp, _vp]),
     "thrift_get_device_status": (ctypes.c_int, [_vp, _vp, ctypes.POINTER(_i32)]),
     "thrift_debug_wait_timeout": (ctypes.c_int, [_vp, _i64, _vp]),

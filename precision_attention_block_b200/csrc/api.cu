@@ -100,6 +100,105 @@ AutoLayout auto_layout(const thrift_cfg& c) {
   return L;
 }
 
+bool dcfg_ok(const thrift_decode_cfg* c) {
+  if (!c) return false;
+  if (c->B <= 0 || c->Hq <= 0 || c->Hkv <= 0 || c->Nq <= 0 || c->Nk <= 0) return false;
+  if (c->Hq % c->Hkv != 0 || c->Nq > c->Nk) return false;
+  if (c->causal != 0 && c->causal != 1) return false;
+  if (c->topk_abs < -1) return false;
+  if (c->topk_abs == -1 && (c->topk_bp < 0 || c->topk_bp > 10000)) return false;
+  if (!(c->softmax_scale >= 0.0f) || std::isinf(c->softmax_scale)) return false;
+  return true;
+}
+
+thrift_status dcfg_supported(const thrift_decode_cfg* c) {
+  if (!dcfg_ok(c)) return THRIFT_ERR_INVALID_ARG;
+  if (c->d != 64 && c->d != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (c->block_k != 64 && c->block_k != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (c->Nk % 128 != 0 || c->Nk % c->block_k != 0) return THRIFT_ERR_UNSUPPORTED;
+  if (c->Nk / c->block_k > 32767) return THRIFT_ERR_UNSUPPORTED;
+  if ((int64_t)(c->Hq / c->Hkv) * c->Nq > 16) return THRIFT_ERR_UNSUPPORTED;
+  if ((int64_t)c->B * c->Hkv * c->Nk > (int64_t)INT32_MAX / 2) return THRIFT_ERR_UNSUPPORTED;
+  return THRIFT_OK;
+}
+
+int decode_mode(const thrift_decode_cfg* c) {
+  if (c->topk_abs == 0 || (c->topk_abs < 0 && c->topk_bp == 0)) return 1;
+  if (c->topk_abs < 0 && c->topk_bp == 10000) return 2;
+  return 0;
+}
+
+struct DecodeLayout {
+  size_t q4c, q4s, q4m, qts, select, mask, counts, lists, part_o, part_ml, bytes;
+};
+
+DecodeLayout decode_layout(const thrift_decode_cfg& c) {
+  DecodeLayout L;
+  const size_t qn = (size_t)c.B * c.Hq * c.Nq * c.d;
+  const size_t heads = (size_t)c.B * c.Hq, nkb = (size_t)(c.Nk / c.block_k);
+  const size_t parts = (size_t)c.B * c.Hkv * decode_split_cap((int)nkb);
+  size_t off = kWsHeader;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.q4c = take(qn / 2);
+  L.q4s = take(qn / 16);
+  L.q4m = take(scales_mma_bytes((int64_t)heads, c.Nq, c.d, 0));
+  L.qts = take(sizeof(float));
+  L.select = take(decode_select_scratch_bytes(c));
+  L.mask = take(heads * ((nkb + 31) / 32) * 4);
+  L.counts = take(heads * 4);
+  L.lists = take(heads * nkb * 2);
+  L.part_o = take(parts * 16 * c.d * sizeof(float));
+  L.part_ml = take(parts * 16 * 2 * sizeof(float));
+  L.bytes = off;
+  return L;
+}
+
+bool al16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
+
+thrift_status decode_attn_common(const void* q, const void* k, const void* v, const thrift_nvfp4* k4,
+                                 const thrift_nvfp4* v4, const uint32_t* mask, void* out, float* lse,
+                                 const thrift_decode_cfg* cfg, void* ws, size_t ws_bytes, cudaStream_t s) {
+  const int mode = decode_mode(cfg);
+  if (!q || !out || !al16(q)) return THRIFT_ERR_INVALID_ARG;
+  if (mode != 1 && (!k || !v || !al16(k) || !al16(v))) return THRIFT_ERR_INVALID_ARG;
+  if (mode != 2) {
+    if (!nvfp4_ok(k4, 0) || !nvfp4_ok(v4, 1)) return THRIFT_ERR_INVALID_ARG;
+    if (!al16(k4->codes) || !al16(k4->scales) || !al16(v4->codes) || !al16(v4->scales_mma))
+      return THRIFT_ERR_INVALID_ARG;
+  }
+  if (mode == 0 && !mask) return THRIFT_ERR_INVALID_ARG;
+  const DecodeLayout L = decode_layout(*cfg);
+  if (!ws_ok(ws, ws_bytes, L.bytes)) return THRIFT_ERR_WORKSPACE;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  thrift_nvfp4 q4 = {w + L.q4c, w + L.q4s, w + L.q4m, reinterpret_cast<float*>(w + L.qts), 0};
+  const thrift_decode_cfg& c = *cfg;
+  if (mode != 2) {
+    unsigned int* amax = reinterpret_cast<unsigned int*>(w + kWsAmaxOff);
+    thrift_status st = quantize_launch(q, (int64_t)c.B * c.Hq, c.Nq, c.d, &q4, amax, s);
+    if (st != THRIFT_OK) return st;
+  }
+  DecodeArgs a;
+  a.cfg = cfg;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.q4 = &q4;
+  a.k4 = k4;
+  a.v4 = v4;
+  a.mask = mode == 0 ? mask : nullptr;
+  a.mode = mode;
+  a.out = out;
+  a.lse = lse;
+  a.part_o = reinterpret_cast<float*>(w + L.part_o);
+  a.part_ml = reinterpret_cast<float*>(w + L.part_ml);
+  a.status = status_ptr(ws);
+  return decode_attn_launch(a, s);
+}
+
 }  // namespace
 }  // namespace thrift
 
@@ -219,6 +318,59 @@ thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, 
   }
   return attn_launch_dbg(q, k, v, &q4, &k4, &v4, mode == 0 ? mask : nullptr, mode, out, lse, c, status_ptr(ws),
                          nullptr, -1, s);
+}
+
+thrift_status thrift_kv_block_means(const void* k, int64_t outer, int32_t Nk, int32_t d, int32_t block_k,
+                                    double* kbar, void* stream) {
+  if (!k || !kbar || outer <= 0 || Nk <= 0) return THRIFT_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (block_k != 64 && block_k != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (Nk % block_k != 0 || outer > 65535) return THRIFT_ERR_UNSUPPORTED;
+  return kv_means_launch(k, outer, Nk, d, block_k, kbar, static_cast<cudaStream_t>(stream));
+}
+
+size_t thrift_decode_workspace_bytes(const thrift_decode_cfg* cfg) {
+  if (dcfg_supported(cfg) != THRIFT_OK) return 0;
+  return decode_layout(*cfg).bytes;
+}
+
+thrift_status thrift_decode_select(const void* q, const double* kbar, const thrift_decode_cfg* cfg, uint32_t* mask,
+                                   int32_t* counts, int16_t* lists, double* scores, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  thrift_status st = dcfg_supported(cfg);
+  if (st != THRIFT_OK) return st;
+  if (!q || !kbar || !mask || !counts || !lists) return THRIFT_ERR_INVALID_ARG;
+  const DecodeLayout L = decode_layout(*cfg);
+  if (!ws_ok(ws, ws_bytes, L.bytes)) return THRIFT_ERR_WORKSPACE;
+  return decode_select_launch(q, kbar, *cfg, mask, counts, lists, scores, static_cast<uint8_t*>(ws) + L.select,
+                              static_cast<cudaStream_t>(stream));
+}
+
+thrift_status thrift_decode_attn(const void* q, const void* k, const void* v, const thrift_nvfp4* k4,
+                                 const thrift_nvfp4* v4, const uint32_t* mask, void* out, float* lse,
+                                 const thrift_decode_cfg* cfg, void* ws, size_t ws_bytes, void* stream) {
+  thrift_status st = dcfg_supported(cfg);
+  if (st != THRIFT_OK) return st;
+  return decode_attn_common(q, k, v, k4, v4, mask, out, lse, cfg, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+thrift_status thrift_decode_fwd(const void* q, const void* k, const void* v, const thrift_nvfp4* k4,
+                                const thrift_nvfp4* v4, const double* kbar, void* out, float* lse,
+                                const thrift_decode_cfg* cfg, void* ws, size_t ws_bytes, void* stream) {
+  thrift_status st = dcfg_supported(cfg);
+  if (st != THRIFT_OK) return st;
+  const DecodeLayout L = decode_layout(*cfg);
+  if (!ws_ok(ws, ws_bytes, L.bytes)) return THRIFT_ERR_WORKSPACE;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* mask = reinterpret_cast<uint32_t*>(w + L.mask);
+  if (decode_mode(cfg) == 0) {
+    if (!q || !kbar) return THRIFT_ERR_INVALID_ARG;
+    st = decode_select_launch(q, kbar, *cfg, mask, reinterpret_cast<int32_t*>(w + L.counts),
+                              reinterpret_cast<int16_t*>(w + L.lists), nullptr, w + L.select, s);
+    if (st != THRIFT_OK) return st;
+  }
+  return decode_attn_common(q, k, v, k4, v4, mask, out, lse, cfg, ws, ws_bytes, s);
 }
 
 thrift_status thrift_reset_device_status(void* ws, void* stream) {

@@ -260,4 +260,43 @@ thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, u
   return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 
+thrift_status kv_means_launch(const void* k, int64_t outer, int32_t Nk, int32_t d, int32_t block_k, double* kbar,
+                              cudaStream_t stream) {
+  int tpb = d >= 128 ? 128 : d;
+  block_mean_kernel<<<dim3(Nk / block_k, (unsigned)outer), tpb, 0, stream>>>(reinterpret_cast<const __half*>(k), Nk,
+                                                                             d, block_k, kbar);
+  return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
+}
+
+size_t decode_select_scratch_bytes(const thrift_decode_cfg& c) {
+  size_t heads = (size_t)c.B * c.Hq, nkb = (size_t)(c.Nk / c.block_k);
+  return align256(heads * c.d * sizeof(double)) + align256(heads * nkb * sizeof(double));
+}
+
+// The decode selection is the prefill selection with one query block of Nq rows per head.
+// Every key block holds a key visible to the newest row, so every pair is valid.
+thrift_status decode_select_launch(const void* q, const double* kbar, const thrift_decode_cfg& c, uint32_t* mask,
+                                   int32_t* counts, int16_t* lists, double* scores_out, uint8_t* scratch,
+                                   cudaStream_t stream) {
+  const int nkb = c.Nk / c.block_k;
+  const int mask_words = (nkb + 31) / 32;
+  const size_t heads = (size_t)c.B * c.Hq;
+  double* qbar = reinterpret_cast<double*>(scratch);
+  double* scores = scores_out ? scores_out
+                              : reinterpret_cast<double*>(scratch + align256(heads * c.d * sizeof(double)));
+  int tpb = c.d >= 128 ? 128 : c.d;
+  block_mean_kernel<<<dim3(1, (unsigned)heads), tpb, 0, stream>>>(reinterpret_cast<const __half*>(q), c.Nq, c.d,
+                                                                  c.Nq, qbar);
+  size_t smem = (size_t)(kTileQ + kTileK) * (c.d + 1) * sizeof(double);
+  dim3 g((nkb + kTileK - 1) / kTileK, 1, (unsigned)heads);
+  block_score_kernel<<<g, kTileQ * kTileK, smem, stream>>>(qbar, kbar, c.Hq, c.Hkv, 1, nkb, c.d, c.Nq, c.block_k, 0,
+                                                           scores);
+  if (cudaMemsetAsync(mask, 0, heads * mask_words * sizeof(uint32_t), stream) != cudaSuccess) return THRIFT_ERR_CUDA;
+  topk_kernel<<<(unsigned)heads, kSelThreads, 0, stream>>>(scores, (int64_t)nkb, nkb, c.topk_abs, c.topk_bp,
+                                                           mask_words, mask);
+  lists_kernel<<<(unsigned)((heads + 127) / 128), 128, 0, stream>>>(mask, (int64_t)heads, nkb, mask_words, counts,
+                                                                    lists);
+  return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
+}
+
 }  // namespace thrift

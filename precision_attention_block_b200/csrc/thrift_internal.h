@@ -41,4 +41,33 @@ thrift_status attn_launch(const void* q, const void* k, const void* v, const thr
 
 thrift_status wait_timeout_launch(int* status, long long limit, cudaStream_t stream);
 
+// ---- decode
+struct DecodeArgs {
+  const thrift_decode_cfg* cfg;
+  const void *q, *k, *v;
+  const thrift_nvfp4 *q4, *k4, *v4;  // q4: the query rows' NVFP4 copy (workspace)
+  const uint32_t* mask;
+  int mode;  // as attn_launch
+  void* out;
+  float* lse;
+  float* part_o;   // [B*Hkv, n_split, 16, d]
+  float* part_ml;  // [B*Hkv, n_split, 16, 2]
+  int* status;
+};
+
+// Upper bound of the number of key-block splits of a decode step with nkb key blocks.
+int decode_split_cap(int nkb);
+
+thrift_status decode_attn_launch(const DecodeArgs& a, cudaStream_t stream);
+
+thrift_status kv_means_launch(const void* k, int64_t outer, int32_t Nk, int32_t d, int32_t block_k, double* kbar,
+                              cudaStream_t stream);
+
+// Decode selection: qbar [B*Hq, d] and scores [B*Hq, nkb] live in `scratch`
+// (decode_select_scratch_bytes) unless scores_out is given.
+size_t decode_select_scratch_bytes(const thrift_decode_cfg& c);
+thrift_status decode_select_launch(const void* q, const double* kbar, const thrift_decode_cfg& c, uint32_t* mask,
+                                   int32_t* counts, int16_t* lists, double* scores_out, uint8_t* scratch,
+                                   cudaStream_t stream);
+
 }  // namespace thrift

@@ -95,3 +95,64 @@ def test_null_and_workspace_errors(L):
     assert L.thrift_attn_fwd(None, None, None, ctypes.byref(nv), ctypes.byref(nv), ctypes.byref(nv), p, p, p, p,
                              None, ctypes.byref(cfg(topk_bp=10000)), p, 256, None) == 1
     assert L.thrift_status_str(4) == b"device wait timed out"
+
+
+def dcfg(**kw):
+    from precision_attention_block_b200 import DecodeConfig
+    base = dict(B=1, Hq=32, Hkv=8, Nq=1, Nk=131072, d=128, causal=True, block_k=128, topk_bp=200)
+    base.update(kw)
+    return DecodeConfig(**base).c()
+
+
+def test_decode_workspace_sizes(L):
+    c = dcfg()
+    n = L.thrift_decode_workspace_bytes(ctypes.byref(c))
+    # at least the selection scratch (qbar + scores in float64) and the lists
+    assert n >= 256 + 32 * 128 * 8 + 32 * 1024 * 8 + 32 * 1024 * 2
+    assert n < 64 << 20
+    assert L.thrift_decode_workspace_bytes(ctypes.byref(dcfg(Nq=4))) > 0          # 4 heads x 4 rows = 16
+    assert L.thrift_decode_workspace_bytes(ctypes.byref(dcfg(Nq=1, Hkv=2))) > 0   # 16 heads x 1 row
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), 2), (dict(Hkv=5), 1), (dict(block_k=32), 2), (dict(Nk=1000), 2), (dict(topk_bp=20000), 1),
+    (dict(causal=2), 1), (dict(Nq=0), 1), (dict(Nq=5), 2), (dict(Hkv=1), 2), (dict(Nq=200, Nk=128), 1)])
+def test_bad_decode_config_rejected_on_host(L, kw, status):
+    c = dcfg(**kw)
+    assert L.thrift_decode_workspace_bytes(ctypes.byref(c)) == 0
+    p = ctypes.c_void_p(0x1000)
+    ws = ctypes.c_void_p(0x100000)
+    assert L.thrift_decode_attn(p, p, p, None, None, p, p, None, ctypes.byref(c), ws, 1 << 30, None) == status
+    assert L.thrift_decode_select(p, p, ctypes.byref(c), p, p, p, None, ws, 1 << 30, None) == status
+    assert L.thrift_decode_fwd(p, p, p, None, None, p, p, None, ctypes.byref(c), ws, 1 << 30, None) == status
+
+
+def test_decode_null_and_workspace_errors(L):
+    from precision_attention_block_b200 import _lib
+    c = dcfg()
+    p = ctypes.c_void_p(0x1000)
+    nv0 = _lib.CNVFP4(0x1000, 0x1000, 0x1000, 0x1000, 0)
+    nv1 = _lib.CNVFP4(0x1000, 0x1000, 0x1000, 0x1000, 1)
+    big = 1 << 40
+    # missing query rows, missing NVFP4 cache, wrong group axis, missing mask, misaligned pointers
+    assert L.thrift_decode_attn(None, p, p, ctypes.byref(nv0), ctypes.byref(nv1), p, p, None, ctypes.byref(c), p,
+                                big, None) == 1
+    assert L.thrift_decode_attn(p, p, p, None, None, p, p, None, ctypes.byref(c), p, big, None) == 1
+    assert L.thrift_decode_attn(p, p, p, ctypes.byref(nv1), ctypes.byref(nv1), p, p, None, ctypes.byref(c), p,
+                                big, None) == 1
+    assert L.thrift_decode_attn(p, p, p, ctypes.byref(nv0), ctypes.byref(nv1), None, p, None, ctypes.byref(c), p,
+                                big, None) == 1
+    odd = ctypes.c_void_p(0x1008)
+    assert L.thrift_decode_attn(odd, p, p, ctypes.byref(nv0), ctypes.byref(nv1), p, p, None, ctypes.byref(c), p,
+                                big, None) == 1
+    # all-FP16 needs no NVFP4 cache but the FP16 one; uniform NVFP4 needs no mask
+    assert L.thrift_decode_attn(p, None, None, None, None, None, p, None, ctypes.byref(dcfg(topk_bp=10000)), p,
+                                big, None) == 1
+    # workspace too small or misaligned
+    assert L.thrift_decode_attn(p, p, p, ctypes.byref(nv0), ctypes.byref(nv1), p, p, None, ctypes.byref(c), p,
+                                1024, None) == 5
+    assert L.thrift_decode_fwd(p, p, p, ctypes.byref(nv0), ctypes.byref(nv1), p, p, None, ctypes.byref(c),
+                               ctypes.c_void_p(0x1001), big, None) == 5
+    assert L.thrift_kv_block_means(None, 1, 128, 128, 64, p, None) == 1
+    assert L.thrift_kv_block_means(p, 1, 100, 128, 64, p, None) == 2
+    assert L.thrift_kv_block_means(p, 1, 128, 96, 64, p, None) == 2
