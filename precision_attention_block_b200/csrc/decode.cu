@@ -19,7 +19,8 @@
 //   attend     split over key blocks: CTA (split, batch * KV head) walks its key blocks.  A
 //              producer warp streams each block's NVFP4 K and V (and, when one of the group's
 //              heads selected the block, its FP16 K and V) into shared memory with bulk and
-//              tensor copies; eight consumer warps compute S = Q K^T, the per-row block maximum
+//              tensor copies; seven consumer warps, each on its own key blocks, compute S = Q K^T
+//              (fragments kept in registers), the per-row block maximum
 //              M, P^ = exp(S - M), the two-level NVFP4 re-quantisation of P^ (FP16 rounding on
 //              selected blocks), P V, and merge with weight exp(M - m) into FP32 partial sums;
 //   combine    the splits' partial (O, m, l) of each row into O / l (FP16) and lse.
@@ -45,12 +46,16 @@ namespace thrift {
 namespace {
 
 constexpr int kRowsMax = 16;           // query rows of one KV-head group (the MMA's M)
-constexpr int kConsumers = 256;        // eight consumer warps
+constexpr int kConsumers = 224;        // seven consumer warps (with the producer, 256 threads: up to 255 registers)
+constexpr int kConsumerWarps = kConsumers / 32;
+constexpr int kTab = 2048;             // key blocks of a split whose selection bits are staged
 constexpr int kThreads = kConsumers + 32;
 constexpr long long kWaitLimit = 1ll << 32;
 constexpr int kMinBlocksPerSplit = 4;
 constexpr int kMaxSplit = 320;
 constexpr float kNegInf = -__builtin_huge_valf();
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 
 struct DecodeParams {
   const __half* q;        // [B*Hq*Nq, D]
@@ -82,21 +87,24 @@ struct DLayout {
   static constexpr int OFF_K4S = K4C;
   static constexpr int OFF_V4C = K4C + K4S;
   static constexpr int OFF_V4S = OFF_V4C + V4C;
-  static constexpr int ST4 = OFF_V4S + V4S;            // one NVFP4 stage
+  static constexpr int ST4 = OFF_V4S + V4S;            // one NVFP4 stage: K codes, K scales, V codes, V scales
   static constexpr int ST16 = 2 * BK * D * 2;          // one FP16 slot: K then V
-  static constexpr int NST = 4;
-  static constexpr int NF = 1;
+  static constexpr int NST = BK == 64 ? 12 : 6;
+  static constexpr int NF = BK == 64 ? 2 : 1;
   static constexpr int OFF_ST16 = NST * ST4;
-  static constexpr int OFF_S = OFF_ST16 + NF * ST16;   // S   [16][BK] f32
-  static constexpr int OFF_PC = OFF_S + kRowsMax * BK * 4;       // P codes [16][BK/2]
-  static constexpr int OFF_PS = OFF_PC + kRowsMax * BK / 2;      // P scales [16][BK/16]
-  static constexpr int OFF_P16 = OFF_PS + ((kRowsMax * BK / 16 + 15) & ~15);  // P16 [16][BK]
-  static constexpr int OFF_Q16 = OFF_P16 + kRowsMax * BK * 2;    // Q16 [16][D]
-  static constexpr int OFF_ROW = OFF_Q16 + kRowsMax * D * 2;     // alpha, gq4, gq16 [16] each
-  static constexpr int OFF_BAR = OFF_ROW + 3 * kRowsMax * 4;
-  static constexpr int BAR_BYTES = 8 * (2 * NST + 2 * NF) + 16;
+  static constexpr int OFF_QA = OFF_ST16 + NF * ST16;           // query A fragments: NVFP4, then FP16
+  static constexpr int QA_BYTES = 2 * (D / 16) * 32 * 16;
+  static constexpr int OFF_PA = OFF_QA + QA_BYTES;              // per-warp P A fragments
+  static constexpr int PA_BYTES = kConsumerWarps * (BK / 16) * 32 * 16;
+  static constexpr int OFF_TAB = OFF_PA + PA_BYTES;             // FP16-head bits of the split's blocks
+  static constexpr int OFF_BAR = OFF_TAB + kTab * 2;
+  static constexpr int BAR_BYTES = 8 * (2 * NST + 2 * NF) + 4 * (NST + NF) + 16;
   static constexpr int SMEM = OFF_BAR + BAR_BYTES;
-  static_assert(ST4 % 128 == 0 && ST16 % 128 == 0 && OFF_S % 16 == 0 && OFF_BAR % 8 == 0, "alignment");
+  // after the main loop the consumer warps' partial results reuse the stage area
+  static constexpr int COMB_ML = kConsumerWarps * kRowsMax * D * 4;  // after [warps][16][D] f32 outputs
+  static_assert(COMB_ML + kConsumerWarps * kRowsMax * 2 * 4 <= OFF_QA, "combine area");
+  static_assert(ST4 % 128 == 0 && ST16 % 128 == 0 && OFF_QA % 16 == 0 && OFF_BAR % 8 == 0, "alignment");
+  static_assert(SMEM <= 232448, "shared memory");
 };
 
 // ------------------------------------------------------------------ device helpers
@@ -166,467 +174,531 @@ __device__ __forceinline__ uint32_t group_bits(const DecodeParams& p, int b, int
   return bits;
 }
 
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float lg2f(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Bounded wait until a shared word holds `want` (see tag4 in decode_attn_kernel).
+__device__ __forceinline__ bool wait_tag(volatile int* tag, int want, volatile int* abort_flag, int* status,
+                                         long long limit) {
+  if (*tag == want) return true;
+  const long long t0 = clock64();
+  while (*tag != want) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > limit) {
+      *abort_flag = 1;
+      if (status) atomicOr(status, kStatusTimeout);
+      return false;
+    }
+    __nanosleep(64);
+  }
+  return true;
+}
+
+// Key of column n of S n-tile nt.  Lane quad tig of a warp then holds the keys
+// [tig*BK/4, (tig+1)*BK/4) of its rows, and the S fragments of n-tiles 2ks and 2ks+1 are the A
+// fragment of k-step ks of P V with contraction slot 2*tig+e = key tig*BK/4 + 4*ks + e and slot
+// 8+2*tig+e = that key + 2: the order in which the lane reads V's token-grouped codes.
+template <int BK>
+__device__ __forceinline__ int key_of(int nt, int n) {
+  return (n >> 1) * (BK / 4) + 4 * (nt >> 1) + 2 * (nt & 1) + (n & 1);
+}
+
 template <int D, int BK>
-__global__ void __launch_bounds__(kThreads, BK == 64 ? 2 : 1) decode_attn_kernel(const __grid_constant__ CUtensorMap tm_v4c,
-                                                               const DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 1) decode_attn_kernel(const __grid_constant__ CUtensorMap tm_v4c,
+                                                                  const DecodeParams p) {
   using L = DLayout<D, BK>;
+  constexpr int NST = L::NST, NF = L::NF;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full4 = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint64_t* empty4 = full4 + L::NST;
-  uint64_t* full16 = empty4 + L::NST;
-  uint64_t* empty16 = full16 + L::NF;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty16 + L::NF);
+  uint64_t* empty4 = full4 + NST;
+  uint64_t* full16 = empty4 + NST;
+  uint64_t* empty16 = full16 + NF;
+  // tag4[s] / tag16[s]: the block (FP16-slot use) a stage (slot) is being filled for, written by
+  // the producer once the stage's previous use is released.  Consumers take blocks round-robin,
+  // so the warp that waits for a use of a stage may come before the warp of the stage's previous
+  // use has seen that one complete; a parity wait cannot tell those two phases apart, so a
+  // consumer first waits until the tag names its own use.
+  volatile int* tag4 = reinterpret_cast<volatile int*>(empty16 + NF);
+  volatile int* tag16 = tag4 + NST;
+  volatile int* abort_flag = tag16 + NF;
+  uint16_t* tab = reinterpret_cast<uint16_t*>(smem + L::OFF_TAB);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = blockIdx.y, split = blockIdx.x;
   const int b = grp / p.Hkv, hk = grp % p.Hkv;
   const int j0 = split * p.bps;
-  const int j1 = min(p.nkb, j0 + p.bps);
+  const int nblk = min(p.bps, p.nkb - j0);
   const uint32_t all_heads = (1u << p.G) - 1u;
+  const bool use4 = p.mode != 2;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < L::NST; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&full4[s], 1);
-      mbar_init(&empty4[s], kConsumers / 32);
+      mbar_init(&empty4[s], 1);
+      tag4[s] = -1;
     }
-    for (int s = 0; s < L::NF; ++s) {
+    for (int s = 0; s < NF; ++s) {
       mbar_init(&full16[s], 1);
-      mbar_init(&empty16[s], kConsumers / 32);
+      mbar_init(&empty16[s], 1);
+      tag16[s] = -1;
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // zero the P buffers once (rows that never hold probabilities stay finite), the row
-  // parameters of rows >= R, and stage the FP16 query rows
-  for (int i = threadIdx.x; i < (L::OFF_ROW - L::OFF_PC) / 4; i += blockDim.x)
-    reinterpret_cast<uint32_t*>(smem + L::OFF_PC)[i] = 0u;
-  __syncthreads();
   {
+    // The query rows as m16n8k16 A fragments, [k-step][lane] (rows >= R zero): dequantised NVFP4
+    // rows, then FP16 rows.  Contraction slot 2*tig+e of k-step ks holds d = tig*D/4 + 4*ks + e,
+    // slot 8+2*tig+e holds d + 2.  Also the selection bits of the split's first kTab blocks.
     const int64_t qrow0 = ((int64_t)b * p.Hq + (int64_t)hk * p.G) * p.Nq;
-    __half* q16 = reinterpret_cast<__half*>(smem + L::OFF_Q16);
-    for (int i = threadIdx.x; i < p.R * D; i += blockDim.x) q16[i] = p.q[qrow0 * D + i];
-    float* rowp = reinterpret_cast<float*>(smem + L::OFF_ROW);
-    if (threadIdx.x < kRowsMax) {
-      rowp[threadIdx.x] = 1.0f;               // alpha
-      rowp[kRowsMax + threadIdx.x] = 0.0f;    // gq4
-      rowp[2 * kRowsMax + threadIdx.x] = 0.0f;  // gq16
+    uint4* qa = reinterpret_cast<uint4*>(smem + L::OFF_QA);
+    for (int f = threadIdx.x; f < 2 * (D / 16) * 32; f += blockDim.x) {
+      const bool fp16 = f >= (D / 16) * 32;
+      const int ks = (f % ((D / 16) * 32)) / 32, ln = f % 32;
+      const int gg = ln >> 2, tg = ln & 3;
+      const int d0 = tg * (D / 4) + 4 * ks;
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int rs = 0; rs < 2; ++rs) {
+        const int r = gg + 8 * rs;
+        if (r >= p.R) continue;
+        if (fp16) {
+          const __half* qr = p.q + (qrow0 + r) * D + d0;
+          w[rs] = *reinterpret_cast<const uint32_t*>(qr);
+          w[2 + rs] = *reinterpret_cast<const uint32_t*>(qr + 2);
+        } else if (use4) {
+          const uint8_t* qc = p.q4c + (qrow0 + r) * (D / 2);
+          const uint32_t sc = e4m3_to_h2x(__ldg(p.q4s + (qrow0 + r) * (D / 16) + d0 / 16));
+          w[rs] = hmul2(e2m1x2_to_h2(__ldg(qc + d0 / 2)), sc);
+          w[2 + rs] = hmul2(e2m1x2_to_h2(__ldg(qc + d0 / 2 + 1)), sc);
+        }
+      }
+      qa[f] = make_uint4(w[0], w[1], w[2], w[3]);
     }
+    for (int i = threadIdx.x; i < min(nblk, kTab); i += blockDim.x) tab[i] = (uint16_t)group_bits(p, b, hk, j0 + i);
   }
   __syncthreads();
+  auto bits_of = [&](int i) -> uint32_t { return i < kTab ? (uint32_t)tab[i] : group_bits(p, b, hk, j0 + i); };
 
-  if (warp == kConsumers / 32) {
+  if (warp == kConsumerWarps) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       prefetch_tmap(&tm_v4c);
       const int64_t krow0 = (int64_t)grp * p.Nk;
       const int vrow0 = grp * D;  // first V code row of this KV head
       const int64_t vsf_block = (int64_t)(vrow0 >> 7) * (p.Nk / 64);
-      int c4 = 0, c16 = 0;
+      int c16 = 0;
       bool ok = true;
-      for (int j = j0; j < j1 && ok; ++j) {
-        const uint32_t bits = group_bits(p, b, hk, j);
-        if (bits != all_heads) {
-          const int s = c4 % L::NST;
-          ok = mbar_wait(&empty4[s], ((c4 / L::NST) & 1) ^ 1, abort_flag, p.status, p.wait_limit);
+      for (int i = 0; i < nblk && ok; ++i) {
+        const int j = j0 + i;
+        const uint32_t bits = bits_of(i);
+        const int64_t kr = krow0 + (int64_t)j * BK;
+        if (use4) {
+          const int s = i % NST;
+          ok = mbar_wait(&empty4[s], ((i / NST) & 1) ^ 1, abort_flag, p.status, p.wait_limit);
           if (!ok) break;
           uint8_t* st = smem + s * L::ST4;
+          tag4[s] = i;
           mbar_arrive_expect_tx(&full4[s], L::ST4);
-          const int64_t kr = krow0 + (int64_t)j * BK;
           bulk_load(st, p.k4c + kr * (D / 2), L::K4C, &full4[s]);
           bulk_load(st + L::OFF_K4S, p.k4s + kr * (D / 16), L::K4S, &full4[s]);
           tma_load_2d(st + L::OFF_V4C, &tm_v4c, &full4[s], j * (BK / 2), vrow0);
           bulk_load(st + L::OFF_V4S, p.v4sm + (vsf_block + (int64_t)j * (BK / 64)) * 512, L::V4S, &full4[s]);
-          ++c4;
         }
         if (bits != 0u) {
-          const int s = c16 % L::NF;
-          ok = mbar_wait(&empty16[s], ((c16 / L::NF) & 1) ^ 1, abort_flag, p.status, p.wait_limit);
+          const int s = c16 % NF;
+          ok = mbar_wait(&empty16[s], ((c16 / NF) & 1) ^ 1, abort_flag, p.status, p.wait_limit);
           if (!ok) break;
           uint8_t* st = smem + L::OFF_ST16 + s * L::ST16;
+          tag16[s] = c16;
           mbar_arrive_expect_tx(&full16[s], L::ST16);
-          const int64_t kr = krow0 + (int64_t)j * BK;
           bulk_load(st, p.k16 + kr * D, BK * D * 2, &full16[s]);
           bulk_load(st + BK * D * 2, p.v16 + kr * D, BK * D * 2, &full16[s]);
           ++c16;
         }
       }
       // every copy issued must land before the CTA exits: wait (bounded) for the last fill of
-      // each stage; on the normal path the consumers have already waited for all of them
-      for (int i = 0; i < L::NST && i < c4; ++i) {
-        const int c = c4 - 1 - i;
-        mbar_wait(&full4[c % L::NST], (c / L::NST) & 1, abort_flag, nullptr, p.wait_limit);
-      }
-      for (int i = 0; i < L::NF && i < c16; ++i) {
-        const int c = c16 - 1 - i;
-        mbar_wait(&full16[c % L::NF], (c / L::NF) & 1, abort_flag, nullptr, p.wait_limit);
-      }
+      // each stage and slot; on the normal path the consumers have already waited for them
+      if (use4)
+        for (int i = max(0, nblk - NST); i < nblk; ++i)
+          mbar_wait(&full4[i % NST], (i / NST) & 1, abort_flag, nullptr, p.wait_limit);
+      for (int c = max(0, c16 - NF); c < c16; ++c)
+        mbar_wait(&full16[c % NF], (c / NF) & 1, abort_flag, nullptr, p.wait_limit);
     }
     return;
   }
 
   // ------------------------------------------------------------------ consumers
+  // Warp w takes the split's blocks w, w + 7, ...; each warp keeps its own output, maximum and
+  // denominator for rows g and g + 8, combined with the other warps' at the end.
   const int g = lane >> 2, tig = lane & 3;
   const int R = p.R;
-  const float sv4 = (p.mode == 2 ? 0.0f : __ldg(p.v_ts)) * (1.0f / 2688.0f);
-  const float mult4 = p.mode == 2 ? 0.0f : p.tau * __ldg(p.q_ts) * __ldg(p.k_ts);
-  const int64_t qrow0 = ((int64_t)b * p.Hq + (int64_t)hk * p.G) * p.Nq;
+  const float sv4 = use4 ? __ldg(p.v_ts) * (1.0f / 2688.0f) : 0.0f;
+  const float sl4 = use4 ? p.tau * __ldg(p.q_ts) * __ldg(p.k_ts) * kLog2e : 0.0f;  // FP4 score -> log2 units
+  const float sl16 = p.tau * kLog2e;
+  const int64_t qpos0 = (int64_t)p.Nk - p.Nq;  // position of query row 0 among the keys
+  const uint4* qa4 = reinterpret_cast<const uint4*>(smem + L::OFF_QA);             // [D/16][32] A fragments
+  const uint4* qa16 = qa4 + (D / 16) * 32;
+  uint4* pa_w = reinterpret_cast<uint4*>(smem + L::OFF_PA) + warp * (BK / 16) * 32;  // this warp's P fragments
+  const int vrow_in_blk = (grp * D) & 127;  // this head's first row inside its 128-row scale block
+  // query row r is the (r % Nq)-th row of head hk*G + r/Nq
+  const int hrow[2] = {g / p.Nq, (g + 8) / p.Nq};
+  const int64_t qpos[2] = {qpos0 + g % p.Nq, qpos0 + (g + 8) % p.Nq};
 
-  // dequantised NVFP4 query rows as m16n8k16 A fragments (rows >= R are zero); contraction
-  // slot 2*tig+e of k-step ks holds d = tig*D/4 + 4*ks + e, slot 8+2*tig+e holds d + 2
-  uint32_t qa[D / 16][4];
+  float o[D / 8][4];
 #pragma unroll
-  for (int ks = 0; ks < D / 16; ++ks)
+  for (int t = 0; t < D / 8; ++t)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) qa[ks][i] = 0u;
-  if (p.mode != 2) {
+    for (int e = 0; e < 4; ++e) o[t][e] = 0.0f;
+  float m_ref[2] = {kNegInf, kNegInf}, l_run[2] = {0.0f, 0.0f};  // m in log2 units
+
+  int scan_i = 0, c16_acc = 0;
+  bool ok = true;
+  for (int i = warp; i < nblk; i += kConsumerWarps) {
+    while (scan_i < i) c16_acc += bits_of(scan_i++) != 0u ? 1 : 0;
+    const int j = j0 + i;
+    const uint32_t bits = bits_of(i);
+    const bool n16 = bits != 0u, n4 = use4 && bits != all_heads;
+    const int s4 = i % NST, s16 = c16_acc % NF;
+    if (use4) {
+      ok = wait_tag(&tag4[s4], i, abort_flag, p.status, p.wait_limit);
+      ok = ok && mbar_wait(&full4[s4], (i / NST) & 1, abort_flag, p.status, p.wait_limit);
+    }
+    if (ok && n16) {
+      ok = wait_tag(&tag16[s16], c16_acc, abort_flag, p.status, p.wait_limit);
+      ok = ok && mbar_wait(&full16[s16], (c16_acc / NF) & 1, abort_flag, p.status, p.wait_limit);
+    }
+    if (!ok) break;
+    const uint8_t* st4 = smem + s4 * L::ST4;
+    const uint8_t* st16 = smem + L::OFF_ST16 + s16 * L::ST16;
+    const bool f16r[2] = {((bits >> hrow[0]) & 1u) != 0u, ((bits >> hrow[1]) & 1u) != 0u};
+
+    // ---- S = Q K^T (log2 units); n-tile nt holds keys key_of(nt, .).  NVFP4 pass, then FP16 pass
+    // for the rows whose head selected the block.
+    float sc[BK / 8][4];
+    {
+      float c[BK / 8][4];
+      if (n4) {
+#pragma unroll
+        for (int nt = 0; nt < BK / 8; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) c[nt][e] = 0.0f;
+#pragma unroll
+        for (int q = 0; q < D / 64; ++q) {  // the lane's 16-element scale group q
+          uint32_t sk[BK / 8];
+#pragma unroll
+          for (int nt = 0; nt < BK / 8; ++nt)
+            sk[nt] = e4m3_to_h2x(st4[L::OFF_K4S + key_of<BK>(nt, g) * (D / 16) + tig * (D / 64) + q]);
+#pragma unroll 1
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int ks = 4 * q + k4;
+            const uint4 a4 = qa4[ks * 32 + lane];
+            const uint32_t a[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+            for (int nt = 0; nt < BK / 8; ++nt) {
+              const uint32_t two =
+                  *reinterpret_cast<const uint16_t*>(st4 + key_of<BK>(nt, g) * (D / 2) + tig * (D / 8) + 2 * ks);
+              mma16816(c[nt], a, hmul2(e2m1x2_to_h2(two & 0xFFu), sk[nt]), hmul2(e2m1x2_to_h2(two >> 8), sk[nt]));
+            }
+          }
+        }
+#pragma unroll
+        for (int nt = 0; nt < BK / 8; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[nt][e] = c[nt][e] * sl4;
+      }
+      if (n16) {
+#pragma unroll
+        for (int nt = 0; nt < BK / 8; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) c[nt][e] = 0.0f;
+#pragma unroll 1
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint4 a4 = qa16[ks * 32 + lane];
+          const uint32_t a[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+          for (int nt = 0; nt < BK / 8; ++nt) {
+            const uint2 bw = *reinterpret_cast<const uint2*>(reinterpret_cast<const __half*>(st16) +
+                                                             key_of<BK>(nt, g) * D + tig * (D / 4) + 4 * ks);
+            mma16816(c[nt], a, bw.x, bw.y);
+          }
+        }
+#pragma unroll
+        for (int nt = 0; nt < BK / 8; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (f16r[e >> 1] || !n4) sc[nt][e] = c[nt][e] * sl16;
+      }
+#pragma unroll
+      for (int nt = 0; nt < BK / 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int rs = e >> 1;
+          const int kk = tig * (BK / 4) + 4 * (nt >> 1) + 2 * (nt & 1) + (e & 1);
+          if (g + 8 * rs >= R || (p.causal && (int64_t)j * BK + kk > qpos[rs])) sc[nt][e] = kNegInf;
+        }
+    }
+
+    // ---- per row: block maximum, probabilities (re-quantised for NVFP4 rows), merge weights
+    uint32_t pa[BK / 8][2];  // P V A fragments: pa[nt][rs] = keys of S n-tile nt, row g + 8 rs
+    float al[2], w4[2], w16[2];
+#pragma unroll
+    for (int rs = 0; rs < 2; ++rs) {
+      float mx = kNegInf;
+#pragma unroll
+      for (int nt = 0; nt < BK / 8; ++nt) mx = fmaxf(mx, fmaxf(sc[nt][2 * rs], sc[nt][2 * rs + 1]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      const float M = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      float sum = 0.0f;
+      if (M == kNegInf) {  // row >= R, or no key of this block visible to it
+#pragma unroll
+        for (int nt = 0; nt < BK / 8; ++nt) pa[nt][rs] = 0u;
+      } else if (!f16r[rs]) {
+        // P' = 2688 exp(S - M); s_b = E4M3(max16 P' / 6) per 16 keys (the lane's keys hold whole
+        // groups); code = E2M1(P' / s_b) evaluated as exp2(S - M + log2(2688 / s_b))
+#pragma unroll
+        for (int q = 0; q < BK / 64; ++q) {
+          float gm = kNegInf;
+#pragma unroll
+          for (int nt = 8 * q; nt < 8 * q + 8; ++nt) gm = fmaxf(gm, fmaxf(sc[nt][2 * rs], sc[nt][2 * rs + 1]));
+          const float pm = gm != kNegInf ? 448.0f * ex2f(gm - M) : 0.0f;
+          const uint32_t sb = cvt_e4m3(pm);
+          const float sbv = e4m3_to_f32(sb);
+          const float sbe = sbv > 0.0f ? sbv : 448.0f;
+          const float bias = (11.392317422778761f - lg2f(sbe)) - M;  // log2(2688 / s_b) - M
+          const uint32_t sb2 = e4m3_to_h2x(sb);
+          float gs = 0.0f;
+#pragma unroll
+          for (int nt = 8 * q; nt < 8 * q + 8; ++nt) {
+            const float y0 = ex2f(sc[nt][2 * rs] + bias), y1 = ex2f(sc[nt][2 * rs + 1] + bias);
+            gs += y0 + y1;
+            pa[nt][rs] = hmul2(e2m1x2_to_h2(cvt_e2m1x2(y0, y1)), sb2);  // code * s_b, exact in FP16
+          }
+          sum = fmaf(gs, sbe * (1.0f / 2688.0f), sum);
+        }
+      } else {
+#pragma unroll
+        for (int nt = 0; nt < BK / 8; ++nt) {
+          const float p0 = ex2f(sc[nt][2 * rs] - M), p1 = ex2f(sc[nt][2 * rs + 1] - M);
+          sum += p0 + p1;
+          pa[nt][rs] = pack_h2(p0, p1);
+        }
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      if (M == kNegInf) {
+        al[rs] = 1.0f;
+        w4[rs] = w16[rs] = 0.0f;
+      } else {
+        const float m_new = fmaxf(m_ref[rs], M);
+        al[rs] = m_ref[rs] == kNegInf ? 0.0f : ex2f(m_ref[rs] - m_new);
+        const float gw = ex2f(M - m_new);
+        l_run[rs] = l_run[rs] * al[rs] + gw * sum;
+        m_ref[rs] = m_new;
+        w4[rs] = f16r[rs] ? 0.0f : gw * sv4;
+        w16[rs] = f16r[rs] ? gw : 0.0f;
+      }
+    }
+    // the A fragment of k-step ks is S n-tiles 2ks and 2ks + 1 (rows g, g + 8)
+#pragma unroll
+    for (int ks = 0; ks < BK / 16; ++ks)
+      pa_w[ks * 32 + lane] = make_uint4(pa[2 * ks][0], pa[2 * ks][1], pa[2 * ks + 1][0], pa[2 * ks + 1][1]);
+    __syncwarp();
+    if (__any_sync(0xffffffffu, al[0] != 1.0f || al[1] != 1.0f)) {
+#pragma unroll
+      for (int t = 0; t < D / 8; ++t) {
+        o[t][0] *= al[0];
+        o[t][1] *= al[0];
+        o[t][2] *= al[1];
+        o[t][3] *= al[1];
+      }
+    }
+
+    // ---- P V into the running output; n-tile t holds output columns 8t .. 8t + 7.  NVFP4 pass
+    // (rows of NVFP4 heads carry weight w4), then FP16 pass (weight w16).
+    {
+      float c[D / 8][4];
+      if (n4) {
+#pragma unroll
+        for (int t = 0; t < D / 8; ++t)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) c[t][e] = 0.0f;
+#pragma unroll
+        for (int q = 0; q < BK / 64; ++q) {  // the lane's 16-key scale group q
+          uint32_t vsc[D / 8];
+#pragma unroll
+          for (int t = 0; t < D / 8; ++t) {
+            const int crow = vrow_in_blk + t * 8 + g;
+            const int gg = tig * (BK / 64) + q;  // 16-key group within the block
+            vsc[t] = e4m3_to_h2x(st4[L::OFF_V4S + (gg >> 2) * 512 + (crow & 31) * 16 + ((crow >> 5) & 3) * 4 + (gg & 3)]);
+          }
+#pragma unroll 1
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int ks = 4 * q + k4;
+            const uint4 a4 = pa_w[ks * 32 + lane];
+            const uint32_t a[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+            for (int t = 0; t < D / 8; ++t) {
+              const uint32_t two = *reinterpret_cast<const uint16_t*>(st4 + L::OFF_V4C + (t * 8 + g) * (BK / 2) +
+                                                                      tig * (BK / 8) + 2 * ks);
+              mma16816(c[t], a, hmul2(e2m1x2_to_h2(two & 0xFFu), vsc[t]), hmul2(e2m1x2_to_h2(two >> 8), vsc[t]));
+            }
+          }
+        }
+#pragma unroll
+        for (int t = 0; t < D / 8; ++t)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[t][e] = fmaf(w4[e >> 1], c[t][e], o[t][e]);
+      }
+      if (n16) {
+#pragma unroll
+        for (int t = 0; t < D / 8; ++t)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) c[t][e] = 0.0f;
+        const __half* vr = reinterpret_cast<const __half*>(st16 + BK * D * 2);
+#pragma unroll 1
+        for (int ks = 0; ks < BK / 16; ++ks) {
+          const uint4 a4 = pa_w[ks * 32 + lane];
+          const uint32_t a[4] = {a4.x, a4.y, a4.z, a4.w};
+          const int k0 = tig * (BK / 4) + 4 * ks;
+#pragma unroll
+          for (int t = 0; t < D / 8; ++t) {
+            const int n = t * 8 + g;
+            const __half2 b0h = __halves2half2(vr[(k0 + 0) * D + n], vr[(k0 + 1) * D + n]);
+            const __half2 b1h = __halves2half2(vr[(k0 + 2) * D + n], vr[(k0 + 3) * D + n]);
+            mma16816(c[t], a, *reinterpret_cast<const uint32_t*>(&b0h), *reinterpret_cast<const uint32_t*>(&b1h));
+          }
+        }
+#pragma unroll
+        for (int t = 0; t < D / 8; ++t)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[t][e] = fmaf(w16[e >> 1], c[t][e], o[t][e]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      if (use4) mbar_arrive(&empty4[s4]);
+      if (n16) mbar_arrive(&empty16[s16]);
+    }
+  }
+
+  // ---- combine the consumer warps' partial results of this split (through the stage area: every
+  // copy has landed and been read once all consumer warps are past their loops)
+  if (named_sync_or(!ok)) return;
+  float* co = reinterpret_cast<float*>(smem);
+  float* cml = reinterpret_cast<float*>(smem + L::COMB_ML);
+#pragma unroll
+  for (int t = 0; t < D / 8; ++t) {
+    const int col = t * 8 + 2 * tig;
+#pragma unroll
+    for (int rs = 0; rs < 2; ++rs) {
+      const int r = g + 8 * rs;
+      if (r < R)
+        *reinterpret_cast<float2*>(co + (warp * kRowsMax + r) * D + col) = make_float2(o[t][2 * rs], o[t][2 * rs + 1]);
+    }
+  }
+  if (tig == 0) {
 #pragma unroll
     for (int rs = 0; rs < 2; ++rs) {
       const int r = g + 8 * rs;
       if (r < R) {
-        const uint8_t* qc = p.q4c + (qrow0 + r) * (D / 2);
-        const uint8_t* qs = p.q4s + (qrow0 + r) * (D / 16);
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const int d0 = tig * (D / 4) + 4 * ks;
-          const uint32_t sc = e4m3_to_h2x(__ldg(qs + d0 / 16));
-          qa[ks][rs] = hmul2(e2m1x2_to_h2(__ldg(qc + d0 / 2)), sc);
-          qa[ks][2 + rs] = hmul2(e2m1x2_to_h2(__ldg(qc + d0 / 2 + 1)), sc);
-        }
+        cml[(warp * kRowsMax + r) * 2] = m_ref[rs];
+        cml[(warp * kRowsMax + r) * 2 + 1] = l_run[rs];
       }
     }
   }
-
-  constexpr int NT_QK = BK / 8 / 8;   // key n-tiles per warp
-  constexpr int NT_PV = D / 8 / 8;    // output-column n-tiles per warp
-  constexpr int KPL = BK / 32;        // keys per lane in the softmax
-  float o[NT_PV][4];
+  named_sync();
+  float* po = p.part_o + ((int64_t)grp * p.n_split + split) * kRowsMax * D;
+  float* pml = p.part_ml + ((int64_t)grp * p.n_split + split) * kRowsMax * 2;
+  for (int idx = threadIdx.x; idx < R * D; idx += kConsumers) {
+    const int r = idx / D;
+    float m = kNegInf;
 #pragma unroll
-  for (int t = 0; t < NT_PV; ++t)
+    for (int w = 0; w < kConsumerWarps; ++w) m = fmaxf(m, cml[(w * kRowsMax + r) * 2]);
+    float acc = 0.0f, l = 0.0f;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o[t][e] = 0.0f;
-  // running maximum and denominator of rows warp and warp + 8 (replicated over the warp)
-  float m_run[2] = {kNegInf, kNegInf}, l_run[2] = {0.0f, 0.0f};
-
-  float* S = reinterpret_cast<float*>(smem + L::OFF_S);
-  uint8_t* PC = smem + L::OFF_PC;
-  uint8_t* PS = smem + L::OFF_PS;
-  __half* P16 = reinterpret_cast<__half*>(smem + L::OFF_P16);
-  const __half* Q16 = reinterpret_cast<const __half*>(smem + L::OFF_Q16);
-  float* alpha_s = reinterpret_cast<float*>(smem + L::OFF_ROW);
-  float* gq4_s = alpha_s + kRowsMax;
-  float* gq16_s = gq4_s + kRowsMax;
-  const int vrow_in_blk = (grp * D) & 127;  // this head's first row inside its 128-row scale block
-  const int64_t qpos0 = (int64_t)p.Nk - p.Nq;  // position of query row 0 among the keys
-
-  int c4 = 0, c16 = 0;
-  bool ok = true;
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t bits = group_bits(p, b, hk, j);
-    const bool n4 = bits != all_heads, n16 = bits != 0u;
-    const int s4 = c4 % L::NST, s16 = c16 % L::NF;
-    if (n4) ok = ok && mbar_wait(&full4[s4], (c4 / L::NST) & 1, abort_flag, p.status, p.wait_limit);
-    if (n16) ok = ok && mbar_wait(&full16[s16], (c16 / L::NF) & 1, abort_flag, p.status, p.wait_limit);
-    const uint8_t* st4 = smem + s4 * L::ST4;
-    const uint8_t* st16 = smem + L::OFF_ST16 + s16 * L::ST16;
-
-    // ---- S = Q K^T for the warp's key n-tiles
-    if (ok) {
-#pragma unroll
-      for (int t = 0; t < NT_QK; ++t) {
-        const int nt = warp + 8 * t;
-        const int key = nt * 8 + g;
-        float c4r[4] = {0.f, 0.f, 0.f, 0.f}, c16r[4] = {0.f, 0.f, 0.f, 0.f};
-        if (n4) {
-          const uint8_t* kc = st4 + key * (D / 2) + tig * (D / 8);
-          uint32_t w[D / 32];
-          if constexpr (D == 128) {
-            const uint4 v = *reinterpret_cast<const uint4*>(kc);
-            w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-          } else {
-            const uint2 v = *reinterpret_cast<const uint2*>(kc);
-            w[0] = v.x; w[1] = v.y;
-          }
-          const uint8_t* ksc = st4 + L::OFF_K4S + key * (D / 16) + tig * (D / 64);
-          uint32_t sc[D / 64];
-#pragma unroll
-          for (int i = 0; i < D / 64; ++i) sc[i] = e4m3_to_h2x(ksc[i]);
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t word = w[ks >> 1];
-            const int sh = (ks & 1) * 16;
-            const uint32_t s2 = sc[ks >> 2];
-            const uint32_t b0 = hmul2(e2m1x2_to_h2((word >> sh) & 0xFFu), s2);
-            const uint32_t b1 = hmul2(e2m1x2_to_h2((word >> (sh + 8)) & 0xFFu), s2);
-            mma16816(c4r, qa[ks], b0, b1);
-          }
-        }
-        if (n16) {
-          const __half* kr = reinterpret_cast<const __half*>(st16) + key * D + tig * (D / 4);
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint2 bw = *reinterpret_cast<const uint2*>(kr + 4 * ks);
-            const int d0 = tig * (D / 4) + 4 * ks;
-            uint32_t a[4];
-            a[0] = *reinterpret_cast<const uint32_t*>(Q16 + g * D + d0);
-            a[1] = *reinterpret_cast<const uint32_t*>(Q16 + (g + 8) * D + d0);
-            a[2] = *reinterpret_cast<const uint32_t*>(Q16 + g * D + d0 + 2);
-            a[3] = *reinterpret_cast<const uint32_t*>(Q16 + (g + 8) * D + d0 + 2);
-            if (g >= R) a[0] = a[2] = 0u;
-            if (g + 8 >= R) a[1] = a[3] = 0u;
-            mma16816(c16r, a, bw.x, bw.y);
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int r = g + 8 * (e >> 1);
-          const int kk = nt * 8 + 2 * tig + (e & 1);
-          float v = kNegInf;
-          if (r < R) {
-            const bool f16 = (bits >> (r / p.Nq)) & 1u;
-            v = f16 ? c16r[e] * p.tau : c4r[e] * mult4;
-            if (p.causal && (int64_t)j * BK + kk > qpos0 + (r % p.Nq)) v = kNegInf;
-          }
-          S[r * BK + kk] = v;
-        }
-      }
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float mw = cml[(w * kRowsMax + r) * 2];
+      const float f = (mw == kNegInf) ? 0.0f : ex2f(mw - m);
+      acc = fmaf(f, co[(w * kRowsMax + r) * D + idx % D], acc);
+      l = fmaf(f, cml[(w * kRowsMax + r) * 2 + 1], l);
     }
-    // every consumer warp passes each barrier; a failed wait anywhere stops all of them here
-    if (named_sync_or(!ok)) {
-      ok = false;
-      break;
-    }
-
-    // ---- softmax, re-quantisation and merge weights for rows warp and warp + 8
-#pragma unroll
-    for (int rs = 0; rs < 2; ++rs) {
-      const int r = warp + 8 * rs;
-      if (r >= R) continue;
-      float s[KPL];
-#pragma unroll
-      for (int t = 0; t < KPL; ++t) s[t] = S[r * BK + lane * KPL + t];
-      float mx = s[0];
-#pragma unroll
-      for (int t = 1; t < KPL; ++t) mx = fmaxf(mx, s[t]);
-      const float M = warp_max(mx);
-      const bool f16 = (bits >> (r / p.Nq)) & 1u;
-      if (M == kNegInf) {  // no key of this block is visible to the row
-        if (lane == 0) {
-          alpha_s[r] = 1.0f;
-          gq4_s[r] = 0.0f;
-          gq16_s[r] = 0.0f;
-        }
-        continue;
-      }
-      float ph[KPL];
-      float sum = 0.0f;
-#pragma unroll
-      for (int t = 0; t < KPL; ++t) {
-        ph[t] = s[t] == kNegInf ? 0.0f : expf(s[t] - M);
-        sum += ph[t];
-      }
-      sum = warp_sum(sum);
-      if (f16) {
-#pragma unroll
-        for (int t = 0; t < KPL; ++t) P16[r * BK + lane * KPL + t] = __float2half_rn(ph[t]);
-      } else {
-        // P' = 2688 P^; s_b = E4M3(amax16(P') / 6); code = E2M1(P' / s_b)
-        float pp[KPL];
-        float am = 0.0f;
-#pragma unroll
-        for (int t = 0; t < KPL; ++t) {
-          pp[t] = __fmul_rn(2688.0f, ph[t]);
-          am = fmaxf(am, pp[t]);
-        }
-#pragma unroll
-        for (int o = 1; o < 16 / KPL; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-        const uint32_t sb = cvt_e4m3(__fdiv_rn(am, 6.0f));
-        const float sbv = e4m3_to_f32(sb);
-        uint32_t byte0 = 0u, byte1 = 0u;
-        if (sbv > 0.0f) {
-          byte0 = cvt_e2m1x2(__fdiv_rn(pp[0], sbv), __fdiv_rn(pp[1], sbv));
-          if constexpr (KPL == 4) byte1 = cvt_e2m1x2(__fdiv_rn(pp[2], sbv), __fdiv_rn(pp[3], sbv));
-        }
-        if constexpr (KPL == 2) {
-          PC[r * (BK / 2) + lane] = (uint8_t)byte0;
-        } else {
-          *reinterpret_cast<uint16_t*>(PC + r * (BK / 2) + 2 * lane) = (uint16_t)(byte0 | (byte1 << 8));
-        }
-        if ((lane & (16 / KPL - 1)) == 0) PS[r * (BK / 16) + lane * KPL / 16] = (uint8_t)sb;
-      }
-      const float m_new = fmaxf(m_run[rs], M);
-      const float alpha = m_run[rs] == kNegInf ? 0.0f : expf(m_run[rs] - m_new);
-      const float gw = expf(M - m_new);
-      l_run[rs] = l_run[rs] * alpha + gw * sum;
-      m_run[rs] = m_new;
-      if (lane == 0) {
-        alpha_s[r] = alpha;
-        gq4_s[r] = f16 ? 0.0f : gw * sv4;
-        gq16_s[r] = f16 ? gw : 0.0f;
-      }
-    }
-    named_sync();
-
-    // ---- P V for the warp's output-column n-tiles, merged into the partial output
-    {
-      float al[2], w4[2], w16[2];
-#pragma unroll
-      for (int rs = 0; rs < 2; ++rs) {
-        al[rs] = alpha_s[g + 8 * rs];
-        w4[rs] = gq4_s[g + 8 * rs];
-        w16[rs] = gq16_s[g + 8 * rs];
-      }
-      // P operand (rows g and g + 8): slot 2*tig+e of k-step ks holds key tig*BK/4 + 4*ks + e
-      uint32_t pw[2][BK / 32];
-      uint32_t psc[2][BK / 64];
-      if (n4) {
-#pragma unroll
-        for (int rs = 0; rs < 2; ++rs) {
-          const uint8_t* pc = PC + (g + 8 * rs) * (BK / 2) + tig * (BK / 8);
-          if constexpr (BK == 64) {
-            const uint2 v = *reinterpret_cast<const uint2*>(pc);
-            pw[rs][0] = v.x; pw[rs][1] = v.y;
-          } else {
-            const uint4 v = *reinterpret_cast<const uint4*>(pc);
-            pw[rs][0] = v.x; pw[rs][1] = v.y; pw[rs][2] = v.z; pw[rs][3] = v.w;
-          }
-#pragma unroll
-          for (int i = 0; i < BK / 64; ++i) psc[rs][i] = e4m3_to_h2x(PS[(g + 8 * rs) * (BK / 16) + tig * (BK / 64) + i]);
-        }
-      }
-#pragma unroll
-      for (int t = 0; t < NT_PV; ++t) {
-        const int nt = warp + 8 * t;
-        const int n = nt * 8 + g;  // output column (d index) of this lane's B fragment
-        float c4r[4] = {0.f, 0.f, 0.f, 0.f}, c16r[4] = {0.f, 0.f, 0.f, 0.f};
-        if (n4) {
-          const uint8_t* vc = st4 + L::OFF_V4C + n * (BK / 2) + tig * (BK / 8);
-          uint32_t vw[BK / 32];
-          if constexpr (BK == 64) {
-            const uint2 v = *reinterpret_cast<const uint2*>(vc);
-            vw[0] = v.x; vw[1] = v.y;
-          } else {
-            const uint4 v = *reinterpret_cast<const uint4*>(vc);
-            vw[0] = v.x; vw[1] = v.y; vw[2] = v.z; vw[3] = v.w;
-          }
-          const int crow = vrow_in_blk + n;
-          uint32_t vsc[BK / 64];
-#pragma unroll
-          for (int i = 0; i < BK / 64; ++i) {
-            const int gg = tig * (BK / 64) + i;  // 16-key group within the block
-            vsc[i] = e4m3_to_h2x(st4[L::OFF_V4S + (gg >> 2) * 512 + (crow & 31) * 16 + ((crow >> 5) & 3) * 4 + (gg & 3)]);
-          }
-#pragma unroll
-          for (int ks = 0; ks < BK / 16; ++ks) {
-            const int sh = (ks & 1) * 16;
-            uint32_t a[4];
-#pragma unroll
-            for (int rs = 0; rs < 2; ++rs) {
-              const uint32_t word = pw[rs][ks >> 1];
-              a[rs] = hmul2(e2m1x2_to_h2((word >> sh) & 0xFFu), psc[rs][ks >> 2]);
-              a[2 + rs] = hmul2(e2m1x2_to_h2((word >> (sh + 8)) & 0xFFu), psc[rs][ks >> 2]);
-            }
-            const uint32_t word = vw[ks >> 1];
-            const uint32_t b0 = hmul2(e2m1x2_to_h2((word >> sh) & 0xFFu), vsc[ks >> 2]);
-            const uint32_t b1 = hmul2(e2m1x2_to_h2((word >> (sh + 8)) & 0xFFu), vsc[ks >> 2]);
-            mma16816(c4r, a, b0, b1);
-          }
-        }
-        if (n16) {
-          const __half* vr = reinterpret_cast<const __half*>(st16 + BK * D * 2);
-#pragma unroll
-          for (int ks = 0; ks < BK / 16; ++ks) {
-            const int k0 = tig * (BK / 4) + 4 * ks;
-            uint32_t a[4];
-#pragma unroll
-            for (int rs = 0; rs < 2; ++rs) {
-              const uint2 pw16 = *reinterpret_cast<const uint2*>(P16 + (g + 8 * rs) * BK + k0);
-              a[rs] = pw16.x;
-              a[2 + rs] = pw16.y;
-            }
-            const __half2 b0h = __halves2half2(vr[(k0 + 0) * D + n], vr[(k0 + 1) * D + n]);
-            const __half2 b1h = __halves2half2(vr[(k0 + 2) * D + n], vr[(k0 + 3) * D + n]);
-            mma16816(c16r, a, *reinterpret_cast<const uint32_t*>(&b0h), *reinterpret_cast<const uint32_t*>(&b1h));
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int rs = e >> 1;
-          o[t][e] = o[t][e] * al[rs] + w4[rs] * c4r[e] + w16[rs] * c16r[e];
-        }
-      }
-    }
-    // this warp is done with the stage (and with S, P of this block)
-    __syncwarp();
-    if (lane == 0) {
-      if (n4) mbar_arrive(&empty4[s4]);
-      if (n16) mbar_arrive(&empty16[s16]);
-    }
-    c4 += n4 ? 1 : 0;
-    c16 += n16 ? 1 : 0;
-  }
-
-  // ---- partial results of this split
-  if (ok) {
-    float* po = p.part_o + ((int64_t)grp * p.n_split + split) * kRowsMax * D;
-#pragma unroll
-    for (int t = 0; t < NT_PV; ++t) {
-      const int col = (warp + 8 * t) * 8 + 2 * tig;
-#pragma unroll
-      for (int rs = 0; rs < 2; ++rs) {
-        const int r = g + 8 * rs;
-        if (r < R) *reinterpret_cast<float2*>(po + r * D + col) = make_float2(o[t][2 * rs], o[t][2 * rs + 1]);
-      }
-    }
-    if (lane == 0) {
-      float* pml = p.part_ml + ((int64_t)grp * p.n_split + split) * kRowsMax * 2;
-#pragma unroll
-      for (int rs = 0; rs < 2; ++rs) {
-        const int r = warp + 8 * rs;
-        if (r < R) {
-          pml[2 * r] = m_run[rs];
-          pml[2 * r + 1] = l_run[rs];
-        }
-      }
+    po[idx] = acc;
+    if (idx % D == 0) {
+      pml[2 * r] = m;  // log2 units
+      pml[2 * r + 1] = l;
     }
   }
 }
 
-// Combine the splits of every row: O = sum_s w_s O_s / sum_s w_s l_s with w_s = exp(m_s - m).
-// One CTA per (batch, KV head); thread c handles output column c of every row.
-__global__ void decode_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
-                                      int n_split, int D, int R, int Hq, int Hkv, int Nq,
-                                      __half* __restrict__ out, float* __restrict__ lse) {
-  extern __shared__ float wsh[];  // [n_split] weights of the current row
-  __shared__ float s_m, s_l;
-  const int grp = blockIdx.x;
+// Combine the splits of every row: O = sum_s w_s O_s / sum_s w_s l_s with w_s = 2^(m_s - m)
+// (the partial maxima are in log2 units of the tau-scaled scores).  One CTA per (batch * KV head,
+// row); thread (part, c) sums output column c over the splits s = part (mod kCombineParts).
+constexpr int kCombineParts = 4;
+__global__ void __launch_bounds__(512) decode_combine_kernel(const float* __restrict__ part_o,
+                                                             const float* __restrict__ part_ml, int n_split, int D,
+                                                             int Hq, int Hkv, int Nq, __half* __restrict__ out,
+                                                             float* __restrict__ lse) {
+  extern __shared__ float wsh[];  // [n_split] weights, then [kCombineParts][D] column sums
+  __shared__ float red[16];
+  const int grp = blockIdx.x, r = blockIdx.y;
   const int b = grp / Hkv, hk = grp % Hkv, G = Hq / Hkv;
-  for (int r = 0; r < R; ++r) {
-    const float* ml = part_ml + (int64_t)grp * n_split * kRowsMax * 2 + 2 * r;
-    if (threadIdx.x == 0) {
-      float m = kNegInf;
-      for (int s = 0; s < n_split; ++s) m = fmaxf(m, ml[(int64_t)s * kRowsMax * 2]);
-      float l = 0.0f;
-      for (int s = 0; s < n_split; ++s) {
-        const float ms = ml[(int64_t)s * kRowsMax * 2];
-        const float w = (ms == kNegInf) ? 0.0f : expf(ms - m);
-        wsh[s] = w;
-        l += w * ml[(int64_t)s * kRowsMax * 2 + 1];
-      }
-      s_m = m;
-      s_l = l;
-    }
-    __syncthreads();
-    const int64_t orow = ((int64_t)b * Hq + (int64_t)hk * G + r / Nq) * Nq + r % Nq;
-    const float inv = s_l > 0.0f ? 1.0f / s_l : 0.0f;
-    for (int c = threadIdx.x; c < D; c += blockDim.x) {
-      float acc = 0.0f;
-      for (int s = 0; s < n_split; ++s)
-        acc += wsh[s] * part_o[(((int64_t)grp * n_split + s) * kRowsMax + r) * D + c];
-      out[orow * D + c] = __float2half_rn(acc * inv);
-    }
-    if (threadIdx.x == 0 && lse) lse[orow] = s_l > 0.0f ? s_m + logf(s_l) : kNegInf;
-    __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const float* ml = part_ml + (int64_t)grp * n_split * kRowsMax * 2 + 2 * r;
+  float m = kNegInf;
+  for (int s = threadIdx.x; s < n_split; s += blockDim.x) m = fmaxf(m, ml[(int64_t)s * kRowsMax * 2]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  m = red[0];
+  for (int i = 1; i < nw; ++i) m = fmaxf(m, red[i]);
+  __syncthreads();
+  float l = 0.0f;
+  for (int s = threadIdx.x; s < n_split; s += blockDim.x) {
+    const float ms = ml[(int64_t)s * kRowsMax * 2];
+    const float w = (ms == kNegInf) ? 0.0f : exp2f(ms - m);
+    wsh[s] = w;
+    l += w * ml[(int64_t)s * kRowsMax * 2 + 1];
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  if (lane == 0) red[warp] = l;
+  __syncthreads();
+  l = 0.0f;
+  for (int i = 0; i < nw; ++i) l += red[i];
+  const int64_t orow = ((int64_t)b * Hq + (int64_t)hk * G + r / Nq) * Nq + r % Nq;
+  const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+  const float* po = part_o + ((int64_t)grp * n_split * kRowsMax + r) * D;
+  float* colsum = wsh + n_split;
+  {
+    const int c = threadIdx.x % D, part = threadIdx.x / D;
+    float acc = 0.0f;
+#pragma unroll 4
+    for (int s = part; s < n_split; s += kCombineParts) acc = fmaf(wsh[s], po[(int64_t)s * kRowsMax * D + c], acc);
+    colsum[part * D + c] = acc;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int part = 0; part < kCombineParts; ++part) acc += colsum[part * D + c];
+    out[orow * D + c] = __float2half_rn(acc * inv);
+  }
+  if (threadIdx.x == 0 && lse) lse[orow] = l > 0.0f ? m * kLn2 + logf(l) : kNegInf;
 }
 
 // ------------------------------------------------------------------ host side
@@ -668,14 +740,21 @@ thrift_status decode_launch_t(const DecodeArgs& a, DecodeParams& prm, cudaStream
     if (!make_u8_map(&tm, a.part_o, 64, 1, 16, 1)) return THRIFT_ERR_CUDA;
   }
   auto kern = decode_attn_kernel<D, BK>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) != cudaSuccess)
-    return THRIFT_ERR_CUDA;
+  // once per device (a host-side attribute; keeping it out of later calls keeps them capturable)
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return THRIFT_ERR_CUDA;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) != cudaSuccess)
+      return THRIFT_ERR_CUDA;
+    attr_set[dev] = true;
+  }
   dim3 grid(prm.n_split, prm.B * prm.Hkv);
   kern<<<grid, kThreads, L::SMEM, stream>>>(tm, prm);
   if (cudaPeekAtLastError() != cudaSuccess) return THRIFT_ERR_CUDA;
-  decode_combine_kernel<<<prm.B * prm.Hkv, D, prm.n_split * sizeof(float), stream>>>(
-      prm.part_o, prm.part_ml, prm.n_split, D, prm.R, prm.Hq, prm.Hkv, prm.Nq, reinterpret_cast<__half*>(a.out),
-      a.lse);
+  decode_combine_kernel<<<dim3(prm.B * prm.Hkv, prm.R), D * kCombineParts,
+                          (prm.n_split + kCombineParts * D) * sizeof(float), stream>>>(
+      prm.part_o, prm.part_ml, prm.n_split, D, prm.Hq, prm.Hkv, prm.Nq, reinterpret_cast<__half*>(a.out), a.lse);
   return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 
@@ -687,7 +766,7 @@ int ctas_per_sm(int D, int BK) {
   if (D == 64 && BK == 128) smem = DLayout<64, 128>::SMEM;
   const int per_sm = 232448;  // shared memory of one SM, 1 KB of it reserved per CTA
   int n = per_sm / (smem + 1024);
-  return n < 1 ? 1 : (n > 4 ? 4 : n);
+  return n < 1 ? 1 : (n > 1 ? 1 : n);  // the kernel is built for one CTA per SM
 }
 
 }  // namespace
@@ -731,10 +810,10 @@ thrift_status decode_attn_launch(const DecodeArgs& a, cudaStream_t stream) {
   prm.mode = a.mode;
   prm.tau = c.softmax_scale > 0.0f ? c.softmax_scale : 1.0f / sqrtf((float)c.d);
   prm.wait_limit = kWaitLimit;
-  // splits: enough CTAs to fill every SM once, at least kMinBlocksPerSplit key blocks each
+  // splits: as many CTAs as fit on the GPU at once, at least kMinBlocksPerSplit key blocks each
   const int groups = c.B * c.Hkv;
   const int resident = num_sms() * ctas_per_sm(c.d, c.block_k);
-  int n_split = (resident + groups - 1) / groups;
+  int n_split = resident / groups;  // one wave: every CTA resident at once
   const int cap = decode_split_cap(prm.nkb);
   if (n_split > cap) n_split = cap;
   if (n_split < 1) n_split = 1;

@@ -163,7 +163,10 @@ thrift_status quantize_launch(const void* x, int64_t outer, int32_t N, int32_t d
   int64_t total = outer * (int64_t)N * d;
   if (cudaMemsetAsync(amax_slot, 0, sizeof(unsigned int), stream) != cudaSuccess) return THRIFT_ERR_CUDA;
   int sms = num_sms();
-  amax_kernel<<<sms * 8, 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), total / 8, amax_slot);
+  int64_t amax_blocks = (total / 8 + 4 * 256 - 1) / (4 * 256);  // about four vectors per thread
+  if (amax_blocks > (int64_t)sms * 8) amax_blocks = (int64_t)sms * 8;
+  if (amax_blocks < 1) amax_blocks = 1;
+  amax_kernel<<<(unsigned)amax_blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), total / 8, amax_slot);
   if (out->group_axis == 0) {
     int64_t groups = total / 16;
     int64_t blocks = (groups + 255) / 256;

@@ -87,7 +87,9 @@ __device__ __forceinline__ uint64_t score_key(double s) {
 }
 
 constexpr int kSelThreads = 1024;
+constexpr int kSelSmemKeys = 4096;
 
+template <int THREADS>
 __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int& total) {
   int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
@@ -99,7 +101,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int& total
   if (lane == 31) warp_sums[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int w = lane < (kSelThreads / 32) ? warp_sums[lane] : 0;
+    int w = lane < (THREADS / 32) ? warp_sums[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       int y = __shfl_up_sync(0xffffffffu, w, o);
@@ -109,13 +111,15 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int& total
   }
   __syncthreads();
   int before = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
-  total = warp_sums[kSelThreads / 32 - 1];
+  total = warp_sums[THREADS / 32 - 1];
   __syncthreads();
   return before;
 }
 
-// One CTA per (batch, query head).
-__global__ void __launch_bounds__(kSelThreads) topk_kernel(const double* __restrict__ scores, int64_t n,
+// One CTA per (batch, query head).  THREADS = kSelThreads for long rows; short rows (decode: one
+// query block) run with fewer threads, which makes the block-wide barriers of each pass cheaper.
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS) topk_kernel(const double* __restrict__ scores, int64_t n,
                                                            int nkb, int topk_abs, int topk_bp, int mask_words,
                                                            uint32_t* __restrict__ mask) {
   __shared__ unsigned int hist[256];
@@ -123,15 +127,21 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const double* __restr
   __shared__ unsigned long long s_prefix;
   __shared__ long long s_need;
   __shared__ unsigned long long s_nvalid;
+  __shared__ unsigned long long keys_sm[kSelSmemKeys];
   const double* sc = scores + (int64_t)blockIdx.x * n;
   int nqb = (int)(n / nkb);
   uint32_t* mk = mask + (int64_t)blockIdx.x * nqb * mask_words;
+  // rows of up to kSelSmemKeys scores are read from global memory once and kept in shared memory
+  const bool in_smem = n <= kSelSmemKeys;
+  if (in_smem)
+    for (int64_t t = threadIdx.x; t < n; t += THREADS) keys_sm[t] = score_key(sc[t]);
+  auto key_at = [&](int64_t t) -> uint64_t { return in_smem ? keys_sm[t] : score_key(sc[t]); };
 
   // count valid pairs
   if (threadIdx.x == 0) s_nvalid = 0;
   __syncthreads();
   unsigned long long cnt = 0;
-  for (int64_t t = threadIdx.x; t < n; t += kSelThreads) cnt += score_key(sc[t]) != 0ull;
+  for (int64_t t = threadIdx.x; t < n; t += THREADS) cnt += key_at(t) != 0ull;
   atomicAdd(&s_nvalid, cnt);
   __syncthreads();
   long long nvalid = (long long)s_nvalid;
@@ -143,23 +153,45 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const double* __restr
   unsigned long long prefix = 0ull;
   long long need = k;  // rank (1-based) of the wanted key among keys matching the prefix
   for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int b = threadIdx.x; b < 256; b += kSelThreads) hist[b] = 0;
+    for (int b = threadIdx.x; b < 256; b += THREADS) hist[b] = 0;
     __syncthreads();
     unsigned long long hi_mask = shift == 56 ? 0ull : (~0ull << (shift + 8));
-    for (int64_t t = threadIdx.x; t < n; t += kSelThreads) {
-      uint64_t key = score_key(sc[t]);
-      if (key != 0ull && (key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1u);
+    // scores of one head share their leading bits, so most keys fall in the same few bins: one
+    // shared-memory atomic per distinct bin of a warp instead of one per key
+    for (int64_t base = 0; base < n; base += THREADS) {
+      const int64_t t = base + threadIdx.x;
+      const uint64_t key = t < n ? key_at(t) : 0ull;
+      const bool in = key != 0ull && (key & hi_mask) == prefix;
+      const int bin = in ? (int)((key >> shift) & 255) : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (unsigned)__popc(peers));
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      long long acc = 0;
-      int b = 255;
-      for (; b >= 0; --b) {
-        if (acc + (long long)hist[b] >= need) break;
-        acc += hist[b];
+    if (threadIdx.x < 32) {
+      // bins from the top: lane l holds bins 255 - 8l .. 248 - 8l; find the bin where the
+      // count of keys at or above it first reaches `need`
+      const int lane = threadIdx.x;
+      long long mine = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mine += hist[255 - 8 * lane - i];
+      long long incl = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
-      s_prefix = prefix | ((unsigned long long)b << shift);
-      s_need = need - acc;
+      const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
+      const int L = __ffs(hit) - 1;  // need <= total count, so some lane hits
+      if (lane == L) {
+        long long acc = incl - mine;
+        int b = 255 - 8 * lane;
+        for (int i = 0; i < 7; ++i, --b) {
+          if (acc + (long long)hist[b] >= need) break;
+          acc += hist[b];
+        }
+        s_prefix = prefix | ((unsigned long long)b << shift);
+        s_need = need - acc;
+      }
     }
     __syncthreads();
     prefix = s_prefix;
@@ -168,12 +200,12 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const double* __restr
   }
   // prefix is now the k-th largest key; take every key above it and the first `need` ties.
   long long taken_ties = 0;
-  for (int64_t base = 0; base < n; base += kSelThreads) {
+  for (int64_t base = 0; base < n; base += THREADS) {
     int64_t t = base + threadIdx.x;
-    uint64_t key = t < n ? score_key(sc[t]) : 0ull;
+    uint64_t key = t < n ? key_at(t) : 0ull;
     int tie = (key != 0ull && key == prefix) ? 1 : 0;
     int total;
-    int before = block_excl_scan(tie, warp_sums, total);
+    int before = block_excl_scan<THREADS>(tie, warp_sums, total);
     bool take = (key > prefix) || (tie && (taken_ties + before) < need);
     if (take) {
       int i = (int)(t / nkb), j = (int)(t % nkb);
@@ -183,23 +215,75 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const double* __restr
   }
 }
 
-__global__ void lists_kernel(const uint32_t* __restrict__ mask, int64_t rows, int nkb, int mask_words,
-                             int32_t* __restrict__ counts, int16_t* __restrict__ lists) {
-  int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (r >= rows) return;
+constexpr int kListThreads = 256;
+
+// Sorted list of the set bits of one mask row: one CTA per row, thread t owns a contiguous run of
+// mask words; a block scan of the per-thread counts gives each thread its output offset.
+__global__ void __launch_bounds__(kListThreads) lists_kernel(const uint32_t* __restrict__ mask, int64_t rows,
+                                                             int nkb, int mask_words, int32_t* __restrict__ counts,
+                                                             int16_t* __restrict__ lists) {
+  __shared__ int warp_tot[kListThreads / 32];
+  const int64_t r = blockIdx.x;
   const uint32_t* mw = mask + r * mask_words;
   int16_t* out = lists + r * nkb;
-  int c = 0;
-  for (int w = 0; w < mask_words; ++w) {
+  const int wpt = (mask_words + kListThreads - 1) / kListThreads;
+  const int w0 = min(mask_words, (int)threadIdx.x * wpt), w1 = min(mask_words, w0 + wpt);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(mw[w]);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  int c = x - cnt, total = 0;
+#pragma unroll
+  for (int i = 0; i < kListThreads / 32; ++i) {
+    const int t = warp_tot[i];
+    if (i < warp) c += t;
+    total += t;
+  }
+  for (int w = w0; w < w1; ++w) {
     uint32_t bits = mw[w];
     while (bits) {
-      int b = __ffs(bits) - 1;
+      const int b = __ffs(bits) - 1;
       bits &= bits - 1;
       out[c++] = (int16_t)(w * 32 + b);
     }
   }
-  counts[r] = c;
-  for (int t = c; t < nkb; ++t) out[t] = -1;
+  for (int t = total + threadIdx.x; t < nkb; t += kListThreads) out[t] = -1;
+  if (threadIdx.x == 0) counts[r] = total;
+}
+
+// Decode scores S^[b, h, j] = qbar[b, h] . kbar[b, h / G, j]: a CTA stages kDecScoreBlocks key-block
+// means of one KV head in shared memory; thread (hl, jj) scores block jj for query head hk*G + hl,
+// the sum in the order c = 0 .. d-1 with no fused multiply-add (the evaluation the prefill scores
+// use).
+constexpr int kDecScoreBlocks = 16;
+__global__ void decode_score_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar, int Hq,
+                                    int Hkv, int nkb, int d, double* __restrict__ scores) {
+  __shared__ double ks[kDecScoreBlocks * 129];
+  __shared__ double qs[16 * 128];
+  const int G = Hq / Hkv, grp = blockIdx.y;
+  const int b = grp / Hkv, hk = grp % Hkv;
+  const int j0 = blockIdx.x * kDecScoreBlocks;
+  const int nb = min(kDecScoreBlocks, nkb - j0);
+  const double* kb = kbar + ((int64_t)grp * nkb + j0) * d;
+  for (int e = threadIdx.x; e < nb * d; e += blockDim.x) ks[(e / d) * (d + 1) + e % d] = kb[e];
+  const double* qb = qbar + ((int64_t)b * Hq + (int64_t)hk * G) * d;
+  for (int e = threadIdx.x; e < G * d; e += blockDim.x) qs[e] = qb[e];
+  __syncthreads();
+  const int jj = threadIdx.x % kDecScoreBlocks, hl = threadIdx.x / kDecScoreBlocks;
+  if (jj >= nb || hl >= G) return;
+  const double* qr = qs + hl * d;
+  const double* kr = ks + jj * (d + 1);
+  double acc = 0.0;
+#pragma unroll 8
+  for (int c = 0; c < d; ++c) acc = __dadd_rn(acc, __dmul_rn(qr[c], kr[c]));
+  scores[((int64_t)b * Hq + (int64_t)hk * G + hl) * nkb + j0 + jj] = acc;
 }
 
 }  // namespace
@@ -253,10 +337,10 @@ thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, u
                                                            c.block_k, c.causal, scores);
   size_t mask_bytes = (size_t)c.B * c.Hq * nqb * mask_words * sizeof(uint32_t);
   if (cudaMemsetAsync(mask, 0, mask_bytes, stream) != cudaSuccess) return THRIFT_ERR_CUDA;
-  topk_kernel<<<c.B * c.Hq, kSelThreads, 0, stream>>>(scores, (int64_t)nqb * nkb, nkb, c.topk_abs, c.topk_bp,
-                                                      mask_words, mask);
+  topk_kernel<kSelThreads><<<c.B * c.Hq, kSelThreads, 0, stream>>>(scores, (int64_t)nqb * nkb, nkb, c.topk_abs,
+                                                                    c.topk_bp, mask_words, mask);
   int64_t rows = (int64_t)c.B * c.Hq * nqb;
-  lists_kernel<<<(unsigned)((rows + 127) / 128), 128, 0, stream>>>(mask, rows, nkb, mask_words, counts, lists);
+  lists_kernel<<<(unsigned)rows, kListThreads, 0, stream>>>(mask, rows, nkb, mask_words, counts, lists);
   return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 
@@ -287,15 +371,17 @@ thrift_status decode_select_launch(const void* q, const double* kbar, const thri
   int tpb = c.d >= 128 ? 128 : c.d;
   block_mean_kernel<<<dim3(1, (unsigned)heads), tpb, 0, stream>>>(reinterpret_cast<const __half*>(q), c.Nq, c.d,
                                                                   c.Nq, qbar);
-  size_t smem = (size_t)(kTileQ + kTileK) * (c.d + 1) * sizeof(double);
-  dim3 g((nkb + kTileK - 1) / kTileK, 1, (unsigned)heads);
-  block_score_kernel<<<g, kTileQ * kTileK, smem, stream>>>(qbar, kbar, c.Hq, c.Hkv, 1, nkb, c.d, c.Nq, c.block_k, 0,
-                                                           scores);
+  dim3 g((nkb + kDecScoreBlocks - 1) / kDecScoreBlocks, (unsigned)(c.B * c.Hkv));
+  decode_score_kernel<<<g, kDecScoreBlocks * (c.Hq / c.Hkv), 0, stream>>>(qbar, kbar, c.Hq, c.Hkv, nkb, c.d,
+                                                                          scores);
   if (cudaMemsetAsync(mask, 0, heads * mask_words * sizeof(uint32_t), stream) != cudaSuccess) return THRIFT_ERR_CUDA;
-  topk_kernel<<<(unsigned)heads, kSelThreads, 0, stream>>>(scores, (int64_t)nkb, nkb, c.topk_abs, c.topk_bp,
-                                                           mask_words, mask);
-  lists_kernel<<<(unsigned)((heads + 127) / 128), 128, 0, stream>>>(mask, (int64_t)heads, nkb, mask_words, counts,
-                                                                    lists);
+  if (nkb <= kSelSmemKeys)
+    topk_kernel<256><<<(unsigned)heads, 256, 0, stream>>>(scores, (int64_t)nkb, nkb, c.topk_abs, c.topk_bp,
+                                                          mask_words, mask);
+  else
+    topk_kernel<kSelThreads><<<(unsigned)heads, kSelThreads, 0, stream>>>(scores, (int64_t)nkb, nkb, c.topk_abs,
+                                                                          c.topk_bp, mask_words, mask);
+  lists_kernel<<<(unsigned)heads, kListThreads, 0, stream>>>(mask, (int64_t)heads, nkb, mask_words, counts, lists);
   return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 
