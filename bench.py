@@ -8,6 +8,10 @@ the attention kernel's fraction of the blended NVFP4/FP16 tensor-core roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
+With --workload decode131k (or another decode workload) it times one decode step instead: the new
+query rows against a 131K-key cache held in FP16 and NVFP4 (selection + attention), reported as
+the step's algorithmic cache bytes per second against the measured HBM bandwidth.
+
 One process per GPU (torchrun for N > 1); each rank runs its own copy of the workload (weak
 scaling, no collective on the data path); timing is CUDA events on the launching stream, max over
 ranks.  Rank 0 prints one JSON line.
@@ -33,6 +37,7 @@ if ROOT not in sys.path:
 import workloads  # noqa: E402
 
 METRIC = "attn fwd effective TFLOPS & % of NVFP4/FP16 tensor roofline, N=32K causal k=5%"
+DECODE_METRIC = "decode step: algorithmic KV-cache GB/s (NVFP4 + selected FP16 blocks) & % of HBM roofline"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_traffic.json")
 ATTN_SRC = os.path.join(ROOT, "precision_attention_block_b200", "csrc", "attn.cu")
@@ -203,6 +208,9 @@ def run_reference(args, rank):
         w = w.with_budget(args.budget_bp)
     q, k, v = workloads.make_qkv(w)
     threads = os.cpu_count() or 1
+    if w.is_decode:
+        run_reference_decode(args, w, q, k, v, threads)
+        return
     t0 = time.perf_counter()
     q4, k4, v4 = oracle.quantize_all(q, k, v)
     scores = oracle.block_scores(q, k, w)
@@ -231,6 +239,34 @@ def run_reference(args, rank):
                              "sample": f"{per_step} (b, head, query block) units per step, cycled from a "
                                        f"stratified sample, plus their share of the full quantise/select"},
             "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_decode(args, w, q, k, v, threads):
+    """--impl reference on a decode workload: whole oracle decode steps (the cache's NVFP4 copies
+    built once beforehand), the same bytes-per-second metric as the GPU line."""
+    import oracle
+    k4, v4 = oracle.quantize_nvfp4(k, 0), oracle.quantize_nvfp4(v, 1)
+    r = oracle.decode_forward(w, q, k, v, k4=k4, v4=v4, threads=threads)
+    alg_bytes, _, _ = decode_bytes(w, r["sel"][:, :, 0, :].astype(bool))
+    steps = max(1, min(args.steps, 10))
+    secs = 0.0
+    for s in range(min(args.warmup, 1) + steps):
+        t0 = time.perf_counter()
+        oracle.decode_forward(w, q, k, v, k4=k4, v4=v4, threads=threads)
+        if s >= min(args.warmup, 1):
+            secs += time.perf_counter() - t0
+    value = alg_bytes * steps / secs / 1e9
+    line = {"impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": min(args.warmup, 1), "ms_per_step": 1e3 * secs / steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.n_query, "Nk": w.N,
+                       "d": w.d, "causal": w.causal, "block_k": w.block_k, "topk_bp": w.topk_bp},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{steps} whole decode steps (quantise the query rows, score, select, "
+                                       f"attend); cache NVFP4 copies built once beforehand"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
@@ -268,6 +304,9 @@ def main():
     w = workloads.WORKLOADS[args.workload]
     if args.budget_bp is not None:
         w = w.with_budget(args.budget_bp)
+    if w.is_decode:
+        main_decode(args, w, pab, torch, device, world, rank, local_rank, dist)
+        return
     cfg = pab.Config.from_workload(w)
     q, k, v = workloads.make_qkv(w)
     gq, gk, gv = (torch.from_numpy(x).to(device) for x in (q, k, v))
@@ -368,6 +407,137 @@ def main():
         line["e2e"] = e2e_measure(pab, torch, w, cfg, q, k, v, device, args, world, dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, q, k, v, args.cpu_units)
+    line["clocks"] = sampler.summary()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+def decode_bytes(w, mask_bits):
+    """Algorithmic HBM bytes of one decode step for a selection: per (batch, KV head, key block)
+    the NVFP4 K and V (codes and E4M3 scales) when some query head of the group computes the block
+    in NVFP4, the FP16 K and V when some head selected it, plus the key-block means the selection
+    reads.  mask_bits: bool [B, Hq, nKb]."""
+    G = w.Hq // w.Hkv
+    g = mask_bits.reshape(w.B, w.Hkv, G, -1)
+    blocks16 = int(g.any(2).sum())
+    blocks4 = int((~g).any(2).sum())
+    per4 = 2 * w.block_k * w.d * (1 / 2 + 1 / 16)
+    per16 = 2 * w.block_k * w.d * 2
+    kbar = w.B * w.Hkv * (w.N // w.block_k) * w.d * 8
+    return blocks4 * per4 + blocks16 * per16 + kbar, blocks4, blocks16
+
+
+def main_decode(args, w, pab, torch, device, world, rank, local_rank, dist):
+    """One decode step per iteration: quantise the query rows, select key blocks, attend.  The
+    cache (FP16, NVFP4 copies, key block means) is built once and stays resident.  Steps are
+    replayed from a CUDA graph of one step (the launches of a step take less GPU time than the
+    host needs to issue them one by one)."""
+    cfg = pab.DecodeConfig.from_workload(w)
+    q, k, v = workloads.make_qkv(w)
+    gq, gk, gv = (torch.from_numpy(x).to(device) for x in (q, k, v))
+    cache = pab.KVCache.build(gk, gv, w.block_k)
+    ws = cfg.workspace(device)
+    out = torch.empty_like(gq)
+    lse = torch.empty((w.B, w.Hq, w.n_query), dtype=torch.float32, device=device)
+    sel = pab.decode_select(gq, cache, cfg, ws=ws)
+    torch.cuda.synchronize()
+    mask = sel.mask.cpu().numpy().view(np.uint32)
+    bits = ((mask[..., :, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(w.B, w.Hq, -1)[..., :cfg.n_kb]
+    alg_bytes, blocks4, blocks16 = decode_bytes(w, bits.astype(bool))
+    cache_mb = (gk.numel() + gv.numel()) * 2 / 1e6
+
+    side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream())
+
+    def graph_of(fn):
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            fn()
+        return g
+
+    step_graph = graph_of(lambda: pab.decode_fwd(gq, cache, cfg, out=out, lse=lse, ws=ws))
+    attn_graph = graph_of(lambda: pab.decode_attn(gq, cache, sel, cfg, out=out, lse=lse, ws=ws))
+    cfg16 = pab.DecodeConfig.from_workload(w.with_budget(10000))
+    ws16 = cfg16.workspace(device)
+    fp16_graph = graph_of(lambda: pab.decode_attn(gq, cache, None, cfg16, out=out, lse=lse, ws=ws16))
+
+    def timed(g, steps, warmup):
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        t = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=device)
+        if dist:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t[0]) / steps
+
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        step_ms = timed(step_graph, args.steps, args.warmup)
+    attn_ms = timed(attn_graph, args.steps, args.warmup)
+    fp16_ms = timed(fp16_graph, max(3, args.steps // 4), 2)
+    status = pab.device_status(ws)
+    _, _, hbm_gbs, peak_src = peaks()
+    attn_bytes = alg_bytes - w.B * w.Hkv * (w.N // w.block_k) * w.d * 8
+    achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
+    value = world * alg_bytes / (step_ms * 1e-3) / 1e9
+    line = {"metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4+fp16 (fp32 accumulate)", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.n_query, "Nk": w.N,
+                       "d": w.d, "causal": w.causal, "block_k": w.block_k, "topk_bp": w.topk_bp,
+                       "parallelism": f"replica x{world} (each rank its own batch)",
+                       "l2": f"cache larger than L2 (K, V {cache_mb:.0f} MB FP16 + NVFP4 copies)"
+                             if cache_mb > 126 else f"cache {cache_mb:.0f} MB: L2 not flushed"},
+            "breakdown_us": {"step": 1e3 * step_ms, "attention": 1e3 * attn_ms,
+                             "select_and_quantize": 1e3 * (step_ms - attn_ms),
+                             "all_fp16_attention_same_kernel": 1e3 * fp16_ms},
+            "blocks": {"nvfp4": blocks4, "fp16": blocks16, "of": w.B * w.Hkv * (w.N // w.block_k)},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": achieved / hbm_gbs, "traffic": None,
+                         "peak_note": f"{peak_src} HBM copy bandwidth; achieved = the attention kernels' "
+                                      f"algorithmic bytes ({attn_bytes / 1e6:.1f} MB) / their time"},
+            "gpu_launches": 8 * args.steps,
+            "device_status": status}
+    if not args.no_e2e:
+        hq = torch.from_numpy(q).pin_memory()
+        ho = torch.empty(out.shape, dtype=torch.float16).pin_memory()
+        hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            gq.copy_(hq, non_blocking=True)
+            pab.decode_fwd(gq, cache, cfg, out=out, lse=lse, ws=ws)
+            ho.copy_(out, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        e2e_ms = timed(graph_of(e2e_step), args.steps, args.warmup)
+        line["e2e"] = {"value": world * alg_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                       "h2d_bytes_per_step": int(hq.numel() * 2),
+                       "d2h_bytes_per_step": int(ho.numel() * 2 + hl.numel() * 4), "ms_per_step": e2e_ms,
+                       "note": "query rows copied in and the output copied out every step; the cache stays "
+                               "resident, as in a decode loop"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        threads = os.cpu_count() or 1
+        k4o, v4o = oracle.quantize_nvfp4(k, 0), oracle.quantize_nvfp4(v, 1)
+        t0 = time.perf_counter()
+        oracle.decode_forward(w, q, k, v, k4=k4o, v4=v4o, threads=threads)
+        t = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": alg_bytes / t / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                "sample": f"one whole decode step of {w.name} ({t:.2f} s on {threads} threads); "
+                                          "cache NVFP4 copies built beforehand, outside the timing"}
     line["clocks"] = sampler.summary()
     if rank == 0:
         print(json.dumps(line), flush=True)

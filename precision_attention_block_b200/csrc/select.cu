@@ -156,15 +156,23 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const double* __restrict_
     for (int b = threadIdx.x; b < 256; b += THREADS) hist[b] = 0;
     __syncthreads();
     unsigned long long hi_mask = shift == 56 ? 0ull : (~0ull << (shift + 8));
-    // scores of one head share their leading bits, so most keys fall in the same few bins: one
-    // shared-memory atomic per distinct bin of a warp instead of one per key
-    for (int64_t base = 0; base < n; base += THREADS) {
-      const int64_t t = base + threadIdx.x;
-      const uint64_t key = t < n ? key_at(t) : 0ull;
-      const bool in = key != 0ull && (key & hi_mask) == prefix;
-      const int bin = in ? (int)((key >> shift) & 255) : -1;
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (unsigned)__popc(peers));
+    if (shift >= 48) {
+      // the leading bytes (sign, exponent, top of the mantissa) are shared by most scores of a
+      // head, so most keys fall in the same few bins: one shared-memory atomic per distinct bin of
+      // a warp instead of one per key
+      for (int64_t base = 0; base < n; base += THREADS) {
+        const int64_t t = base + threadIdx.x;
+        const uint64_t key = t < n ? key_at(t) : 0ull;
+        const bool in = key != 0ull && (key & hi_mask) == prefix;
+        const int bin = in ? (int)((key >> shift) & 255) : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (unsigned)__popc(peers));
+      }
+    } else {
+      for (int64_t t = threadIdx.x; t < n; t += THREADS) {
+        const uint64_t key = key_at(t);
+        if (key != 0ull && (key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1u);
+      }
     }
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -215,37 +223,31 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const double* __restrict_
   }
 }
 
-constexpr int kListThreads = 256;
+constexpr int kListRowsPerCta = 8;
 
-// Sorted list of the set bits of one mask row: one CTA per row, thread t owns a contiguous run of
-// mask words; a block scan of the per-thread counts gives each thread its output offset.
-__global__ void __launch_bounds__(kListThreads) lists_kernel(const uint32_t* __restrict__ mask, int64_t rows,
-                                                             int nkb, int mask_words, int32_t* __restrict__ counts,
-                                                             int16_t* __restrict__ lists) {
-  __shared__ int warp_tot[kListThreads / 32];
-  const int64_t r = blockIdx.x;
+// Sorted list of the set bits of each mask row: one warp per row, lane l owns a contiguous run of
+// the row's mask words; a warp scan of the per-lane counts gives each lane its output offset.
+__global__ void __launch_bounds__(32 * kListRowsPerCta) lists_kernel(const uint32_t* __restrict__ mask, int64_t rows,
+                                                                      int nkb, int mask_words,
+                                                                      int32_t* __restrict__ counts,
+                                                                      int16_t* __restrict__ lists) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * kListRowsPerCta + (threadIdx.x >> 5);
+  if (r >= rows) return;
   const uint32_t* mw = mask + r * mask_words;
   int16_t* out = lists + r * nkb;
-  const int wpt = (mask_words + kListThreads - 1) / kListThreads;
-  const int w0 = min(mask_words, (int)threadIdx.x * wpt), w1 = min(mask_words, w0 + wpt);
+  const int wpl = (mask_words + 31) / 32;
+  const int w0 = min(mask_words, lane * wpl), w1 = min(mask_words, w0 + wpl);
   int cnt = 0;
   for (int w = w0; w < w1; ++w) cnt += __popc(mw[w]);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = cnt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) warp_tot[warp] = x;
-  __syncthreads();
-  int c = x - cnt, total = 0;
-#pragma unroll
-  for (int i = 0; i < kListThreads / 32; ++i) {
-    const int t = warp_tot[i];
-    if (i < warp) c += t;
-    total += t;
-  }
+  const int total = __shfl_sync(0xffffffffu, x, 31);
+  int c = x - cnt;
   for (int w = w0; w < w1; ++w) {
     uint32_t bits = mw[w];
     while (bits) {
@@ -254,8 +256,8 @@ __global__ void __launch_bounds__(kListThreads) lists_kernel(const uint32_t* __r
       out[c++] = (int16_t)(w * 32 + b);
     }
   }
-  for (int t = total + threadIdx.x; t < nkb; t += kListThreads) out[t] = -1;
-  if (threadIdx.x == 0) counts[r] = total;
+  for (int t = total + lane; t < nkb; t += 32) out[t] = -1;
+  if (lane == 0) counts[r] = total;
 }
 
 // Decode scores S^[b, h, j] = qbar[b, h] . kbar[b, h / G, j]: a CTA stages kDecScoreBlocks key-block
@@ -340,7 +342,8 @@ thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, u
   topk_kernel<kSelThreads><<<c.B * c.Hq, kSelThreads, 0, stream>>>(scores, (int64_t)nqb * nkb, nkb, c.topk_abs,
                                                                     c.topk_bp, mask_words, mask);
   int64_t rows = (int64_t)c.B * c.Hq * nqb;
-  lists_kernel<<<(unsigned)rows, kListThreads, 0, stream>>>(mask, rows, nkb, mask_words, counts, lists);
+  lists_kernel<<<(unsigned)((rows + kListRowsPerCta - 1) / kListRowsPerCta), 32 * kListRowsPerCta, 0, stream>>>(
+      mask, rows, nkb, mask_words, counts, lists);
   return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 
@@ -381,7 +384,8 @@ thrift_status decode_select_launch(const void* q, const double* kbar, const thri
   else
     topk_kernel<kSelThreads><<<(unsigned)heads, kSelThreads, 0, stream>>>(scores, (int64_t)nkb, nkb, c.topk_abs,
                                                                           c.topk_bp, mask_words, mask);
-  lists_kernel<<<(unsigned)heads, kListThreads, 0, stream>>>(mask, (int64_t)heads, nkb, mask_words, counts, lists);
+  lists_kernel<<<(unsigned)((heads + kListRowsPerCta - 1) / kListRowsPerCta), 32 * kListRowsPerCta, 0, stream>>>(
+      mask, (int64_t)heads, nkb, mask_words, counts, lists);
   return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 
