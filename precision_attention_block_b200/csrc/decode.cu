@@ -98,7 +98,7 @@ struct DLayout {
   static constexpr int PA_BYTES = kConsumerWarps * (BK / 16) * 32 * 16;
   static constexpr int OFF_TAB = OFF_PA + PA_BYTES;             // FP16-head bits of the split's blocks
   static constexpr int OFF_BAR = OFF_TAB + kTab * 2;
-  static constexpr int BAR_BYTES = 8 * (2 * NST + 2 * NF) + 4 * (NST + NF) + 16;
+  static constexpr int BAR_BYTES = 8 * (2 * NST + 2 * NF) + 4 * (NST + NF) + 16;  // + abort flag, next block
   static constexpr int SMEM = OFF_BAR + BAR_BYTES;
   // after the main loop the consumer warps' partial results reuse the stage area
   static constexpr int COMB_ML = kConsumerWarps * kRowsMax * D * 4;  // after [warps][16][D] f32 outputs
@@ -235,6 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_kernel(const __grid_c
   volatile int* tag4 = reinterpret_cast<volatile int*>(empty16 + NF);
   volatile int* tag16 = tag4 + NST;
   volatile int* abort_flag = tag16 + NF;
+  int* next_block = const_cast<int*>(abort_flag) + 1;  // the next block a consumer warp takes
   uint16_t* tab = reinterpret_cast<uint16_t*>(smem + L::OFF_TAB);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -257,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_kernel(const __grid_c
       tag16[s] = -1;
     }
     *abort_flag = 0;
+    *next_block = 0;
     fence_mbar_init();
   }
   {
@@ -342,8 +344,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_kernel(const __grid_c
   }
 
   // ------------------------------------------------------------------ consumers
-  // Warp w takes the split's blocks w, w + 7, ...; each warp keeps its own output, maximum and
-  // denominator for rows g and g + 8, combined with the other warps' at the end.
+  // Each consumer warp takes the split's next unclaimed block (in block order) until none is left,
+  // and keeps its own output, maximum and denominator for rows g and g + 8, combined with the
+  // other warps' at the end.
   const int g = lane >> 2, tig = lane & 3;
   const int R = p.R;
   const float sv4 = use4 ? __ldg(p.v_ts) * (1.0f / 2688.0f) : 0.0f;
@@ -367,7 +370,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_kernel(const __grid_c
 
   int scan_i = 0, c16_acc = 0;
   bool ok = true;
-  for (int i = warp; i < nblk; i += kConsumerWarps) {
+  for (;;) {
+    int i = 0;
+    if (lane == 0) i = atomicAdd(next_block, 1);
+    i = __shfl_sync(0xffffffffu, i, 0);
+    if (i >= nblk) break;
     while (scan_i < i) c16_acc += bits_of(scan_i++) != 0u ? 1 : 0;
     const int j = j0 + i;
     const uint32_t bits = bits_of(i);
