@@ -82,7 +82,7 @@ def lib():
              ctypes.c_void_p, _u16p, _f32p, ctypes.c_void_p, _int])
         L.orc_attn_qk.argtypes = (
             [_u16p, _u16p, _u16p, _u8p, _u8p, ctypes.c_float, _u8p, _u8p, ctypes.c_float,
-             _u8p, _u8p, ctypes.c_float, _u8p] + [_int] * 9 + [ctypes.c_float, _i32p, _int, _int,
+             _u8p, _u8p, ctypes.c_float, _u8p] + [_int] * 9 + [ctypes.c_float, _int, _i32p, _int, _int,
              ctypes.c_void_p, _u16p, _f32p, ctypes.c_void_p, _int])
         L.orc_tile_scores.argtypes = (
             [_u16p, _u16p, _u8p, _u8p, ctypes.c_float, _u8p, _u8p, ctypes.c_float] + [_int] * 8
@@ -268,6 +268,31 @@ def attn(q, k, v, q4: NVFP4, k4: NVFP4, v4: NVFP4, sel, w, tau=None, units=None,
     return out.view(np.float16), lse, out64
 
 
+def attn_sparse(q, k, v, sel, w, tau=None, units=None, want_f64=False, threads=None):
+    """Compute-matched sparse variant (reading R-sparse): only the selected pairs, in FP16; every
+    other pair dropped.  A row left with no key gets output 0 and lse -inf.  Same return values as
+    `attn`; no NVFP4 tensor is used."""
+    B, Hq, N, d = q.shape
+    if tau is None:
+        tau = softmax_scale(d)
+    if units is None:
+        units = [(b, h, i) for b in range(B) for h in range(Hq) for i in range(N // w.block_q)]
+    u = np.ascontiguousarray(np.array(units, np.int32).reshape(-1))
+    out = np.zeros((B, Hq, N, d), np.uint16)
+    lse = np.zeros((B, Hq, N), np.float32)
+    out64 = np.zeros((B, Hq, N, d), np.float64) if want_f64 else None
+    if threads is None:
+        threads = os.cpu_count() or 1
+    z8 = np.zeros(1, np.uint8)
+    lib().orc_attn_qk(_u16(q).reshape(-1), _u16(k).reshape(-1), _u16(v).reshape(-1),
+                      z8, z8, np.float32(1), z8, z8, np.float32(1), z8, z8, np.float32(1),
+                      np.ascontiguousarray(sel, np.uint8).reshape(-1),
+                      B, Hq, k.shape[1], N, N, d, w.block_q, w.block_k, int(w.causal), np.float32(tau), 1,
+                      u, len(units), 0, None, out.reshape(-1), lse.reshape(-1),
+                      None if out64 is None else out64.ctypes.data, int(threads))
+    return out.view(np.float16), lse, out64
+
+
 def quantize_all(q, k, v):
     """The three NVFP4 tensors of one problem: Q, K grouped along d; V grouped along tokens."""
     return quantize_nvfp4(q, 0), quantize_nvfp4(k, 0), quantize_nvfp4(v, 1)
@@ -299,11 +324,11 @@ def decode_block_scores(q: np.ndarray, k: np.ndarray, block_k: int, causal: bool
 
 
 def decode_attn(q, k, v, q4: NVFP4, k4: NVFP4, v4: NVFP4, sel, block_k: int, causal: bool, tau=None,
-                want_f64=False, threads=None):
+                want_f64=False, threads=None, sparse=False):
     """Decode attention (reading R-decode): the Nq rows of q [B,Hq,Nq,d] are the newest
     positions of the cache k, v [B,Hkv,Nk,d]; sel [B,Hq,1,Nk/block_k] marks the FP16 key blocks.
-    The same mixed-precision computation as `attn`.  Returns (out fp16 [B,Hq,Nq,d],
-    lse f32 [B,Hq,Nq], out64 or None)."""
+    The same mixed-precision computation as `attn` (sparse: only the selected blocks, reading
+    R-sparse).  Returns (out fp16 [B,Hq,Nq,d], lse f32 [B,Hq,Nq], out64 or None)."""
     B, Hq, Nq, d = q.shape
     Hkv, Nk = k.shape[1], k.shape[2]
     if tau is None:
@@ -320,7 +345,7 @@ def decode_attn(q, k, v, q4: NVFP4, k4: NVFP4, v4: NVFP4, sel, block_k: int, cau
                       k4.codes.reshape(-1), k4.scales.reshape(-1), k4.tensor_scale,
                       v4.codes.reshape(-1), v4.scales.reshape(-1), v4.tensor_scale,
                       np.ascontiguousarray(sel, np.uint8).reshape(-1),
-                      B, Hq, Hkv, Nq, Nk, d, Nq, block_k, int(causal), np.float32(tau),
+                      B, Hq, Hkv, Nq, Nk, d, Nq, block_k, int(causal), np.float32(tau), int(sparse),
                       u, len(units), 0, None, out.reshape(-1), lse.reshape(-1),
                       None if out64 is None else out64.ctypes.data, int(threads))
     return out.view(np.float16), lse, out64

@@ -45,6 +45,9 @@
  *            blocks with qbar the mean of the Nq rows; the query rows are
  *            quantised as their own tensor (their own FP32 tensor scale).
  *            Prefill is the case Nq = Nk.
+ *   R-sparse the compute-matched sparse variant keeps only the selected
+ *            pairs (in FP16) and drops every other pair, as if masked; a row
+ *            left with no key has output 0 and lse -inf.
  */
 #include <math.h>
 #include <pthread.h>
@@ -305,6 +308,7 @@ typedef struct {
   const uint8_t* sel;
   int B, Hq, Hkv, Nq, Nk, d, bq, bk, causal;
   double tau;
+  int sparse; /* 1: only the selected (FP16) pairs, the others dropped (R-sparse) */
 } attn_problem;
 
 /* position of query row 0 among the keys (bottom-right causal alignment) */
@@ -415,7 +419,7 @@ static void attn_unit(const attn_problem* P, int b, int h, int i, int online, co
   for (int r = 0; r < bq; ++r) m[r] = -INFINITY;
 
   for (int j = 0; j < nkb; ++j) {
-    if (!pair_valid(P->causal, qoff, i, j, bq, bk)) {
+    if (!pair_valid(P->causal, qoff, i, j, bq, bk) || (P->sparse && !pair_is_fp16(P, b, h, i, j))) {
       for (int r = 0; r < bq; ++r)
         for (int t = 0; t < bk; ++t) S[r * ldS + (int64_t)j * bk + t] = -INFINITY;
       continue;
@@ -429,6 +433,7 @@ static void attn_unit(const attn_problem* P, int b, int h, int i, int online, co
   for (int jj = 0; jj < nkb; ++jj) {
     int j = order ? order[jj] : jj;
     if (!pair_valid(P->causal, qoff, i, j, bq, bk)) continue;
+    if (P->sparse && !pair_is_fp16(P, b, h, i, j)) continue;
     int fp16 = pair_is_fp16(P, b, h, i, j);
     block_values(P, b, h, j, fp16, vd);
     for (int r = 0; r < bq; ++r) {
@@ -454,11 +459,12 @@ static void attn_unit(const attn_problem* P, int b, int h, int i, int online, co
   for (int r = 0; r < bq; ++r) {
     int64_t orow = ((int64_t)b * P->Hq + h) * P->Nq + (int64_t)i * bq + r;
     for (int c = 0; c < d; ++c) {
-      double o = acc[(int64_t)r * d + c] / l[r];
+      /* l = 0 only when the row kept no key (R-sparse) */
+      double o = l[r] > 0.0 ? acc[(int64_t)r * d + c] / l[r] : 0.0;
       out[orow * d + c] = orc_double_to_half(o);
       if (out64) out64[orow * d + c] = o;
     }
-    lse[orow] = (float)(m[r] + log(l[r]));
+    lse[orow] = l[r] > 0.0 ? (float)(m[r] + log(l[r])) : -INFINITY;
   }
   free(S); free(qd); free(kd); free(vd); free(Pq); free(acc); free(m); free(l);
 }
@@ -497,10 +503,10 @@ static void* attn_worker(void* arg) {
 void orc_attn_qk(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint8_t* q4c, const uint8_t* q4s,
                  float q4t, const uint8_t* k4c, const uint8_t* k4s, float k4t, const uint8_t* v4c,
                  const uint8_t* v4s, float v4t, const uint8_t* sel, int B, int Hq, int Hkv, int Nq, int Nk, int d,
-                 int bq, int bk, int causal, float tau, const int32_t* units, int n_units, int online,
+                 int bq, int bk, int causal, float tau, int sparse, const int32_t* units, int n_units, int online,
                  const int32_t* order, uint16_t* out, float* lse, double* out64, int n_threads) {
   attn_problem P = {q, k, v, q4c, q4s, k4c, k4s, v4c, v4s, q4t, k4t, v4t, sel,
-                    B, Hq, Hkv, Nq, Nk, d, bq, bk, causal, (double)tau};
+                    B, Hq, Hkv, Nq, Nk, d, bq, bk, causal, (double)tau, sparse};
   attn_job J;
   J.P = &P; J.units = units; J.n_units = n_units; J.online = online; J.order = order;
   J.out = out; J.lse = lse; J.out64 = out64; J.next = 0;
@@ -520,7 +526,7 @@ void orc_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uin
               int bk, int causal, float tau, const int32_t* units, int n_units, int online,
               const int32_t* order, uint16_t* out, float* lse, double* out64, int n_threads) {
   orc_attn_qk(q, k, v, q4c, q4s, q4t, k4c, k4s, k4t, v4c, v4s, v4t, sel, B, Hq, Hkv, N, N, d, bq, bk, causal, tau,
-              units, n_units, online, order, out, lse, out64, n_threads);
+              0, units, n_units, online, order, out, lse, out64, n_threads);
 }
 
 /* The tau-scaled scores of one (b, h, query block i, key block j) tile, [bq, bk] float64,
@@ -529,7 +535,7 @@ void orc_tile_scores(const uint16_t* q, const uint16_t* k, const uint8_t* q4c, c
                      const uint8_t* k4c, const uint8_t* k4s, float k4t, int B, int Hq, int Hkv, int N, int d,
                      int bq, int bk, int causal, float tau, int b, int h, int i, int j, int fp16, double* S) {
   attn_problem P = {q, k, NULL, q4c, q4s, k4c, k4s, NULL, NULL, q4t, k4t, 0.0f, NULL,
-                    B, Hq, Hkv, N, N, d, bq, bk, causal, (double)tau};
+                    B, Hq, Hkv, N, N, d, bq, bk, causal, (double)tau, 0};
   double* qd = (double*)malloc(sizeof(double) * (size_t)d);
   double* kd = (double*)malloc(sizeof(double) * (size_t)bk * d);
   block_scores(&P, b, h, i, j, fp16, qd, kd, S, bk);
