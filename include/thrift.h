@@ -145,6 +145,15 @@ thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v,
                               float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes,
                               void* stream);
 
+/* Compute-matched sparse variant of thrift_attn_fwd (ThriftAttention compares against sparse
+ * attention at a matched compute budget): only the selected pairs of `mask` run, in FP16 with the
+ * FP16 q, k, v; every other pair is dropped as if masked.  A row left with no key gets output 0
+ * and lse -inf.  No NVFP4 tensor is read; mask required; counts and lists may be NULL.  The same
+ * fused kernel with an entry list of FP16 entries only. */
+thrift_status thrift_attn_fwd_sparse(const void* q, const void* k, const void* v, const uint32_t* mask,
+                                     const int32_t* counts, const int16_t* lists, void* out, float* lse,
+                                     const thrift_cfg* cfg, void* ws, size_t ws_bytes, void* stream);
+
 /* Workspace bytes of thrift_attn_fwd_auto (it also holds the NVFP4 copies and the selection). */
 size_t thrift_auto_workspace_bytes(const thrift_cfg* cfg);
 
@@ -211,6 +220,13 @@ thrift_status thrift_decode_select(const void* q, const double* kbar, const thri
 thrift_status thrift_decode_attn(const void* q, const void* k, const void* v, const thrift_nvfp4* k4,
                                  const thrift_nvfp4* v4, const uint32_t* mask, void* out, float* lse,
                                  const thrift_decode_cfg* cfg, void* ws, size_t ws_bytes, void* stream);
+
+/* Compute-matched sparse variant of thrift_decode_attn (the baseline the pages compare against:
+ * only the selected key blocks, in FP16, every other block dropped; a row left with no key gets
+ * output 0 and lse -inf).  Same arguments without the NVFP4 cache; mask required. */
+thrift_status thrift_decode_attn_sparse(const void* q, const void* k, const void* v, const uint32_t* mask,
+                                        void* out, float* lse, const thrift_decode_cfg* cfg, void* ws,
+                                        size_t ws_bytes, void* stream);
 
 /* One decode step: thrift_decode_select (selection kept in the workspace), then
  * thrift_decode_attn. */

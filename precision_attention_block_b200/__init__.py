@@ -24,7 +24,8 @@ from ._lib import ThriftError, check, load
 
 __all__ = ["Config", "NVFP4Tensor", "Selection", "Workspace", "quantize_nvfp4", "quantize_qkv",
            "block_select", "attn_fwd", "attn_fwd_auto", "DecodeConfig", "KVCache", "kv_block_means",
-           "decode_select", "decode_attn", "decode_fwd", "device_status", "reset_device_status",
+           "decode_select", "decode_attn", "decode_fwd", "attn_fwd_sparse", "decode_attn_sparse",
+           "device_status", "reset_device_status",
            "ThriftError", "load"]
 
 
@@ -205,6 +206,24 @@ def attn_fwd(q, k, v, q4: Optional[NVFP4Tensor], k4: Optional[NVFP4Tensor], v4: 
     return out, lse
 
 
+def attn_fwd_sparse(q, k, v, sel: Selection, cfg: Config, out=None, lse=None, ws: Optional[Workspace] = None,
+                    want_lse: bool = True):
+    """Compute-matched sparse variant (thrift_attn_fwd_sparse): only the selected pairs, in FP16;
+    rows left with no key get 0 and lse -inf.  Returns (out, lse)."""
+    dev = q.device
+    if out is None:
+        out = torch.empty((cfg.B, cfg.Hq, cfg.N, cfg.d), dtype=torch.float16, device=dev)
+    if lse is None and want_lse:
+        lse = torch.empty((cfg.B, cfg.Hq, cfg.N), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = Workspace(256, dev)
+    c = cfg.c()
+    check(load().thrift_attn_fwd_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(sel.mask), _ptr(sel.counts),
+                                        _ptr(sel.lists), _ptr(out), _ptr(lse), ctypes.byref(c), ws.ptr, ws.nbytes,
+                                        _stream()), "thrift_attn_fwd_sparse")
+    return out, lse
+
+
 def attn_fwd_auto(q, k, v, cfg: Config, out=None, lse=None, ws: Optional[Workspace] = None,
                   want_lse: bool = True):
     """Quantise, select and attend in one call (thrift_attn_fwd_auto).  Returns (out, lse)."""
@@ -379,4 +398,18 @@ def decode_fwd(q: torch.Tensor, cache: KVCache, cfg: DecodeConfig, out=None, lse
     check(load().thrift_decode_fwd(_ptr(q), _ptr(cache.k), _ptr(cache.v), ctypes.byref(k4), ctypes.byref(v4),
                                    _ptr(cache.kbar), _ptr(out), _ptr(lse), ctypes.byref(c), ws.ptr, ws.nbytes,
                                    _stream()), "thrift_decode_fwd")
+    return out, lse
+
+
+def decode_attn_sparse(q: torch.Tensor, cache: KVCache, sel: Selection, cfg: DecodeConfig, out=None, lse=None,
+                       ws: Optional[Workspace] = None, want_lse: bool = True):
+    """Compute-matched sparse decode (thrift_decode_attn_sparse): only the selected key blocks, in
+    FP16.  Returns (out, lse)."""
+    out, lse = _decode_out(q, cfg, out, lse, want_lse)
+    if ws is None:
+        ws = cfg.workspace(q.device)
+    c = cfg.c()
+    check(load().thrift_decode_attn_sparse(_ptr(q), _ptr(cache.k), _ptr(cache.v), _ptr(sel.mask), _ptr(out),
+                                           _ptr(lse), ctypes.byref(c), ws.ptr, ws.nbytes, _stream()),
+          "thrift_decode_attn_sparse")
     return out, lse

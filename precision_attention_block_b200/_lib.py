@@ -74,6 +74,8 @@ SIGNATURES = {
     "thrift_decode_workspace_bytes": (_sz, [_dcfgp]),
     "thrift_decode_select": (ctypes.c_int, [_vp, _vp, _dcfgp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "thrift_decode_attn": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _vp, _vp, _vp, _dcfgp, _vp, _sz, _vp]),
+    "thrift_decode_attn_sparse": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _dcfgp, _vp, _sz, _vp]),
+    "thrift_attn_fwd_sparse": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _cfgp, _vp, _sz, _vp]),
     "thrift_decode_fwd": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _vp, _vp, _vp, _dcfgp, _vp, _sz, _vp]),
     "thrift_reset_device_status": (ctypes.c_int, [_vp, _vp]),
     "thrift_get_device_status": (ctypes.c_int, [_vp, _vp, ctypes.POINTER(_i32)]),

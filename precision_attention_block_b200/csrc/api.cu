@@ -161,22 +161,23 @@ bool al16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
 
 thrift_status decode_attn_common(const void* q, const void* k, const void* v, const thrift_nvfp4* k4,
                                  const thrift_nvfp4* v4, const uint32_t* mask, void* out, float* lse,
-                                 const thrift_decode_cfg* cfg, void* ws, size_t ws_bytes, cudaStream_t s) {
-  const int mode = decode_mode(cfg);
+                                 const thrift_decode_cfg* cfg, void* ws, size_t ws_bytes, cudaStream_t s,
+                                 bool sparse = false) {
+  const int mode = sparse ? 3 : decode_mode(cfg);
   if (!q || !out || !al16(q)) return THRIFT_ERR_INVALID_ARG;
   if (mode != 1 && (!k || !v || !al16(k) || !al16(v))) return THRIFT_ERR_INVALID_ARG;
-  if (mode != 2) {
+  if (mode <= 1) {
     if (!nvfp4_ok(k4, 0) || !nvfp4_ok(v4, 1)) return THRIFT_ERR_INVALID_ARG;
     if (!al16(k4->codes) || !al16(k4->scales) || !al16(v4->codes) || !al16(v4->scales_mma))
       return THRIFT_ERR_INVALID_ARG;
   }
-  if (mode == 0 && !mask) return THRIFT_ERR_INVALID_ARG;
+  if ((mode == 0 || mode == 3) && !mask) return THRIFT_ERR_INVALID_ARG;
   const DecodeLayout L = decode_layout(*cfg);
   if (!ws_ok(ws, ws_bytes, L.bytes)) return THRIFT_ERR_WORKSPACE;
   uint8_t* w = static_cast<uint8_t*>(ws);
   thrift_nvfp4 q4 = {w + L.q4c, w + L.q4s, w + L.q4m, reinterpret_cast<float*>(w + L.qts), 0};
   const thrift_decode_cfg& c = *cfg;
-  if (mode != 2) {
+  if (mode <= 1) {
     unsigned int* amax = reinterpret_cast<unsigned int*>(w + kWsAmaxOff);
     thrift_status st = quantize_launch(q, (int64_t)c.B * c.Hq, c.Nq, c.d, &q4, amax, s);
     if (st != THRIFT_OK) return st;
@@ -189,7 +190,7 @@ thrift_status decode_attn_common(const void* q, const void* k, const void* v, co
   a.q4 = &q4;
   a.k4 = k4;
   a.v4 = v4;
-  a.mask = mode == 0 ? mask : nullptr;
+  a.mask = (mode == 0 || mode == 3) ? mask : nullptr;
   a.mode = mode;
   a.out = out;
   a.lse = lse;
@@ -352,6 +353,28 @@ thrift_status thrift_decode_attn(const void* q, const void* k, const void* v, co
   thrift_status st = dcfg_supported(cfg);
   if (st != THRIFT_OK) return st;
   return decode_attn_common(q, k, v, k4, v4, mask, out, lse, cfg, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+thrift_status thrift_decode_attn_sparse(const void* q, const void* k, const void* v, const uint32_t* mask, void* out,
+                                        float* lse, const thrift_decode_cfg* cfg, void* ws, size_t ws_bytes,
+                                        void* stream) {
+  thrift_status st = dcfg_supported(cfg);
+  if (st != THRIFT_OK) return st;
+  return decode_attn_common(q, k, v, nullptr, nullptr, mask, out, lse, cfg, ws, ws_bytes,
+                            static_cast<cudaStream_t>(stream), true);
+}
+
+thrift_status thrift_attn_fwd_sparse(const void* q, const void* k, const void* v, const uint32_t* mask,
+                                     const int32_t* counts, const int16_t* lists, void* out, float* lse,
+                                     const thrift_cfg* cfg, void* ws, size_t ws_bytes, void* stream) {
+  (void)counts;
+  (void)lists;
+  thrift_status st = cfg_supported(cfg);
+  if (st != THRIFT_OK) return st;
+  if (!q || !k || !v || !mask || !out) return THRIFT_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, kWsHeader)) return THRIFT_ERR_WORKSPACE;
+  return attn_launch_dbg(q, k, v, nullptr, nullptr, nullptr, mask, 3, out, lse, *cfg, status_ptr(ws), nullptr, -1,
+                         static_cast<cudaStream_t>(stream));
 }
 
 thrift_status thrift_decode_fwd(const void* q, const void* k, const void* v, const thrift_nvfp4* k4,

@@ -130,7 +130,7 @@ struct AttnParams {
   int* status;
   float* dbg;  // optional dump of one entry (S, P bytes, PV) of tile 0 of the first unit of CTA 0
   int dbg_entry;
-  int B, Hq, Hkv, N, bq, causal, mode, nqb, nkb, mask_words, n_units;
+  int B, Hq, Hkv, N, bq, causal, mode, nqb, nkb, mask_words, n_units;  // mode as attn_launch
   int npage, maxe, off_bar, off_list;
   float tau;
   long long wait_limit;
@@ -161,9 +161,9 @@ __device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, int u) {
 // The entry list of one 128-row tile of query head h, built by a whole warp: NVFP4 entries, then
 // FP16 entries, each as j | fp16 << 13 | row-half mask << 14 (with 64-row query blocks a key
 // block can be NVFP4 for one half of the tile and FP16 for the other).  Returns the number of
-// entries (same in every lane).
+// entries (same in every lane), at least min_entries.
 template <int BK>
-__device__ int build_list(const AttnParams& p, int b, int h, int t, uint16_t* list, int lane) {
+__device__ int build_list(const AttnParams& p, int b, int h, int t, uint16_t* list, int lane, int min_entries) {
   const bool two = p.bq == 64;
   const int i0 = two ? 2 * t : t, i1 = i0 + 1;
   const uint32_t* base = p.mask ? p.mask + ((int64_t)(b * p.Hq + h) * p.nqb) * p.mask_words : nullptr;
@@ -184,7 +184,8 @@ __device__ int build_list(const AttnParams& p, int b, int h, int t, uint16_t* li
     return (int)((__ldg(m + (jj >> 5)) >> (jj & 31)) & 1u);
   };
   int n = 0;
-  for (int phase = 0; phase < 2; ++phase) {
+  // the sparse variant (mode 3) keeps only the FP16 (selected) entries
+  for (int phase = p.mode == 3 ? 1 : 0; phase < 2; ++phase) {
     for (int jb = 0; jb < jmax; jb += 32) {
       const int jj = jb + lane;
       int rm = 0;
@@ -195,6 +196,17 @@ __device__ int build_list(const AttnParams& p, int b, int h, int t, uint16_t* li
       if (rm) list[n + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)(jj | (phase << 13) | (rm << 14));
       n += __popc(bal);
     }
+  }
+  // The softmax warpgroups merge a tile's last PV products (the last min_entries visits, which lag
+  // that far behind S) while they wait for the next tile's first min_entries visits; those must
+  // come from the next list, since the list after it is built only once this tile is released.
+  // A shorter list (the sparse variant's empty tiles; a first causal tile with a single key block)
+  // is padded with entries in which no row takes part (rm = 0: every probability is 0), NVFP4
+  // ones when only NVFP4 operands exist, FP16 ones otherwise.
+  if (n < min_entries) {
+    if (lane < min_entries - n) list[n + lane] = (uint16_t)(p.mode == 1 ? 0 : (1 << 13));
+    __syncwarp();
+    n = min_entries;
   }
   return n;
 }
@@ -439,7 +451,7 @@ __global__ void __launch_bounds__(384, 1)
     if (warp == 0) {
       // ---------------------------------------------------------------- producer
       if (lane == 0) {
-        if (p.mode != 2) {
+        if (p.mode <= 1) {
           prefetch_tmap(&tm_q4);
           prefetch_tmap(&tm_k4);
           prefetch_tmap(&tm_v4);
@@ -460,7 +472,7 @@ __global__ void __launch_bounds__(384, 1)
         const bool free_ok = mbar_wait(&bars->list_empty[lb], lph ^ 1, abort_flag, p.status, lim);
         if (!__all_sync(0xffffffffu, free_ok)) break;
         uint16_t* list = lists + lb * p.maxe;
-        const int n = build_list<BK>(p, ui.b, ui.h, ui.t, list, lane);
+        const int n = build_list<BK>(p, ui.b, ui.h, ui.t, list, lane, L::NPV);
         __syncwarp();
         if (lane == 0) {
           bars->list_count[lb] = n;
@@ -469,7 +481,7 @@ __global__ void __launch_bounds__(384, 1)
           const int qrow0 = (ui.b * p.Hq + ui.h) * p.N + ui.t * kBQ;
           if ((ok = mbar_wait(&bars->q4_empty, (uc & 1) ^ 1, abort_flag, p.status, lim))) {
             uint8_t* sq = smem + L::OFF_Q4;
-            if (p.mode != 2) {
+            if (p.mode <= 1) {
               mbar_arrive_expect_tx(&bars->q4_full, L::Q4_BYTES + L::QSF_BYTES);
               tma_load_2d(sq, &tm_q4, &bars->q4_full, 0, qrow0);
               bulk_load(sq + L::Q4_BYTES, p.q_sf + (size_t)(qrow0 / 128) * L::QSF_BYTES, L::QSF_BYTES, &bars->q4_full);
@@ -541,7 +553,7 @@ __global__ void __launch_bounds__(384, 1)
           const uint16_t* list = lists + lb * p.maxe;
           if (!(ok = mbar_wait(&bars->q4_full, uc & 1, abort_flag, p.status, lim))) break;
           tc_fence_after();
-          if (p.mode != 2) {
+          if (p.mode <= 1) {
 #pragma unroll
             for (int kk = 0; kk < D / 64; ++kk)
               tc_copy_sf(tmem + L::COL_SFQ + 4 * kk, make_sdesc(qb4 + L::Q4_BYTES + kk * 512, 16, 128, 0));
@@ -701,9 +713,9 @@ __global__ void __launch_bounds__(384, 1)
     const int quarter = warp & 3;
     const int rr = quarter * 32 + lane;  // row of the tile = TMEM lane
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    const float q_ts = (p.mode != 2) ? __ldg(p.q_ts) : 1.0f;
-    const float k_ts = (p.mode != 2) ? __ldg(p.k_ts) : 1.0f;
-    const float v_ts = (p.mode != 2) ? __ldg(p.v_ts) : 1.0f;
+    const float q_ts = (p.mode <= 1) ? __ldg(p.q_ts) : 1.0f;
+    const float k_ts = (p.mode <= 1) ? __ldg(p.k_ts) : 1.0f;
+    const float v_ts = (p.mode <= 1) ? __ldg(p.v_ts) : 1.0f;
     const float sl2_4 = q_ts * k_ts * p.tau * kLog2e;
     const float sl2_16 = p.tau * kLog2e;
     const float pv4_scale = v_ts * (1.0f / 2688.0f);
@@ -960,6 +972,7 @@ thrift_status launch_t(const void* q, const void* k, const void* v, const thrift
   using L = Layout<D, BK>;
   // entry lists: [unit parity][maxe] u16 after the barrier block; the rest goes to pages
   prm.maxe = (prm.bq == 64 ? 2 : 1) * prm.nkb;
+  if (prm.maxe < L::NPV) prm.maxe = L::NPV;  // lists are padded to NPV entries
   const int list_bytes = (2 * prm.maxe * 2 + 1023) & ~1023;
   const int room = kSmemLimit - L::fixed_bytes() - list_bytes;
   int npage = room / L::PAGE;
@@ -975,7 +988,7 @@ thrift_status launch_t(const void* q, const void* k, const void* v, const thrift
   memset(maps, 0, sizeof(maps));
   const uint64_t qrows = (uint64_t)prm.B * prm.Hq * prm.N, krows = (uint64_t)prm.B * prm.Hkv * prm.N;
   bool ok = true;
-  if (prm.mode != 2) {
+  if (prm.mode <= 1) {
     ok &= make_map(&maps[0], q4->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D / 2, qrows, D / 2, kBQ, swz_enum(D / 2));
     ok &= make_map(&maps[1], k4->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D / 2, krows, D / 2, BK, swz_enum(D / 2));
     ok &= make_map(&maps[2], v4->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)prm.N / 2,
@@ -1025,7 +1038,7 @@ thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const
   AttnParams prm;
   memset(&prm, 0, sizeof(prm));
   prm.mask = mask;
-  if (mode != 2) {
+  if (mode <= 1) {
     prm.q_sf = q4->scales_mma;
     prm.k_sf = k4->scales_mma;
     prm.v_sf = v4->scales_mma;

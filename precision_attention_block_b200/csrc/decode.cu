@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_kernel(const __grid_c
   const int j0 = split * p.bps;
   const int nblk = min(p.bps, p.nkb - j0);
   const uint32_t all_heads = (1u << p.G) - 1u;
-  const bool use4 = p.mode != 2;
+  const bool use4 = p.mode <= 1;  // modes 2 and 3 read no NVFP4 operand
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -379,6 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_kernel(const __grid_c
     const int j = j0 + i;
     const uint32_t bits = bits_of(i);
     const bool n16 = bits != 0u, n4 = use4 && bits != all_heads;
+    if (!n4 && !n16 && !use4) continue;  // sparse variant: no head of the group selected this block
     const int s4 = i % NST, s16 = c16_acc % NF;
     if (use4) {
       ok = wait_tag(&tag4[s4], i, abort_flag, p.status, p.wait_limit);
@@ -455,7 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_kernel(const __grid_c
         for (int e = 0; e < 4; ++e) {
           const int rs = e >> 1;
           const int kk = tig * (BK / 4) + 4 * (nt >> 1) + 2 * (nt & 1) + (e & 1);
-          if (g + 8 * rs >= R || (p.causal && (int64_t)j * BK + kk > qpos[rs])) sc[nt][e] = kNegInf;
+          if (g + 8 * rs >= R || (p.causal && (int64_t)j * BK + kk > qpos[rs]) || (p.mode == 3 && !f16r[rs]))
+            sc[nt][e] = kNegInf;
         }
     }
 
@@ -739,7 +741,7 @@ thrift_status decode_launch_t(const DecodeArgs& a, DecodeParams& prm, cudaStream
   using L = DLayout<D, BK>;
   CUtensorMap tm;
   memset(&tm, 0, sizeof(tm));
-  if (prm.mode != 2) {
+  if (prm.mode <= 1) {
     if (!make_u8_map(&tm, a.v4->codes, (uint64_t)prm.Nk / 2, (uint64_t)prm.B * prm.Hkv * D, BK / 2, D))
       return THRIFT_ERR_CUDA;
   } else {
@@ -790,7 +792,7 @@ thrift_status decode_attn_launch(const DecodeArgs& a, cudaStream_t stream) {
   prm.q = reinterpret_cast<const __half*>(a.q);
   prm.k16 = reinterpret_cast<const __half*>(a.k);
   prm.v16 = reinterpret_cast<const __half*>(a.v);
-  if (a.mode != 2) {
+  if (a.mode <= 1) {
     prm.q4c = a.q4->codes;
     prm.q4s = a.q4->scales;
     prm.q_ts = a.q4->tensor_scale;

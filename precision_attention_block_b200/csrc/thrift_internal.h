@@ -34,7 +34,8 @@ thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, u
 size_t noalloc_select_scratch_bytes();
 thrift_status noalloc_select_scratch(uint8_t** out);
 
-// mode: 0 = FP16 pairs from the mask, 1 = every pair NVFP4, 2 = every pair FP16.
+// mode: 0 = FP16 pairs from the mask, 1 = every pair NVFP4, 2 = every pair FP16, 3 = only the
+// FP16 pairs of the mask (the compute-matched sparse variant; no NVFP4 operand is read).
 thrift_status attn_launch(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
                           const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
                           void* out, float* lse, const thrift_cfg& c, int* status, cudaStream_t stream);
