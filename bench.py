@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-units", type=int, default=8)
+    ap.add_argument("--sparse", action="store_true",
+                    help="the compute-matched sparse variant: only the selected pairs, in FP16")
     return ap.parse_args()
 
 
@@ -320,22 +322,26 @@ def main():
     stream = torch.cuda.current_stream()
 
     def step(evs=None):
-        pab.quantize_nvfp4(gq, 0, out=q4, ws=ws)
-        pab.quantize_nvfp4(gk, 0, out=k4, ws=ws)
-        pab.quantize_nvfp4(gv, 1, out=v4, ws=ws)
+        if not args.sparse:
+            pab.quantize_nvfp4(gq, 0, out=q4, ws=ws)
+            pab.quantize_nvfp4(gk, 0, out=k4, ws=ws)
+            pab.quantize_nvfp4(gv, 1, out=v4, ws=ws)
         if evs:
             evs[0].record(stream)
         pab.block_select(gq, gk, cfg, ws=ws, out=sel)
         if evs:
             evs[1].record(stream)
-        pab.attn_fwd(gq, gk, gv, q4, k4, v4, sel, cfg, out=out, lse=lse, ws=ws)
+        if args.sparse:
+            pab.attn_fwd_sparse(gq, gk, gv, sel, cfg, out=out, lse=lse, ws=ws)
+        else:
+            pab.attn_fwd(gq, gk, gv, q4, k4, v4, sel, cfg, out=out, lse=lse, ws=ws)
         if evs:
             evs[2].record(stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    launches_per_step = 3 * 2 + 5 + 1  # amax + encode per tensor; means x2, scores, top-k, lists; attention
+    launches_per_step = (0 if args.sparse else 3 * 2) + 5 + 1  # amax + encode per tensor; selection; attention
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     ev_start = torch.cuda.Event(enable_timing=True)
     ev_end = torch.cuda.Event(enable_timing=True)
@@ -375,12 +381,14 @@ def main():
     k_total = valid_total if mode_fp16_all else (0 if mode_fp4_all else counts)
     per_pair = 4.0 * w.block_q * w.block_k * w.d
     F16, F4 = k_total * per_pair, (valid_total - k_total) * per_pair
+    if args.sparse:  # only the selected pairs run
+        F16, F4 = counts * per_pair, 0.0
     bf16_burst, bf16_sustained, hbm_gbs, peak_src = peaks()
     p16, p4 = bf16_burst * 1e12, bf16_burst * NVFP4_PER_FP16 * 1e12
     t_roof = F16 / p16 + F4 / p4
     achieved = (F16 + F4) / (attn_mean_ms * 1e-3) / 1e12
     peak_blend = (F16 + F4) / t_roof / 1e12
-    traffic = stored_traffic(w.name) if args.budget_bp is None else None
+    traffic = stored_traffic(w.name) if args.budget_bp is None and not args.sparse else None
 
     eff = effective_flops(w)
     qkv_mb = (q.nbytes + k.nbytes + v.nbytes) / 1e6
@@ -396,6 +404,8 @@ def main():
                               else f"inputs smaller than L2 ({qkv_mb:.0f} MB); no flush")},
             "breakdown_ms": {"quantize": statistics.mean(quant_ms), "select": statistics.mean(sel_ms),
                              "attention": attn_mean_ms},
+            "variant": "sparse (selected pairs only, FP16; effective FLOPs of the dense problem)" if args.sparse
+                       else "mixed NVFP4/FP16",
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_blend, "unit": "TFLOP/s",
                          "frac": achieved / peak_blend, "traffic": traffic,
                          "peak_note": f"blend of {peak_src} bf16 burst {bf16_burst:.1f} TF/s (FP16) and "
@@ -403,9 +413,9 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
             "device_status": status}
 
-    if not args.no_e2e:
+    if not args.no_e2e and not args.sparse:
         line["e2e"] = e2e_measure(pab, torch, w, cfg, q, k, v, device, args, world, dist)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.sparse:
         line["cpu_baseline"] = cpu_baseline(w, q, k, v, args.cpu_units)
     line["clocks"] = sampler.summary()
     if rank == 0:
@@ -465,6 +475,7 @@ def main_decode(args, w, pab, torch, device, world, rank, local_rank, dist):
     cfg16 = pab.DecodeConfig.from_workload(w.with_budget(10000))
     ws16 = cfg16.workspace(device)
     fp16_graph = graph_of(lambda: pab.decode_attn(gq, cache, None, cfg16, out=out, lse=lse, ws=ws16))
+    sparse_graph = graph_of(lambda: pab.decode_attn_sparse(gq, cache, sel, cfg, out=out, lse=lse, ws=ws))
 
     def timed(g, steps, warmup):
         for _ in range(warmup):
@@ -488,6 +499,7 @@ def main_decode(args, w, pab, torch, device, world, rank, local_rank, dist):
         step_ms = timed(step_graph, args.steps, args.warmup)
     attn_ms = timed(attn_graph, args.steps, args.warmup)
     fp16_ms = timed(fp16_graph, max(3, args.steps // 4), 2)
+    sparse_ms = timed(sparse_graph, max(3, args.steps // 4), 2)
     status = pab.device_status(ws)
     _, _, hbm_gbs, peak_src = peaks()
     attn_bytes = alg_bytes - w.B * w.Hkv * (w.N // w.block_k) * w.d * 8
@@ -503,13 +515,14 @@ def main_decode(args, w, pab, torch, device, world, rank, local_rank, dist):
                              if cache_mb > 126 else f"cache {cache_mb:.0f} MB: L2 not flushed"},
             "breakdown_us": {"step": 1e3 * step_ms, "attention": 1e3 * attn_ms,
                              "select_and_quantize": 1e3 * (step_ms - attn_ms),
-                             "all_fp16_attention_same_kernel": 1e3 * fp16_ms},
+                             "all_fp16_attention_same_kernel": 1e3 * fp16_ms,
+                             "sparse_attention_selected_blocks_only": 1e3 * sparse_ms},
             "blocks": {"nvfp4": blocks4, "fp16": blocks16, "of": w.B * w.Hkv * (w.N // w.block_k)},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
                          "frac": achieved / hbm_gbs, "traffic": None,
                          "peak_note": f"{peak_src} HBM copy bandwidth; achieved = the attention kernels' "
                                       f"algorithmic bytes ({attn_bytes / 1e6:.1f} MB) / their time"},
-            "gpu_launches": 8 * args.steps,
+            "gpu_launches": 8 * args.steps,  # amax, encode, means, scores, top-k, lists, attention, combine
             "device_status": status}
     if not args.no_e2e:
         hq = torch.from_numpy(q).pin_memory()
