@@ -61,6 +61,16 @@ def parse():
     return ap.parse_args()
 
 
+def max_over_ranks(values, device, dist):
+    """Element-wise maximum of per-rank timings over all ranks (the slowest rank sets the job
+    time); the values themselves when there is a single process."""
+    import torch
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 def effective_flops(w) -> float:
     f = 4.0 * w.B * w.Hq * w.N * w.N * w.d
     return f / 2 if w.causal else f
@@ -365,10 +375,7 @@ def main():
     attn_ms = [evs[s][1].elapsed_time(evs[s][2]) for s in range(args.steps)]
     sel_ms = [evs[s][0].elapsed_time(evs[s][1]) for s in range(args.steps)]
     quant_ms = [step_starts[s].elapsed_time(evs[s][0]) for s in range(args.steps)]
-    t = torch.tensor([total_ms, statistics.mean(attn_ms)], dtype=torch.float64, device=device)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, attn_mean_ms = float(t[0]), float(t[1])
+    total_ms, attn_mean_ms = max_over_ranks([total_ms, statistics.mean(attn_ms)], device, dist)
 
     # status word: any device-side timeout invalidates the run
     status = pab.device_status(ws)
@@ -489,10 +496,7 @@ def main_decode(args, w, pab, torch, device, world, rank, local_rank, dist):
             g.replay()
         b.record()
         torch.cuda.synchronize()
-        t = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=device)
-        if dist:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t[0]) / steps
+        return max_over_ranks([a.elapsed_time(b)], device, dist)[0] / steps
 
     sampler = ClockSampler(local_rank)
     with sampler:
@@ -590,14 +594,12 @@ def e2e_measure(pab, torch, w, cfg, q, k, v, device, args, world, dist):
         step()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=device)
-    if dist:
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-    value = world * effective_flops(w) * steps / (float(ms[0]) * 1e-3) / 1e12
+    ms = max_over_ranks([a.elapsed_time(b)], device, dist)
+    value = world * effective_flops(w) * steps / (ms[0] * 1e-3) / 1e12
     return {"value": value, "unit": "TFLOPS", "steps": steps,
             "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
             "d2h_bytes_per_step": int(ho.numel() * 2 + hl.numel() * 4),
-            "ms_per_step": float(ms[0]) / steps}
+            "ms_per_step": ms[0] / steps}
 
 
 if __name__ == "__main__":
