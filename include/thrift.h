@@ -177,7 +177,14 @@ thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, 
  *
  * The cache: k, v FP16 [B,Hkv,Nk,d]; k4 = thrift_quantize_nvfp4(k, group_axis 0), v4 =
  * thrift_quantize_nvfp4(v, group_axis 1); kbar = thrift_kv_block_means(k).  All owned by the
- * caller and only read. */
+ * caller and only read.  q, k, v and the NVFP4 codes, scales and scales_mma buffers must be
+ * 16-byte aligned (they are copied with bulk/tensor copies).
+ *
+ * Errors (every decode entry point): THRIFT_ERR_INVALID_ARG for a null or misaligned pointer or
+ * an inconsistent configuration, THRIFT_ERR_UNSUPPORTED outside the implemented sizes,
+ * THRIFT_ERR_WORKSPACE for a null, misaligned or too small workspace -- all detected on the host
+ * before anything is launched; a device-side wait that runs out is recorded in the workspace
+ * status word (thrift_get_device_status). */
 typedef struct {
   int32_t B, Hq, Hkv;  /* batch, query heads, key/value heads (Hq % Hkv == 0) */
   int32_t Nq;          /* query rows per head in this step, 1 <= Nq, (Hq/Hkv) * Nq <= 16 */
@@ -193,7 +200,8 @@ typedef struct {
 
 /* Block means of the cache's keys: kbar [outer, Nk/block_k, d] float64, the exact FP16 sum of
  * each column over the block's tokens divided by block_k (k: device FP16 [outer, Nk, d]).
- * Computed once per cache (and per appended block); thrift_decode_select reads it. */
+ * Computed once per cache; thrift_decode_select reads it.  Requires d in {64,128}, block_k in
+ * {64,128}, Nk a multiple of block_k. */
 thrift_status thrift_kv_block_means(const void* k, int64_t outer, int32_t Nk, int32_t d, int32_t block_k,
                                     double* kbar, void* stream);
 

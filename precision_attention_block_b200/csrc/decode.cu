@@ -14,16 +14,17 @@
 //   quantise   the query rows as their own NVFP4 tensor (the quantiser of quantize.cu);
 //   select     qbar = mean of the Nq rows of each head; S^_j = qbar . kbar_j with kbar the
 //              cache's block means (computed once per cache by thrift_kv_block_means); top-k
-//              key blocks per (batch, query head) -- the kernels of select.cu with one query
-//              block;
+//              key blocks per (batch, query head) -- select.cu, one query block per head;
 //   attend     split over key blocks: CTA (split, batch * KV head) walks its key blocks.  A
 //              producer warp streams each block's NVFP4 K and V (and, when one of the group's
 //              heads selected the block, its FP16 K and V) into shared memory with bulk and
-//              tensor copies; seven consumer warps, each on its own key blocks, compute S = Q K^T
-//              (fragments kept in registers), the per-row block maximum
-//              M, P^ = exp(S - M), the two-level NVFP4 re-quantisation of P^ (FP16 rounding on
+//              tensor copies; seven consumer warps, each claiming the next unclaimed block,
+//              compute S = Q K^T (S fragments in registers), the per-row block maximum M,
+//              P^ = exp(S - M), the two-level NVFP4 re-quantisation of P^ (FP16 rounding on
 //              selected blocks), P V, and merge with weight exp(M - m) into FP32 partial sums;
+//              the warps' partials are combined in shared memory at the end of the split;
 //   combine    the splits' partial (O, m, l) of each row into O / l (FP16) and lse.
+// The sparse variant (mode 3) runs only the selected blocks, in FP16.
 //
 // NVFP4 operands enter the tensor cores as FP16: an E2M1 value times its E4M3 scale has at most
 // 6 significant bits and lies in [2^-10, 2688], so the FP16 value is exact, the products are
