@@ -116,44 +116,38 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int& total
   return before;
 }
 
-// One CTA per (batch, query head).  THREADS = kSelThreads for long rows; short rows (decode: one
-// query block) run with fewer threads, which makes the block-wide barriers of each pass cheaper.
-template <int THREADS>
-__global__ void __launch_bounds__(THREADS) topk_kernel(const double* __restrict__ scores, int64_t n,
-                                                           int nkb, int topk_abs, int topk_bp, int mask_words,
-                                                           uint32_t* __restrict__ mask) {
-  __shared__ unsigned int hist[256];
-  __shared__ int warp_sums[32];
-  __shared__ unsigned long long s_prefix;
-  __shared__ long long s_need;
-  __shared__ unsigned long long s_nvalid;
-  __shared__ unsigned long long keys_sm[kSelSmemKeys];
-  const double* sc = scores + (int64_t)blockIdx.x * n;
-  int nqb = (int)(n / nkb);
-  uint32_t* mk = mask + (int64_t)blockIdx.x * nqb * mask_words;
-  // rows of up to kSelSmemKeys scores are read from global memory once and kept in shared memory
-  const bool in_smem = n <= kSelSmemKeys;
-  if (in_smem)
-    for (int64_t t = threadIdx.x; t < n; t += THREADS) keys_sm[t] = score_key(sc[t]);
-  auto key_at = [&](int64_t t) -> uint64_t { return in_smem ? keys_sm[t] : score_key(sc[t]); };
+struct TopkShared {
+  unsigned int hist[256];
+  int warp_sums[32];
+  unsigned long long prefix;
+  long long need;
+  unsigned long long nvalid;
+};
 
+// Top-k of one row of n order-preserving keys (key_at(t); 0 = invalid pair) by a block of THREADS
+// threads: a most-significant-digit-first radix select finds the k-th largest key, every key above
+// it is taken and the first `need` ties in index order.  Chosen index t sets bit (t % nkb) of word
+// (t / nkb) * mask_words + (t % nkb) / 32 of mk, which the caller has zeroed.
+template <int THREADS, typename KeyAt>
+__device__ void topk_row(KeyAt key_at, int64_t n, int nkb, int topk_abs, int topk_bp, int mask_words,
+                         uint32_t* __restrict__ mk, TopkShared& sh) {
   // count valid pairs
-  if (threadIdx.x == 0) s_nvalid = 0;
+  if (threadIdx.x == 0) sh.nvalid = 0;
   __syncthreads();
   unsigned long long cnt = 0;
   for (int64_t t = threadIdx.x; t < n; t += THREADS) cnt += key_at(t) != 0ull;
-  atomicAdd(&s_nvalid, cnt);
+  atomicAdd(&sh.nvalid, cnt);
   __syncthreads();
-  long long nvalid = (long long)s_nvalid;
+  long long nvalid = (long long)sh.nvalid;
   long long k = topk_abs >= 0 ? (long long)topk_abs : ((long long)topk_bp * nvalid + 9999) / 10000;
   if (k > nvalid) k = nvalid;
-  if (k <= 0) return;  // mask already zeroed by the caller
+  if (k <= 0) return;
 
   // radix select: prefix of the k-th largest key, 8 bits at a time from the top
   unsigned long long prefix = 0ull;
   long long need = k;  // rank (1-based) of the wanted key among keys matching the prefix
   for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int b = threadIdx.x; b < 256; b += THREADS) hist[b] = 0;
+    for (int b = threadIdx.x; b < 256; b += THREADS) sh.hist[b] = 0;
     __syncthreads();
     unsigned long long hi_mask = shift == 56 ? 0ull : (~0ull << (shift + 8));
     if (shift >= 48) {
@@ -166,12 +160,12 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const double* __restrict_
         const bool in = key != 0ull && (key & hi_mask) == prefix;
         const int bin = in ? (int)((key >> shift) & 255) : -1;
         const unsigned peers = __match_any_sync(0xffffffffu, bin);
-        if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (unsigned)__popc(peers));
+        if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], (unsigned)__popc(peers));
       }
     } else {
       for (int64_t t = threadIdx.x; t < n; t += THREADS) {
         const uint64_t key = key_at(t);
-        if (key != 0ull && (key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1u);
+        if (key != 0ull && (key & hi_mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & 255], 1u);
       }
     }
     __syncthreads();
@@ -181,7 +175,7 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const double* __restrict_
       const int lane = threadIdx.x;
       long long mine = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mine += hist[255 - 8 * lane - i];
+      for (int i = 0; i < 8; ++i) mine += sh.hist[255 - 8 * lane - i];
       long long incl = mine;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -194,16 +188,16 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const double* __restrict_
         long long acc = incl - mine;
         int b = 255 - 8 * lane;
         for (int i = 0; i < 7; ++i, --b) {
-          if (acc + (long long)hist[b] >= need) break;
-          acc += hist[b];
+          if (acc + (long long)sh.hist[b] >= need) break;
+          acc += sh.hist[b];
         }
-        s_prefix = prefix | ((unsigned long long)b << shift);
-        s_need = need - acc;
+        sh.prefix = prefix | ((unsigned long long)b << shift);
+        sh.need = need - acc;
       }
     }
     __syncthreads();
-    prefix = s_prefix;
-    need = s_need;
+    prefix = sh.prefix;
+    need = sh.need;
     __syncthreads();
   }
   // prefix is now the k-th largest key; take every key above it and the first `need` ties.
@@ -213,7 +207,7 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const double* __restrict_
     uint64_t key = t < n ? key_at(t) : 0ull;
     int tie = (key != 0ull && key == prefix) ? 1 : 0;
     int total;
-    int before = block_excl_scan<THREADS>(tie, warp_sums, total);
+    int before = block_excl_scan<THREADS>(tie, sh.warp_sums, total);
     bool take = (key > prefix) || (tie && (taken_ties + before) < need);
     if (take) {
       int i = (int)(t / nkb), j = (int)(t % nkb);
@@ -221,6 +215,25 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const double* __restrict_
     }
     taken_ties += total;
   }
+}
+
+// One CTA per (batch, query head).  THREADS = kSelThreads for long rows; short rows run with fewer
+// threads, which makes the block-wide barriers of each pass cheaper.
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS) topk_kernel(const double* __restrict__ scores, int64_t n,
+                                                           int nkb, int topk_abs, int topk_bp, int mask_words,
+                                                           uint32_t* __restrict__ mask) {
+  __shared__ TopkShared sh;
+  __shared__ unsigned long long keys_sm[kSelSmemKeys];
+  const double* sc = scores + (int64_t)blockIdx.x * n;
+  int nqb = (int)(n / nkb);
+  uint32_t* mk = mask + (int64_t)blockIdx.x * nqb * mask_words;
+  // rows of up to kSelSmemKeys scores are read from global memory once and kept in shared memory
+  const bool in_smem = n <= kSelSmemKeys;
+  if (in_smem)
+    for (int64_t t = threadIdx.x; t < n; t += THREADS) keys_sm[t] = score_key(sc[t]);
+  auto key_at = [&](int64_t t) -> uint64_t { return in_smem ? keys_sm[t] : score_key(sc[t]); };
+  topk_row<THREADS>(key_at, n, nkb, topk_abs, topk_bp, mask_words, mk, sh);
 }
 
 constexpr int kListRowsPerCta = 8;
