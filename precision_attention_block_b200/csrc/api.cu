@@ -389,8 +389,8 @@ thrift_status thrift_decode_fwd(const void* q, const void* k, const void* v, con
   uint32_t* mask = reinterpret_cast<uint32_t*>(w + L.mask);
   if (decode_mode(cfg) == 0) {
     if (!q || !kbar) return THRIFT_ERR_INVALID_ARG;
-    st = decode_select_launch(q, kbar, *cfg, mask, reinterpret_cast<int32_t*>(w + L.counts),
-                              reinterpret_cast<int16_t*>(w + L.lists), nullptr, w + L.select, s);
+    // the attention reads only the mask: no counts and lists here
+    st = decode_select_launch(q, kbar, *cfg, mask, nullptr, nullptr, nullptr, w + L.select, s);
     if (st != THRIFT_OK) return st;
   }
   return decode_attn_common(q, k, v, k4, v4, mask, out, lse, cfg, ws, ws_bytes, s);

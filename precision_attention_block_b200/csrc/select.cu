@@ -273,12 +273,13 @@ __global__ void __launch_bounds__(32 * kListRowsPerCta) lists_kernel(const uint3
   if (lane == 0) counts[r] = total;
 }
 
-// Decode scores S^[b, h, j] = qbar[b, h] . kbar[b, h / G, j]: a CTA stages kDecScoreBlocks key-block
-// means of one KV head in shared memory; thread (hl, jj) scores block jj for query head hk*G + hl,
-// the sum in the order c = 0 .. d-1 with no fused multiply-add (the evaluation the prefill scores
-// use).
+// Decode scores S^[b, h, j] = qbar[b, h] . kbar[b, h / G, j]: a CTA forms the means of the Nq
+// query rows of the G heads of one KV head (exact FP16 sums in float64, divided by Nq) and stages
+// kDecScoreBlocks key-block means in shared memory; thread (hl, jj) scores block jj for query head
+// hk*G + hl, the sum in the order c = 0 .. d-1 with no fused multiply-add (the evaluation the
+// prefill scores use).
 constexpr int kDecScoreBlocks = 16;
-__global__ void decode_score_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar, int Hq,
+__global__ void decode_score_kernel(const __half* __restrict__ q, int Nq, const double* __restrict__ kbar, int Hq,
                                     int Hkv, int nkb, int d, double* __restrict__ scores) {
   __shared__ double ks[kDecScoreBlocks * 129];
   __shared__ double qs[16 * 128];
@@ -288,8 +289,13 @@ __global__ void decode_score_kernel(const double* __restrict__ qbar, const doubl
   const int nb = min(kDecScoreBlocks, nkb - j0);
   const double* kb = kbar + ((int64_t)grp * nkb + j0) * d;
   for (int e = threadIdx.x; e < nb * d; e += blockDim.x) ks[(e / d) * (d + 1) + e % d] = kb[e];
-  const double* qb = qbar + ((int64_t)b * Hq + (int64_t)hk * G) * d;
-  for (int e = threadIdx.x; e < G * d; e += blockDim.x) qs[e] = qb[e];
+  const __half* qb = q + ((int64_t)b * Hq + (int64_t)hk * G) * Nq * d;
+  for (int e = threadIdx.x; e < G * d; e += blockDim.x) {
+    const int hl = e / d, c = e % d;
+    double sum = 0.0;
+    for (int t = 0; t < Nq; ++t) sum = __dadd_rn(sum, (double)__half2float(qb[((int64_t)hl * Nq + t) * d + c]));
+    qs[e] = sum / (double)Nq;
+  }
   __syncthreads();
   const int jj = threadIdx.x % kDecScoreBlocks, hl = threadIdx.x / kDecScoreBlocks;
   if (jj >= nb || hl >= G) return;
@@ -381,15 +387,11 @@ thrift_status decode_select_launch(const void* q, const double* kbar, const thri
   const int nkb = c.Nk / c.block_k;
   const int mask_words = (nkb + 31) / 32;
   const size_t heads = (size_t)c.B * c.Hq;
-  double* qbar = reinterpret_cast<double*>(scratch);
   double* scores = scores_out ? scores_out
                               : reinterpret_cast<double*>(scratch + align256(heads * c.d * sizeof(double)));
-  int tpb = c.d >= 128 ? 128 : c.d;
-  block_mean_kernel<<<dim3(1, (unsigned)heads), tpb, 0, stream>>>(reinterpret_cast<const __half*>(q), c.Nq, c.d,
-                                                                  c.Nq, qbar);
   dim3 g((nkb + kDecScoreBlocks - 1) / kDecScoreBlocks, (unsigned)(c.B * c.Hkv));
-  decode_score_kernel<<<g, kDecScoreBlocks * (c.Hq / c.Hkv), 0, stream>>>(qbar, kbar, c.Hq, c.Hkv, nkb, c.d,
-                                                                          scores);
+  decode_score_kernel<<<g, kDecScoreBlocks * (c.Hq / c.Hkv), 0, stream>>>(
+      reinterpret_cast<const __half*>(q), c.Nq, kbar, c.Hq, c.Hkv, nkb, c.d, scores);
   if (cudaMemsetAsync(mask, 0, heads * mask_words * sizeof(uint32_t), stream) != cudaSuccess) return THRIFT_ERR_CUDA;
   if (nkb <= kSelSmemKeys)
     topk_kernel<256><<<(unsigned)heads, 256, 0, stream>>>(scores, (int64_t)nkb, nkb, c.topk_abs, c.topk_bp,
@@ -397,8 +399,9 @@ thrift_status decode_select_launch(const void* q, const double* kbar, const thri
   else
     topk_kernel<kSelThreads><<<(unsigned)heads, kSelThreads, 0, stream>>>(scores, (int64_t)nkb, nkb, c.topk_abs,
                                                                           c.topk_bp, mask_words, mask);
-  lists_kernel<<<(unsigned)((heads + kListRowsPerCta - 1) / kListRowsPerCta), 32 * kListRowsPerCta, 0, stream>>>(
-      mask, (int64_t)heads, nkb, mask_words, counts, lists);
+  if (counts && lists)
+    lists_kernel<<<(unsigned)((heads + kListRowsPerCta - 1) / kListRowsPerCta), 32 * kListRowsPerCta, 0, stream>>>(
+        mask, (int64_t)heads, nkb, mask_words, counts, lists);
   return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 

@@ -64,8 +64,8 @@ thrift_status decode_attn_launch(const DecodeArgs& a, cudaStream_t stream);
 thrift_status kv_means_launch(const void* k, int64_t outer, int32_t Nk, int32_t d, int32_t block_k, double* kbar,
                               cudaStream_t stream);
 
-// Decode selection: qbar [B*Hq, d] and scores [B*Hq, nkb] live in `scratch`
-// (decode_select_scratch_bytes) unless scores_out is given.
+// Decode selection: scores [B*Hq, nkb] live in `scratch` (decode_select_scratch_bytes) unless
+// scores_out is given; counts and lists are skipped when either is null.
 size_t decode_select_scratch_bytes(const thrift_decode_cfg& c);
 thrift_status decode_select_launch(const void* q, const double* kbar, const thrift_decode_cfg& c, uint32_t* mask,
                                    int32_t* counts, int16_t* lists, double* scores_out, uint8_t* scratch,
