@@ -400,3 +400,35 @@ def test_rows_of_p_sum_to_one():
     s = np.where(np.triu(np.ones((w.N, w.N), bool), 1), -np.inf, s)
     tot = np.exp(s - r["lse"][0][..., None].astype(np.float64)).sum(-1)
     assert np.abs(tot - 1).max() < 1e-6 * math.log(w.N) * 10
+
+
+def test_denominator_sums_unquantised_probabilities():
+    """Reading R1: the softmax denominator sums the unquantised exp(S - M), not the re-quantised
+    probabilities.  Keys alternate between two levels (c = 1 and c = 1/2, both exact in NVFP4),
+    so every 16-key group holds a block maximum (code 6, scale 448) and keys whose probability
+    r = exp(S_low - S_high) ~ 0.059 re-quantises to the E2M1 value 0.5 (dequantised 1/12): the
+    two denominators differ by ~2 %, far above the oracle's rounding.  The lse and output are
+    derived here from a float64 matmul of the dequantised inputs and the E2M1 grid."""
+    w = small(B=1, Hq=1, Hkv=1, N=64, d=32, causal=False, block_q=64, block_k=32, topk_bp=0)
+    q = np.ones((1, 1, 64, 32), np.float16)
+    c = np.where(np.arange(64) % 2 == 0, 1.0, 0.5).astype(np.float16)
+    k = np.repeat(c[None, None, :, None], 32, axis=3).astype(np.float16)
+    v = workloads.make_qkv(w)[2]
+    r = oracle.forward(w, q, k, v, want_f64=True)
+    qd = oracle.dequantize_nvfp4(r["q4"])[0, 0]
+    kd = oracle.dequantize_nvfp4(r["k4"])[0, 0]
+    vd = np.swapaxes(oracle.dequantize_nvfp4(r["v4"]), -1, -2)[0, 0]
+    tau = float(oracle.softmax_scale(w.d))
+    S = tau * (qd @ kd.T)                                    # [64 rows, 64 keys]
+    M = S.max(1, keepdims=True)                              # the same in both key blocks
+    ph = np.exp(S - M).astype(np.float32).astype(np.float64)  # P^ in FP32
+    assert np.all(np.isin(ph, [1.0, ph[0, 1]])) and 0.05 < ph[0, 1] < 0.07
+    y = 6.0 * ph                                             # P' / s_b with s_b = 448 in every group
+    pq = np.where(ph == 1.0, 6.0, 0.5) * 448 / 2688          # E2M1(6) = 6, E2M1(0.35) = 0.5
+    assert np.all(np.abs(y - np.where(ph == 1.0, 6.0, 0.5)) < 0.2)
+    lse = (M[:, 0] + np.log(ph.sum(1))).astype(np.float32)
+    lse_wrong = (M[:, 0] + np.log(pq.sum(1))).astype(np.float32)
+    assert np.abs(lse - lse_wrong).min() > 1e-2              # the two readings are far apart
+    assert np.abs(r["lse"][0, 0] - lse).max() <= 1e-6
+    out = (pq @ vd) / ph.sum(1, keepdims=True)
+    assert np.abs(r["out64"][0, 0] - out).max() <= 1e-12 * np.abs(out).max()
