@@ -131,7 +131,9 @@ thrift_status thrift_block_select_noalloc(const void* q, const void* k, const th
 /* Attention forward (ThriftAttention "Gemengd-Precisie Berekening & Samenvoeging").
  * q, k, v: device FP16 [B,Hq,N,d], [B,Hkv,N,d], [B,Hkv,N,d] (used for the FP16 pairs);
  * q4, k4 (group_axis 0) and v4 (group_axis 1): NVFP4 copies (used for the other pairs);
- * mask/counts/lists: the selection of thrift_block_select.
+ * mask: the selection bitmask of thrift_block_select.  Only the mask is read: the kernel builds
+ * each query tile's key-block list from it.  counts and lists are accepted for symmetry with
+ * thrift_block_select's outputs, are not read, and may be NULL.
  * out: device FP16 [B,Hq,N,d]; lse: device float [B,Hq,N] (natural log of the softmax
  * denominator of the tau-scaled scores; may be NULL).
  * topk_bp == 0 (or topk_abs == 0): uniform NVFP4; q, k, v, mask, counts, lists may be NULL.
@@ -144,6 +146,19 @@ thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v,
                               const int32_t* counts, const int16_t* lists, void* out,
                               float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes,
                               void* stream);
+
+/* Attn-QAT forward variant of thrift_attn_fwd (Attn-QAT technical summary, "2. Methodik: Attn-QAT",
+ * second principle: the forward pass also computes and stores a high-precision output O', used
+ * only for the backward pass's scalar term).  Reading: O' is the FP32 O / l of the same
+ * mixed-precision computation, written before the FP16 rounding of `out`; out is the FP16 round
+ * to nearest even of out_hp element by element.  out_hp: device float [B,Hq,N,d] (required);
+ * every other argument as thrift_attn_fwd (mask only; no counts or lists).  Same kernel, one
+ * more epilogue store per output row. */
+thrift_status thrift_attn_fwd_qat(const void* q, const void* k, const void* v,
+                                  const thrift_nvfp4* q4, const thrift_nvfp4* k4,
+                                  const thrift_nvfp4* v4, const uint32_t* mask, void* out,
+                                  float* out_hp, float* lse, const thrift_cfg* cfg, void* ws,
+                                  size_t ws_bytes, void* stream);
 
 /* Compute-matched sparse variant of thrift_attn_fwd (ThriftAttention compares against sparse
  * attention at a matched compute budget): only the selected pairs of `mask` run, in FP16 with the

@@ -206,6 +206,33 @@ def attn_fwd(q, k, v, q4: Optional[NVFP4Tensor], k4: Optional[NVFP4Tensor], v4: 
     return out, lse
 
 
+def attn_fwd_qat(q, k, v, q4: Optional[NVFP4Tensor], k4: Optional[NVFP4Tensor], v4: Optional[NVFP4Tensor],
+                 sel: Optional[Selection], cfg: Config, out: Optional[torch.Tensor] = None,
+                 out_hp: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                 ws: Optional[Workspace] = None):
+    """Attn-QAT forward variant (thrift_attn_fwd_qat): the FP16 output plus its FP32 copy O' before
+    the FP16 rounding.  Returns (out, out_hp, lse)."""
+    ref = q if q is not None else q4.codes
+    dev = ref.device
+    shape = (cfg.B, cfg.Hq, cfg.N, cfg.d)
+    if out is None:
+        out = torch.empty(shape, dtype=torch.float16, device=dev)
+    if out_hp is None:
+        out_hp = torch.empty(shape, dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((cfg.B, cfg.Hq, cfg.N), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = Workspace(256, dev)
+    c = cfg.c()
+    n4 = [None if t is None else t.c() for t in (q4, k4, v4)]
+    refs = [None if t is None else ctypes.byref(t) for t in n4]
+    check(load().thrift_attn_fwd_qat(_ptr(q), _ptr(k), _ptr(v), refs[0], refs[1], refs[2],
+                                     None if sel is None else _ptr(sel.mask), _ptr(out), _ptr(out_hp),
+                                     _ptr(lse), ctypes.byref(c), ws.ptr, ws.nbytes, _stream()),
+          "thrift_attn_fwd_qat")
+    return out, out_hp, lse
+
+
 def attn_fwd_sparse(q, k, v, sel: Selection, cfg: Config, out=None, lse=None, ws: Optional[Workspace] = None,
                     want_lse: bool = True):
     """Compute-matched sparse variant (thrift_attn_fwd_sparse): only the selected pairs, in FP16;
@@ -259,6 +286,17 @@ def attn_debug_dump(q, k, v, q4, k4, v4, sel, cfg: Config, entry: int, ws: Optio
                                         ctypes.byref(c), ws.ptr, ws.nbytes, _ptr(dbg), entry, _stream()),
           "thrift_debug_attn_dump")
     return out, lse, dbg
+
+
+def pipe_rates(device=None):
+    """Measured MUFU ex2 and FMA lanes per SM clock (thrift_debug_pipe_rates); synchronises."""
+    dev = torch.device("cuda") if device is None else device
+    L = load()
+    ws = Workspace(L.thrift_debug_pipe_rates_ws_bytes(), dev)
+    out = torch.zeros(2, dtype=torch.float64, device=dev)
+    check(L.thrift_debug_pipe_rates(ws.ptr, ws.nbytes, _ptr(out), _stream()), "thrift_debug_pipe_rates")
+    r = out.cpu().tolist()
+    return {"mufu_ex2": r[0], "fma": r[1]}
 
 
 def reset_device_status(ws: Workspace) -> None:

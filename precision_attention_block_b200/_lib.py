@@ -70,6 +70,8 @@ SIGNATURES = {
     "thrift_attn_fwd": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _nvp, _vp, _vp, _vp, _vp, _vp, _cfgp,
                                        _vp, _sz, _vp]),
     "thrift_attn_fwd_auto": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _cfgp, _vp, _sz, _vp]),
+    "thrift_attn_fwd_qat": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _nvp, _vp, _vp, _vp, _vp, _cfgp, _vp, _sz,
+                                           _vp]),
     "thrift_kv_block_means": (ctypes.c_int, [_vp, _i64, _i32, _i32, _i32, _vp, _vp]),
     "thrift_decode_workspace_bytes": (_sz, [_dcfgp]),
     "thrift_decode_select": (ctypes.c_int, [_vp, _vp, _dcfgp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -80,6 +82,9 @@ SIGNATURES = {
     "thrift_reset_device_status": (ctypes.c_int, [_vp, _vp]),
     "thrift_get_device_status": (ctypes.c_int, [_vp, _vp, ctypes.POINTER(_i32)]),
     "thrift_debug_wait_timeout": (ctypes.c_int, [_vp, _i64, _vp]),
+    "thrift_debug_ex2": (ctypes.c_int, [_vp, _vp, _i64, _i32, _vp]),
+    "thrift_debug_pipe_rates_ws_bytes": (_sz, []),
+    "thrift_debug_pipe_rates": (ctypes.c_int, [_vp, _sz, _vp, _vp]),
     "thrift_status_str": (ctypes.c_char_p, [ctypes.c_int]),
     "thrift_debug_attn_dump": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _nvp, _vp, _vp, _vp, _cfgp, _vp,
                                               _sz, _vp, _i32, _vp]),

@@ -13,8 +13,8 @@ namespace thrift {
 
 thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
                               const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
-                              void* out, float* lse, const thrift_cfg& c, int* status, float* dbg, int dbg_entry,
-                              cudaStream_t stream);
+                              void* out, float* out_hp, float* lse, const thrift_cfg& c, int* status, float* dbg,
+                              int dbg_entry, cudaStream_t stream);
 
 int num_sms() {
   static int cache[64] = {0};
@@ -259,8 +259,8 @@ thrift_status thrift_block_select_noalloc(const void* q, const void* k, const th
 
 static thrift_status attn_common(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
                                  const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, void* out,
-                                 float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes, float* dbg,
-                                 int dbg_entry, void* stream) {
+                                 float* out_hp, float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes,
+                                 float* dbg, int dbg_entry, void* stream) {
   thrift_status st = cfg_supported(cfg);
   if (st != THRIFT_OK) return st;
   if (!out) return THRIFT_ERR_INVALID_ARG;
@@ -269,7 +269,7 @@ static thrift_status attn_common(const void* q, const void* k, const void* v, co
   if (mode != 1 && (!q || !k || !v)) return THRIFT_ERR_INVALID_ARG;
   if (mode == 0 && !mask) return THRIFT_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, kWsHeader)) return THRIFT_ERR_WORKSPACE;
-  return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, lse, *cfg, status_ptr(ws), dbg, dbg_entry,
+  return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, out_hp, lse, *cfg, status_ptr(ws), dbg, dbg_entry,
                          static_cast<cudaStream_t>(stream));
 }
 
@@ -279,7 +279,15 @@ thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, const
                               const thrift_cfg* cfg, void* ws, size_t ws_bytes, void* stream) {
   (void)counts;
   (void)lists;
-  return attn_common(q, k, v, q4, k4, v4, mask, out, lse, cfg, ws, ws_bytes, nullptr, -1, stream);
+  return attn_common(q, k, v, q4, k4, v4, mask, out, nullptr, lse, cfg, ws, ws_bytes, nullptr, -1, stream);
+}
+
+thrift_status thrift_attn_fwd_qat(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
+                                  const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, void* out,
+                                  float* out_hp, float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  if (!out_hp) return THRIFT_ERR_INVALID_ARG;
+  return attn_common(q, k, v, q4, k4, v4, mask, out, out_hp, lse, cfg, ws, ws_bytes, nullptr, -1, stream);
 }
 
 thrift_status thrift_debug_attn_dump(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
@@ -287,7 +295,7 @@ thrift_status thrift_debug_attn_dump(const void* q, const void* k, const void* v
                                      void* out, float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes,
                                      float* dbg, int32_t dbg_entry, void* stream) {
   if (!dbg) return THRIFT_ERR_INVALID_ARG;
-  return attn_common(q, k, v, q4, k4, v4, mask, out, lse, cfg, ws, ws_bytes, dbg, dbg_entry, stream);
+  return attn_common(q, k, v, q4, k4, v4, mask, out, nullptr, lse, cfg, ws, ws_bytes, dbg, dbg_entry, stream);
 }
 
 thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, void* out, float* lse,
@@ -317,8 +325,8 @@ thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, 
                        nullptr, w + L.select, s);
     if (st != THRIFT_OK) return st;
   }
-  return attn_launch_dbg(q, k, v, &q4, &k4, &v4, mode == 0 ? mask : nullptr, mode, out, lse, c, status_ptr(ws),
-                         nullptr, -1, s);
+  return attn_launch_dbg(q, k, v, &q4, &k4, &v4, mode == 0 ? mask : nullptr, mode, out, nullptr, lse, c,
+                         status_ptr(ws), nullptr, -1, s);
 }
 
 thrift_status thrift_kv_block_means(const void* k, int64_t outer, int32_t Nk, int32_t d, int32_t block_k,
@@ -373,7 +381,7 @@ thrift_status thrift_attn_fwd_sparse(const void* q, const void* k, const void* v
   if (st != THRIFT_OK) return st;
   if (!q || !k || !v || !mask || !out) return THRIFT_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, kWsHeader)) return THRIFT_ERR_WORKSPACE;
-  return attn_launch_dbg(q, k, v, nullptr, nullptr, nullptr, mask, 3, out, lse, *cfg, status_ptr(ws), nullptr, -1,
+  return attn_launch_dbg(q, k, v, nullptr, nullptr, nullptr, mask, 3, out, nullptr, lse, *cfg, status_ptr(ws), nullptr, -1,
                          static_cast<cudaStream_t>(stream));
 }
 
@@ -418,6 +426,20 @@ thrift_status thrift_debug_wait_timeout(void* ws, int64_t limit_cycles, void* st
   if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 != 0) return THRIFT_ERR_WORKSPACE;
   if (limit_cycles <= 0 || limit_cycles > (int64_t)1 << 34) return THRIFT_ERR_INVALID_ARG;
   return wait_timeout_launch(status_ptr(ws), limit_cycles, static_cast<cudaStream_t>(stream));
+}
+
+thrift_status thrift_debug_ex2(const float* x, float* y, int64_t n, int32_t which, void* stream) {
+  if (!x || !y || n < 0 || (which != 0 && which != 1)) return THRIFT_ERR_INVALID_ARG;
+  if (n == 0) return THRIFT_OK;
+  return ex2_probe_launch(x, y, n, which, static_cast<cudaStream_t>(stream));
+}
+
+size_t thrift_debug_pipe_rates_ws_bytes(void) { return pipe_rates_ws_bytes(); }
+
+thrift_status thrift_debug_pipe_rates(void* ws, size_t ws_bytes, double* out, void* stream) {
+  if (!out) return THRIFT_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, pipe_rates_ws_bytes())) return THRIFT_ERR_WORKSPACE;
+  return pipe_rates_launch(ws, out, static_cast<cudaStream_t>(stream));
 }
 
 const char* thrift_status_str(thrift_status s) {

@@ -126,6 +126,7 @@ struct AttnParams {
   const float* k_ts;
   const float* v_ts;
   __half* out;
+  float* out_hp;  // optional FP32 copy of the output before its FP16 rounding (Attn-QAT's O')
   float* lse;
   int* status;
   float* dbg;  // optional dump of one entry (S, P bytes, PV) of tile 0 of the first unit of CTA 0
@@ -238,11 +239,12 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // 2^x on the FMA pipe: x = n + f with n = round(x) (by the 1.5 * 2^23 rounding constant) and f in
-// [-1/2, 1/2]; 2^f by a degree-5 polynomial (a relative-error minimax fit on [-1/2, 1/2]; relative
-// error below 2.2e-7 including FP32 rounding, about that of the MUFU ex2 approximation, so the
-// E2M1 code decisions of the two paths agree as often); n is added to the exponent field.  Inputs
-// are clamped at -125 so that the result stays a normal number (2^-125 is far below anything that
-// can change a sum or a code).
+// [-1/2, 1/2]; 2^f by a degree-5 polynomial whose coefficients are a relative-error minimax fit
+// on [-1/2, 1/2] (Lawson's iteratively reweighted least squares over Chebyshev-spaced nodes,
+// rounded to FP32; relative error below 2.2e-7 including FP32 rounding, about that of the MUFU
+// ex2 approximation, so the E2M1 code decisions of the two paths agree as often); n is added to
+// the exponent field.  Inputs are clamped at -125 so that the result stays a normal number
+// (2^-125 is far below anything that can change a sum or a code).
 __device__ __forceinline__ float ex2_poly1(float x) {
   x = fmaxf(x, -125.0f);
   const float t = x + 12582912.0f;
@@ -918,6 +920,12 @@ __global__ void __launch_bounds__(384, 1)
         v.w = pack_half2(O[8 * c + 6] * inv_l, O[8 * c + 7] * inv_l);
         dst[c] = v;
       }
+      if (p.out_hp) {
+        float4* dh = reinterpret_cast<float4*>(p.out_hp + orow * D + wg * DH);
+#pragma unroll
+        for (int c = 0; c < DH / 4; ++c)
+          dh[c] = make_float4(O[4 * c] * inv_l, O[4 * c + 1] * inv_l, O[4 * c + 2] * inv_l, O[4 * c + 3] * inv_l);
+      }
       if (p.lse && wg == 0) p.lse[orow] = (m_ref + __log2f(l_tot)) * kLn2;
     }
   }
@@ -1016,6 +1024,12 @@ thrift_status launch_t(const void* q, const void* k, const void* v, const thrift
   return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 
+// y = 2^x by the kernel's polynomial (which = 0) or the MUFU approximation (which = 1).
+__global__ void ex2_probe_kernel(const float* x, float* y, int64_t n, int which) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    y[i] = which == 0 ? ex2_poly1(x[i]) : ex2(x[i]);
+}
+
 __global__ void wait_timeout_kernel(int* status, long long limit) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -1033,8 +1047,8 @@ __global__ void wait_timeout_kernel(int* status, long long limit) {
 
 thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
                               const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
-                              void* out, float* lse, const thrift_cfg& c, int* status, float* dbg, int dbg_entry,
-                              cudaStream_t stream) {
+                              void* out, float* out_hp, float* lse, const thrift_cfg& c, int* status, float* dbg,
+                              int dbg_entry, cudaStream_t stream) {
   AttnParams prm;
   memset(&prm, 0, sizeof(prm));
   prm.mask = mask;
@@ -1047,6 +1061,7 @@ thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const
     prm.v_ts = v4->tensor_scale;
   }
   prm.out = reinterpret_cast<__half*>(out);
+  prm.out_hp = out_hp;
   prm.lse = lse;
   prm.status = status;
   prm.dbg = dbg;
@@ -1074,7 +1089,13 @@ thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const
 thrift_status attn_launch(const void* q, const void* k, const void* v, const thrift_nvfp4* q4, const thrift_nvfp4* k4,
                           const thrift_nvfp4* v4, const uint32_t* mask, int mode, void* out, float* lse,
                           const thrift_cfg& c, int* status, cudaStream_t stream) {
-  return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, lse, c, status, nullptr, -1, stream);
+  return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, nullptr, lse, c, status, nullptr, -1, stream);
+}
+
+thrift_status ex2_probe_launch(const float* x, float* y, int64_t n, int which, cudaStream_t stream) {
+  int grid = num_sms() * 4;
+  ex2_probe_kernel<<<grid, 256, 0, stream>>>(x, y, n, which);
+  return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 
 thrift_status wait_timeout_launch(int* status, long long limit, cudaStream_t stream) {

@@ -95,6 +95,9 @@ def test_null_and_workspace_errors(L):
     assert L.thrift_attn_fwd(None, None, None, ctypes.byref(nv), ctypes.byref(nv), ctypes.byref(nv), p, p, p, p,
                              None, ctypes.byref(cfg(topk_bp=10000)), p, 256, None) == 1
     assert L.thrift_status_str(4) == b"device wait timed out"
+    # the Attn-QAT variant needs its FP32 output
+    assert L.thrift_attn_fwd_qat(p, p, p, ctypes.byref(nv), ctypes.byref(nv), ctypes.byref(nv), p, p, None, None,
+                                 ctypes.byref(c), p, 256, None) == 1
 
 
 def dcfg(**kw):
