@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-units", type=int, default=8)
+    ap.add_argument("--quality-units", type=int, default=8, help="query blocks sampled for the quality context "
+                    "(0: skip it)")
     ap.add_argument("--sparse", action="store_true",
                     help="the compute-matched sparse variant: only the selected pairs, in FP16")
     return ap.parse_args()
@@ -69,6 +71,74 @@ def max_over_ranks(values, device, dist):
     if dist is not None:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return [float(x) for x in t.tolist()]
+
+
+def elementwise_bound(n_elem, d, block_k, mufu_lanes, fma_lanes, sm_count, sm_mhz, poly_fma_ops=8):
+    """Lower bound on the attention kernel's time from the elementwise work of reading R1 alone,
+    at the measured pipe rates (lanes per SM clock).  Per score element: one exponential, and on
+    the FMA pipe the exponent argument (1), the unquantised sum (1) and the merge of the key
+    block's PV product into the output (d / block_k: d output columns per row per block of
+    block_k keys).  An exponential runs on the MUFU unit or as a polynomial on the FMA pipe
+    (poly_fma_ops operations); the bound takes the split that balances the two pipes.  Ignores
+    instruction issue, the E2M1/E4M3 conversions and the group maxima (other pipes), so the real
+    floor is higher."""
+    e = float(n_elem)
+    f = e * (2.0 + d / block_k)
+    rm = mufu_lanes * sm_count
+    rf = fma_lanes * sm_count
+    x = (e * rf - f * rm) / (rf + poly_fma_ops * rm)
+    x = min(max(x, 0.0), e)
+    cycles = max((e - x) / rm, (f + poly_fma_ops * x) / rf)
+    return {"ms": cycles / (sm_mhz * 1e6) * 1e3, "exps_per_elem": 1.0, "fma_ops_per_elem": 2.0 + d / block_k,
+            "poly_share": x / e if e else 0.0, "elements": e, "mufu_lanes_per_clk_sm": mufu_lanes,
+            "fma_lanes_per_clk_sm": fma_lanes, "sm_mhz": sm_mhz, "poly_fma_ops": poly_fma_ops}
+
+
+def reference_rows(q, k, v, w, units, tau):
+    """float64 softmax attention (every pair exact, FP16 inputs widened) for the rows of the
+    listed (b, h, i) units: the quality context's full-precision reference.  [rows, d]."""
+    g = w.Hq // w.Hkv
+    out = []
+    for (b, h, i) in units:
+        rows = np.arange(i * w.block_q, (i + 1) * w.block_q)
+        kend = (i + 1) * w.block_q if w.causal else w.N
+        qq = q[b, h, rows].astype(np.float64)
+        kk = k[b, h // g, :kend].astype(np.float64)
+        vv = v[b, h // g, :kend].astype(np.float64)
+        s = tau * (qq @ kk.T)
+        if w.causal:
+            s = np.where(np.arange(kend)[None, :] > rows[:, None], -np.inf, s)
+        s = s - s.max(1, keepdims=True)
+        p = np.exp(s)
+        out.append((p @ vv) / p.sum(1, keepdims=True))
+    return np.concatenate(out)
+
+
+def gap_recovery(err_fp4, err_k):
+    """Share of the uniform-NVFP4 error removed by the FP16 budget: (err_FP4 - err_k) / err_FP4."""
+    return (err_fp4 - err_k) / err_fp4 if err_fp4 > 0 else 0.0
+
+
+def quality_block(pab, torch, w, q, k, v, gq, gk, gv, n_units):
+    """rel-L2 of the library's output against float64 softmax attention on a stratified sample of
+    query blocks, for uniform NVFP4 (k = 0), the workload's budget and every pair in FP16, and the
+    synthetic gap recovery.  Context only (the pages' quality figures come from model benchmarks)."""
+    units = workloads.sample_units(w, n_units)
+    tau = float(np.float32(1.0) / np.sqrt(np.float32(w.d)))
+    ref = reference_rows(q, k, v, w, units, tau)
+    rel = {}
+    for bp in (0, w.topk_bp, 10000):
+        wb = w.with_budget(bp)
+        cfg = pab.Config.from_workload(wb)
+        out, _ = pab.attn_fwd_auto(gq, gk, gv, cfg)
+        o = out.cpu().numpy().astype(np.float64)
+        rows = np.concatenate([o[b, h, i * w.block_q:(i + 1) * w.block_q] for (b, h, i) in units])
+        rel[bp] = float(np.linalg.norm(rows - ref) / np.linalg.norm(ref))
+    return {"reference": "float64 softmax attention of the FP16 inputs",
+            "sample": f"{len(units)} stratified (b, head, query block) units",
+            "rel_l2": {"k=0 (uniform NVFP4)": rel[0], f"k={w.topk_bp / 100:g}%": rel[w.topk_bp],
+                       "k=all (FP16)": rel[10000]},
+            "gap_recovery": gap_recovery(rel[0], rel[w.topk_bp])}
 
 
 def effective_flops(w) -> float:
@@ -348,6 +418,7 @@ def main():
         if evs:
             evs[2].record(stream)
 
+    rates = pab.pipe_rates(device) if not args.sparse else None
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -420,11 +491,22 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
             "device_status": status}
 
+    line["clocks"] = sampler.summary()
+    if rates is not None:
+        sm_mhz = line["clocks"].get("sm_mhz") or 1965.0
+        eb = elementwise_bound((F16 + F4) / (4.0 * w.d), w.d, w.block_k, rates["mufu_ex2"], rates["fma"],
+                               torch.cuda.get_device_properties(device).multi_processor_count, sm_mhz)
+        eb["attention_ms"] = attn_mean_ms
+        eb["frac"] = eb["ms"] / attn_mean_ms
+        eb["tensor_roofline_ms"] = t_roof * 1e3
+        eb["max_tensor_frac"] = min(1.0, t_roof * 1e3 / eb["ms"])
+        line["roofline"]["elementwise"] = eb
+    if rank == 0 and not args.sparse and args.quality_units > 0:
+        line["quality"] = quality_block(pab, torch, w, q, k, v, gq, gk, gv, args.quality_units)
     if not args.no_e2e and not args.sparse:
         line["e2e"] = e2e_measure(pab, torch, w, cfg, q, k, v, device, args, world, dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.sparse:
         line["cpu_baseline"] = cpu_baseline(w, q, k, v, args.cpu_units)
-    line["clocks"] = sampler.summary()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

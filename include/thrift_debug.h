@@ -26,6 +26,20 @@ thrift_status thrift_debug_attn_dump(const void* q, const void* k, const void* v
                                      size_t ws_bytes, float* dbg, int32_t dbg_entry,
                                      void* stream);
 
+/* The attention kernel's 2^x on device, for accuracy tests: y[i] = 2^x[i] for n elements by the
+ * FMA-pipe polynomial the softmax uses for part of its exponentials (which = 0) or by the MUFU
+ * approximation (which = 1).  x, y: device float arrays. */
+thrift_status thrift_debug_ex2(const float* x, float* y, int64_t n, int32_t which, void* stream);
+
+/* Measured pipe rates for the attention kernel's elementwise bound (bench and tests only):
+ * out (device double[2]) receives the lanes of ex2.approx.f32 (MUFU) and of fma.rn.f32 (FMA pipe)
+ * completed per SM clock, measured by one 512-thread CTA per SM running eight independent
+ * dependency chains per thread.  ws: 256-byte aligned device workspace of at least
+ * thrift_debug_pipe_rates_ws_bytes() bytes (its status header is left alone).  Three launches
+ * on `stream`; nothing is synchronised. */
+size_t thrift_debug_pipe_rates_ws_bytes(void);
+thrift_status thrift_debug_pipe_rates(void* ws, size_t ws_bytes, double* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libthrift.so")
 BUILD = os.path.join(HERE, "_build")
-SOURCES = ["quantize.cu", "select.cu", "attn.cu", "decode.cu", "api.cu"]
+SOURCES = ["quantize.cu", "select.cu", "attn.cu", "decode.cu", "probe.cu", "api.cu"]
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-I", INCLUDE]

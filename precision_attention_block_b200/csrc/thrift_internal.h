@@ -42,6 +42,10 @@ thrift_status attn_launch(const void* q, const void* k, const void* v, const thr
 
 thrift_status wait_timeout_launch(int* status, long long limit, cudaStream_t stream);
 
+thrift_status pipe_rates_launch(void* ws, double* out, cudaStream_t stream);
+thrift_status ex2_probe_launch(const float* x, float* y, int64_t n, int which, cudaStream_t stream);
+size_t pipe_rates_ws_bytes();
+
 // ---- decode
 struct DecodeArgs {
   const thrift_decode_cfg* cfg;
