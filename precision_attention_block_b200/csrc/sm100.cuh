@@ -58,7 +58,8 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity.  Gives up after `limit` clock cycles,
+// Bounded wait for the phase with the given parity (polls with a short sleep between tries).
+// Gives up after `limit` clock cycles,
 // records the timeout in the global status word (and, in the word after it, which wait gave up
 // first) and raises the CTA's abort flag (a shared flag:
 // once any wait of the CTA gives up, every later wait returns at once, so that all warps reach
@@ -69,7 +70,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   long long t0 = clock64();
   while (true) {
     if (*abort_flag) return false;
-    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+    // back off between polls: a waiting warp that polls continuously takes issue slots from the
+    // warps on its SM sub-partition that do the work it waits for
+    __nanosleep(60);
+    if (mbar_try_wait(bar, parity)) return true;
     if (clock64() - t0 > limit) {
       *abort_flag = 1;
       if (status) {
@@ -206,6 +210,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
         "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
         "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+// Load 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15])
       : "r"(taddr));
 }
 

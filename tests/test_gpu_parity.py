@@ -147,7 +147,9 @@ def compare_attention(out_g, lse_g, out_o, lse_o, w, units):
     # Both sides round their result to FP16 independently: where one FP16 step exceeds 1e-2
     # (|O| >= 16) the outputs may differ by that one step.
     bound = np.maximum(MAX_ABS, fp16_ulp(e))
-    print(f"parity: rel-L2 {rel:.3e} max-abs {mx:.3e} lse {lmx:.3e} worst err/bound {(err / bound).max():.3f}")
+    n_wide = int(np.count_nonzero(err > MAX_ABS))  # elements inside the bound only through its FP16 step
+    print(f"parity: rel-L2 {rel:.3e} max-abs {mx:.3e} lse {lmx:.3e} worst err/bound {(err / bound).max():.3f} "
+          f"elements past 1e-2 within one FP16 step: {n_wide} of {err.size}")
     assert rel <= REL_L2 and lmx <= LSE_ABS and np.all(err <= bound), (rel, mx, lmx)
     return rel, mx, lmx
 
@@ -199,13 +201,18 @@ def test_attn_diffusion_sampled(pab, bp):
     run_pair(pab, "diffusion", bp, n_units=12)
 
 
+# 64 stratified units plus the first and the last query block (workloads.sample_units draws those
+# two first)
+N_SAMPLED = 66
+
+
 def test_attn_prefill32k_sampled(pab):
-    run_pair(pab, "prefill32k", None, n_units=24)
+    run_pair(pab, "prefill32k", None, n_units=N_SAMPLED)
 
 
 @pytest.mark.slow
 def test_attn_long131k_sampled(pab):
-    run_pair(pab, "long131k", None, n_units=10)
+    run_pair(pab, "long131k", None, n_units=N_SAMPLED)
 
 
 def test_device_wait_timeout_is_reported(pab):

@@ -37,15 +37,18 @@ def _outputs(pab, cfg, device):
         torch.full((cfg.B, cfg.Hq, cfg.n_qb, cfg.n_kb), np.nan, dtype=torch.float64, device=device))
 
 
-def _noalloc(pab, q, k, cfg, sel):
+def _noalloc(pab, q, k, cfg, sel, want_scores=True):
     c = cfg.c()
     p = lambda t: ctypes.c_void_p(t.data_ptr())
     return pab.load().thrift_block_select_noalloc(p(q), p(k), ctypes.byref(c), p(sel.mask), p(sel.counts),
-                                                  p(sel.lists), p(sel.scores), pab._stream())
+                                                  p(sel.lists), p(sel.scores) if want_scores else None,
+                                                  pab._stream())
 
 
+@pytest.mark.parametrize("want_scores", [True, False])
 @pytest.mark.parametrize("name", ["n4k", "tiny"])
-def test_noalloc_select_matches_workspace_select(pab, name):
+def test_noalloc_select_matches_workspace_select(pab, name, want_scores):
+    """With want_scores False the score matrix goes to the library's own array (the usual use)."""
     w = workloads.WORKLOADS[name]
     q, k, _ = workloads.make_qkv(w)
     dev = torch.device("cuda")
@@ -55,11 +58,14 @@ def test_noalloc_select_matches_workspace_select(pab, name):
     torch.cuda.synchronize()
     for call in range(2):
         got = _outputs(pab, cfg, dev)
-        assert _noalloc(pab, gq, gk, cfg, got) == 0
+        assert _noalloc(pab, gq, gk, cfg, got, want_scores) == 0
         torch.cuda.synchronize()
         assert torch.equal(got.mask, ref.mask), f"call {call}: mask"
         assert torch.equal(got.counts, ref.counts), f"call {call}: counts"
         assert torch.equal(got.lists, ref.lists), f"call {call}: lists"
+        if not want_scores:
+            assert torch.isnan(got.scores).all()  # untouched
+            continue
         assert torch.equal(torch.isfinite(got.scores), torch.isfinite(ref.scores))
         fin = torch.isfinite(ref.scores)
         assert torch.equal(got.scores[fin], ref.scores[fin]), f"call {call}: scores"
