@@ -66,8 +66,9 @@ def lib():
         L.orc_double_to_half_array.argtypes = [_f64p, _i64, _u16p]
         L.orc_quantize_nvfp4.restype = ctypes.c_float
         L.orc_quantize_nvfp4.argtypes = [_u16p, _i64, _i32, _i32, _i32, _u8p, _u8p]
+        L.orc_quantize_nvfp4_scaled.argtypes = [_u16p, _i64, _i32, _i32, _i32, ctypes.c_float, _u8p, _u8p]
         L.orc_block_scores.argtypes = [_u16p, _u16p] + [_int] * 8 + [_f64p]
-        L.orc_block_scores_qk.argtypes = [_u16p, _u16p] + [_int] * 9 + [_f64p]
+        L.orc_block_scores_qk.argtypes = [_u16p, _u16p] + [_int] * 10 + [_f64p]
         L.orc_topk_count.restype = _i64
         L.orc_topk_count.argtypes = [_i64, _int, _int]
         L.orc_select.argtypes = [_f64p, _i64, _i64, _int, _int, _u8p, _f64p, _i64p]
@@ -82,7 +83,7 @@ def lib():
              ctypes.c_void_p, _u16p, _f32p, ctypes.c_void_p, _int])
         L.orc_attn_qk.argtypes = (
             [_u16p, _u16p, _u16p, _u8p, _u8p, ctypes.c_float, _u8p, _u8p, ctypes.c_float,
-             _u8p, _u8p, ctypes.c_float, _u8p] + [_int] * 9 + [ctypes.c_float, _int, _i32p, _int, _int,
+             _u8p, _u8p, ctypes.c_float, _u8p] + [_int] * 9 + [ctypes.c_float, _int, _int, _i32p, _int, _int,
              ctypes.c_void_p, _u16p, _f32p, ctypes.c_void_p, _int])
         L.orc_tile_scores.argtypes = (
             [_u16p, _u16p, _u8p, _u8p, ctypes.c_float, _u8p, _u8p, ctypes.c_float] + [_int] * 8
@@ -151,10 +152,12 @@ class NVFP4:
         self.group_axis = group_axis
 
 
-def quantize_nvfp4(x: np.ndarray, group_axis: int) -> NVFP4:
+def quantize_nvfp4(x: np.ndarray, group_axis: int, tensor_scale=None) -> NVFP4:
     """NVFP4 quantisation of x [.., N, d] (ThriftAttention "FP4-pad": NVFP4 microscaling,
     E2M1 values, one E4M3 scale per 16 elements, one FP32 tensor scale).
-    group_axis 0: groups along d, codes [.., N, d/2]; 1: groups along N, codes [.., d, N/2]."""
+    group_axis 0: groups along d, codes [.., N, d/2]; 1: groups along N, codes [.., d, N/2].
+    tensor_scale: a given FP32 tensor scale (reading R-append: a cache encodes with the scale it
+    was built with); None: the tensor's own amax / 2688."""
     *lead, N, d = x.shape
     outer = int(np.prod(lead)) if lead else 1
     if group_axis == 0:
@@ -163,8 +166,13 @@ def quantize_nvfp4(x: np.ndarray, group_axis: int) -> NVFP4:
     else:
         codes = np.empty((*lead, d, N // 2), np.uint8)
         scales = np.empty((*lead, d, N // 16), np.uint8)
-    st = lib().orc_quantize_nvfp4(_u16(x).reshape(-1), outer, N, d, group_axis,
-                                  codes.reshape(-1), scales.reshape(-1))
+    if tensor_scale is None:
+        st = lib().orc_quantize_nvfp4(_u16(x).reshape(-1), outer, N, d, group_axis,
+                                      codes.reshape(-1), scales.reshape(-1))
+    else:
+        st = np.float32(tensor_scale)
+        lib().orc_quantize_nvfp4_scaled(_u16(x).reshape(-1), outer, N, d, group_axis, st,
+                                        codes.reshape(-1), scales.reshape(-1))
     return NVFP4(codes, scales, st, group_axis)
 
 
@@ -287,7 +295,7 @@ def attn_sparse(q, k, v, sel, w, tau=None, units=None, want_f64=False, threads=N
     lib().orc_attn_qk(_u16(q).reshape(-1), _u16(k).reshape(-1), _u16(v).reshape(-1),
                       z8, z8, np.float32(1), z8, z8, np.float32(1), z8, z8, np.float32(1),
                       np.ascontiguousarray(sel, np.uint8).reshape(-1),
-                      B, Hq, k.shape[1], N, N, d, w.block_q, w.block_k, int(w.causal), np.float32(tau), 1,
+                      B, Hq, k.shape[1], N, N, d, w.block_q, w.block_k, int(w.causal), np.float32(tau), 1, N,
                       u, len(units), 0, None, out.reshape(-1), lse.reshape(-1),
                       None if out64 is None else out64.ctypes.data, int(threads))
     return out.view(np.float16), lse, out64
@@ -311,26 +319,30 @@ def forward(w, q, k, v, units=None, want_f64=False, threads=None):
 
 # ------------------------------------------------------------------ decode
 
-def decode_block_scores(q: np.ndarray, k: np.ndarray, block_k: int, causal: bool) -> np.ndarray:
+def decode_block_scores(q: np.ndarray, k: np.ndarray, block_k: int, causal: bool, n_valid=None) -> np.ndarray:
     """Decode selection scores (reading R-decode): the Nq query rows of each (batch, query head)
     form one query block; S^_j = qbar . kbar_j over the key blocks of the cache, float64
-    [B, Hq, 1, Nk/block_k]."""
+    [B, Hq, 1, Nk/block_k].  n_valid: the cache's valid length (reading R-append; default Nk):
+    blocks at or past it are -inf and a partly filled block averages the keys it holds."""
     B, Hq, Nq, d = q.shape
     Hkv, Nk = k.shape[1], k.shape[2]
+    nv = Nk if n_valid is None else int(n_valid)
     out = np.empty((B, Hq, 1, Nk // block_k), np.float64)
     lib().orc_block_scores_qk(_u16(q).reshape(-1), _u16(k).reshape(-1), B, Hq, Hkv, Nq, Nk, d, Nq,
-                              block_k, int(causal), out.reshape(-1))
+                              block_k, int(causal), nv, out.reshape(-1))
     return out
 
 
 def decode_attn(q, k, v, q4: NVFP4, k4: NVFP4, v4: NVFP4, sel, block_k: int, causal: bool, tau=None,
-                want_f64=False, threads=None, sparse=False):
+                want_f64=False, threads=None, sparse=False, n_valid=None):
     """Decode attention (reading R-decode): the Nq rows of q [B,Hq,Nq,d] are the newest
     positions of the cache k, v [B,Hkv,Nk,d]; sel [B,Hq,1,Nk/block_k] marks the FP16 key blocks.
     The same mixed-precision computation as `attn` (sparse: only the selected blocks, reading
-    R-sparse).  Returns (out fp16 [B,Hq,Nq,d], lse f32 [B,Hq,Nq], out64 or None)."""
+    R-sparse).  n_valid: the cache's valid length (default Nk): keys at or past it are masked.
+    Returns (out fp16 [B,Hq,Nq,d], lse f32 [B,Hq,Nq], out64 or None)."""
     B, Hq, Nq, d = q.shape
     Hkv, Nk = k.shape[1], k.shape[2]
+    nv = Nk if n_valid is None else int(n_valid)
     if tau is None:
         tau = softmax_scale(d)
     units = [(b, h, 0) for b in range(B) for h in range(Hq)]
@@ -345,23 +357,24 @@ def decode_attn(q, k, v, q4: NVFP4, k4: NVFP4, v4: NVFP4, sel, block_k: int, cau
                       k4.codes.reshape(-1), k4.scales.reshape(-1), k4.tensor_scale,
                       v4.codes.reshape(-1), v4.scales.reshape(-1), v4.tensor_scale,
                       np.ascontiguousarray(sel, np.uint8).reshape(-1),
-                      B, Hq, Hkv, Nq, Nk, d, Nq, block_k, int(causal), np.float32(tau), int(sparse),
+                      B, Hq, Hkv, Nq, Nk, d, Nq, block_k, int(causal), np.float32(tau), int(sparse), nv,
                       u, len(units), 0, None, out.reshape(-1), lse.reshape(-1),
                       None if out64 is None else out64.ctypes.data, int(threads))
     return out.view(np.float16), lse, out64
 
 
-def decode_forward(w, q, k, v, k4=None, v4=None, want_f64=False, threads=None):
+def decode_forward(w, q, k, v, k4=None, v4=None, want_f64=False, threads=None, n_valid=None):
     """One decode step: quantise the query rows, score and select key blocks, attend.
-    k4, v4: the cache's NVFP4 copies (computed here when None).  Returns a dict."""
+    k4, v4: the cache's NVFP4 copies (computed here when None).  n_valid: the cache's valid
+    length (default: all of k).  Returns a dict."""
     q4 = quantize_nvfp4(q, 0)
     if k4 is None:
         k4 = quantize_nvfp4(k, 0)
     if v4 is None:
         v4 = quantize_nvfp4(v, 1)
-    scores = decode_block_scores(q, k, w.block_k, w.causal)
+    scores = decode_block_scores(q, k, w.block_k, w.causal, n_valid)
     sel, kth, kc = select(scores, w)
     out, lse, out64 = decode_attn(q, k, v, q4, k4, v4, sel, w.block_k, w.causal, want_f64=want_f64,
-                                  threads=threads)
+                                  threads=threads, n_valid=n_valid)
     return dict(q4=q4, k4=k4, v4=v4, scores=scores, sel=sel, kth=kth, k=kc, out=out, lse=lse,
                 out64=out64)

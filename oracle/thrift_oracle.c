@@ -159,19 +159,14 @@ static void quantize_group(const float* xs, float s_t, uint8_t* codes16, uint8_t
   for (int t = 0; t < 16; ++t) codes16[t] = eff == 0.0f ? 0 : orc_e2m1_encode(xs[t] / eff);
 }
 
-/* NVFP4 quantisation of an FP16 tensor viewed as [outer, N, d].
+/* NVFP4 quantisation of an FP16 tensor viewed as [outer, N, d] with a given FP32 tensor scale s_t
+ * (reading R-append: a double-cached KV cache keeps the tensor scales it was built with and
+ * encodes appended tokens with them; a value above the build-time amax saturates).
  *   group_axis 0: groups of 16 along d;  codes [outer, N, d/2], scales [outer, N, d/16].
  *   group_axis 1: groups of 16 along N;  codes [outer, d, N/2], scales [outer, d, N/16].
- * Element 2t of a code row is the low nibble of byte t.  Returns the FP32 tensor scale. */
-float orc_quantize_nvfp4(const uint16_t* x, int64_t outer, int32_t N, int32_t d, int32_t group_axis,
-                         uint8_t* codes, uint8_t* scales) {
-  int64_t total = outer * (int64_t)N * d;
-  float amax = 0.0f;
-  for (int64_t i = 0; i < total; ++i) {
-    float a = (float)fabs(orc_half_to_double(x[i]));
-    if (a > amax) amax = a;
-  }
-  float s_t = amax > 0.0f ? amax / 2688.0f : 1.0f;
+ * Element 2t of a code row is the low nibble of byte t. */
+void orc_quantize_nvfp4_scaled(const uint16_t* x, int64_t outer, int32_t N, int32_t d, int32_t group_axis,
+                               float s_t, uint8_t* codes, uint8_t* scales) {
   float xs[16];
   uint8_t c16[16];
   if (group_axis == 0) {
@@ -195,6 +190,20 @@ float orc_quantize_nvfp4(const uint16_t* x, int64_t outer, int32_t N, int32_t d,
                 (uint8_t)((c16[t] & 15) | ((c16[t + 1] & 15) << 4));
         }
   }
+}
+
+/* NVFP4 quantisation with the tensor's own scale s_t = amax|x| / 2688 (1 for an all-zero
+ * tensor).  Returns s_t. */
+float orc_quantize_nvfp4(const uint16_t* x, int64_t outer, int32_t N, int32_t d, int32_t group_axis,
+                         uint8_t* codes, uint8_t* scales) {
+  int64_t total = outer * (int64_t)N * d;
+  float amax = 0.0f;
+  for (int64_t i = 0; i < total; ++i) {
+    float a = (float)fabs(orc_half_to_double(x[i]));
+    if (a > amax) amax = a;
+  }
+  float s_t = amax > 0.0f ? amax / 2688.0f : 1.0f;
+  orc_quantize_nvfp4_scaled(x, outer, N, d, group_axis, s_t, codes, scales);
   return s_t;
 }
 
@@ -214,32 +223,41 @@ double orc_nvfp4_elem(const uint8_t* codes, const uint8_t* scales, int64_t row, 
 /* ---------------------------------------------------------- block select */
 
 /* Pair (query block i, key block j) is valid when some key of block j is visible to some
- * row of block i; with the causal offset qoff, query row r sits at position qoff + r. */
-static inline int pair_valid(int causal, int64_t qoff, int i, int j, int bq, int bk) {
+ * row of block i; with the causal offset qoff, query row r sits at position qoff + r.  Keys at
+ * or past nvalid (the cache's valid length, reading R-append) are never visible. */
+static inline int pair_valid(int causal, int64_t qoff, int i, int j, int bq, int bk, int64_t nvalid) {
+  if ((int64_t)j * bk >= nvalid) return 0;
   return !causal || (int64_t)j * bk <= qoff + (int64_t)(i + 1) * bq - 1;
 }
 
-int orc_pair_valid(int causal, int i, int j, int bq, int bk) { return pair_valid(causal, 0, i, j, bq, bk); }
+int orc_pair_valid(int causal, int i, int j, int bq, int bk) {
+  return pair_valid(causal, 0, i, j, bq, bk, (int64_t)1 << 62);
+}
 
 /* S^_ij = qbar_i . kbar_j per (batch, query head); -inf for invalid pairs.
- * q [B,Hq,Nq,d], k [B,Hkv,Nk,d] FP16 (query row r at position Nk - Nq + r);
- * scores [B,Hq,Nq/bq,Nk/bk] float64. */
+ * q [B,Hq,Nq,d], k [B,Hkv,Nk,d] FP16, of which the first nvalid keys are the cache's valid
+ * length (query row r at position nvalid - Nq + r); scores [B,Hq,Nq/bq,Nk/bk] float64.  A key
+ * block's mean is over its keys below nvalid (reading R-append: a partly filled last block
+ * averages the keys it holds). */
 void orc_block_scores_qk(const uint16_t* q, const uint16_t* k, int B, int Hq, int Hkv, int Nq, int Nk, int d,
-                         int bq, int bk, int causal, double* scores) {
+                         int bq, int bk, int causal, int nvalid, double* scores) {
   int nqb = Nq / bq, nkb = Nk / bk, grp = Hq / Hkv;
-  int64_t qoff = (int64_t)Nk - Nq;
+  int64_t qoff = (int64_t)nvalid - Nq;
   double* kbar = (double*)malloc(sizeof(double) * (size_t)nkb * d);
   double* qbar = (double*)malloc(sizeof(double) * (size_t)d);
   for (int b = 0; b < B; ++b)
     for (int h = 0; h < Hq; ++h) {
       const uint16_t* kh = k + ((int64_t)b * Hkv + h / grp) * (int64_t)Nk * d;
       const uint16_t* qh = q + ((int64_t)b * Hq + h) * (int64_t)Nq * d;
-      for (int j = 0; j < nkb; ++j)
+      for (int j = 0; j < nkb; ++j) {
+        int64_t cnt = (int64_t)nvalid - (int64_t)j * bk;
+        if (cnt > bk) cnt = bk;
         for (int c = 0; c < d; ++c) {
           double s = 0.0;
-          for (int t = 0; t < bk; ++t) s += orc_half_to_double(kh[((int64_t)j * bk + t) * d + c]);
-          kbar[(int64_t)j * d + c] = s / bk;
+          for (int t = 0; t < cnt; ++t) s += orc_half_to_double(kh[((int64_t)j * bk + t) * d + c]);
+          kbar[(int64_t)j * d + c] = cnt > 0 ? s / (double)cnt : 0.0;
         }
+      }
       for (int i = 0; i < nqb; ++i) {
         for (int c = 0; c < d; ++c) {
           double s = 0.0;
@@ -248,7 +266,7 @@ void orc_block_scores_qk(const uint16_t* q, const uint16_t* k, int B, int Hq, in
         }
         double* row = scores + (((int64_t)b * Hq + h) * nqb + i) * nkb;
         for (int j = 0; j < nkb; ++j) {
-          if (!pair_valid(causal, qoff, i, j, bq, bk)) { row[j] = -INFINITY; continue; }
+          if (!pair_valid(causal, qoff, i, j, bq, bk, nvalid)) { row[j] = -INFINITY; continue; }
           double s = 0.0;
           for (int c = 0; c < d; ++c) s += qbar[c] * kbar[(int64_t)j * d + c];
           row[j] = s;
@@ -262,7 +280,7 @@ void orc_block_scores_qk(const uint16_t* q, const uint16_t* k, int B, int Hq, in
 /* Prefill form: q and k both [.., N, d]. */
 void orc_block_scores(const uint16_t* q, const uint16_t* k, int B, int Hq, int Hkv, int N, int d, int bq,
                       int bk, int causal, double* scores) {
-  orc_block_scores_qk(q, k, B, Hq, Hkv, N, N, d, bq, bk, causal, scores);
+  orc_block_scores_qk(q, k, B, Hq, Hkv, N, N, d, bq, bk, causal, N, scores);
 }
 
 int64_t orc_topk_count(int64_t n_valid, int topk_abs, int topk_bp) {
@@ -309,10 +327,11 @@ typedef struct {
   int B, Hq, Hkv, Nq, Nk, d, bq, bk, causal;
   double tau;
   int sparse; /* 1: only the selected (FP16) pairs, the others dropped (R-sparse) */
+  int nvalid; /* valid keys of the cache (the first nvalid positions of Nk); Nk for prefill */
 } attn_problem;
 
 /* position of query row 0 among the keys (bottom-right causal alignment) */
-static inline int64_t qoff_of(const attn_problem* P) { return (int64_t)P->Nk - P->Nq; }
+static inline int64_t qoff_of(const attn_problem* P) { return (int64_t)P->nvalid - P->Nq; }
 
 static int pair_is_fp16(const attn_problem* P, int b, int h, int i, int j) {
   int nqb = P->Nq / P->bq, nkb = P->Nk / P->bk;
@@ -340,7 +359,7 @@ static void block_scores(const attn_problem* P, int b, int h, int i, int j, int 
     int64_t row = qoff_of(P) + (int64_t)i * P->bq + r;
     for (int t = 0; t < P->bk; ++t) {
       int64_t key = (int64_t)j * P->bk + t;
-      if (P->causal && key > row) { S[r * ldS + t] = -INFINITY; continue; }
+      if ((P->causal && key > row) || key >= P->nvalid) { S[r * ldS + t] = -INFINITY; continue; }
       double s = 0.0;
       for (int c = 0; c < d; ++c) s += qd[c] * kd[t * d + c];
       S[r * ldS + t] = s * mult;
@@ -419,7 +438,7 @@ static void attn_unit(const attn_problem* P, int b, int h, int i, int online, co
   for (int r = 0; r < bq; ++r) m[r] = -INFINITY;
 
   for (int j = 0; j < nkb; ++j) {
-    if (!pair_valid(P->causal, qoff, i, j, bq, bk) || (P->sparse && !pair_is_fp16(P, b, h, i, j))) {
+    if (!pair_valid(P->causal, qoff, i, j, bq, bk, P->nvalid) || (P->sparse && !pair_is_fp16(P, b, h, i, j))) {
       for (int r = 0; r < bq; ++r)
         for (int t = 0; t < bk; ++t) S[r * ldS + (int64_t)j * bk + t] = -INFINITY;
       continue;
@@ -432,7 +451,7 @@ static void attn_unit(const attn_problem* P, int b, int h, int i, int online, co
 
   for (int jj = 0; jj < nkb; ++jj) {
     int j = order ? order[jj] : jj;
-    if (!pair_valid(P->causal, qoff, i, j, bq, bk)) continue;
+    if (!pair_valid(P->causal, qoff, i, j, bq, bk, P->nvalid)) continue;
     if (P->sparse && !pair_is_fp16(P, b, h, i, j)) continue;
     int fp16 = pair_is_fp16(P, b, h, i, j);
     block_values(P, b, h, j, fp16, vd);
@@ -496,17 +515,18 @@ static void* attn_worker(void* arg) {
 }
 
 /* Attention forward over the listed (b, h, i) units.  Inputs: FP16 q [B,Hq,Nq,d], k, v
- * [B,Hkv,Nk,d] (query row r at position Nk - Nq + r); NVFP4 codes/scales of q, k (grouped
+ * [B,Hkv,Nk,d] whose first nvalid keys are valid (query row r at position nvalid - Nq + r;
+ * keys at or past nvalid are masked); NVFP4 codes/scales of q, k (grouped
  * along d) and v (grouped along tokens, [B,Hkv,d,Nk/2]) with their tensor scales;
  * sel [B,Hq,Nq/bq,Nk/bk] (1 = FP16 pair).  Writes O (FP16 [B,Hq,Nq,d], and float64 when
  * out64 != NULL) and lse (natural log, tau-scaled scores) for the rows of the listed units. */
 void orc_attn_qk(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint8_t* q4c, const uint8_t* q4s,
                  float q4t, const uint8_t* k4c, const uint8_t* k4s, float k4t, const uint8_t* v4c,
                  const uint8_t* v4s, float v4t, const uint8_t* sel, int B, int Hq, int Hkv, int Nq, int Nk, int d,
-                 int bq, int bk, int causal, float tau, int sparse, const int32_t* units, int n_units, int online,
-                 const int32_t* order, uint16_t* out, float* lse, double* out64, int n_threads) {
+                 int bq, int bk, int causal, float tau, int sparse, int nvalid, const int32_t* units, int n_units,
+                 int online, const int32_t* order, uint16_t* out, float* lse, double* out64, int n_threads) {
   attn_problem P = {q, k, v, q4c, q4s, k4c, k4s, v4c, v4s, q4t, k4t, v4t, sel,
-                    B, Hq, Hkv, Nq, Nk, d, bq, bk, causal, (double)tau, sparse};
+                    B, Hq, Hkv, Nq, Nk, d, bq, bk, causal, (double)tau, sparse, nvalid};
   attn_job J;
   J.P = &P; J.units = units; J.n_units = n_units; J.online = online; J.order = order;
   J.out = out; J.lse = lse; J.out64 = out64; J.next = 0;
@@ -526,7 +546,7 @@ void orc_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uin
               int bk, int causal, float tau, const int32_t* units, int n_units, int online,
               const int32_t* order, uint16_t* out, float* lse, double* out64, int n_threads) {
   orc_attn_qk(q, k, v, q4c, q4s, q4t, k4c, k4s, k4t, v4c, v4s, v4t, sel, B, Hq, Hkv, N, N, d, bq, bk, causal, tau,
-              0, units, n_units, online, order, out, lse, out64, n_threads);
+              0, N, units, n_units, online, order, out, lse, out64, n_threads);
 }
 
 /* The tau-scaled scores of one (b, h, query block i, key block j) tile, [bq, bk] float64,
@@ -535,7 +555,7 @@ void orc_tile_scores(const uint16_t* q, const uint16_t* k, const uint8_t* q4c, c
                      const uint8_t* k4c, const uint8_t* k4s, float k4t, int B, int Hq, int Hkv, int N, int d,
                      int bq, int bk, int causal, float tau, int b, int h, int i, int j, int fp16, double* S) {
   attn_problem P = {q, k, NULL, q4c, q4s, k4c, k4s, NULL, NULL, q4t, k4t, 0.0f, NULL,
-                    B, Hq, Hkv, N, N, d, bq, bk, causal, (double)tau, 0};
+                    B, Hq, Hkv, N, N, d, bq, bk, causal, (double)tau, 0, N};
   double* qd = (double*)malloc(sizeof(double) * (size_t)d);
   double* kd = (double*)malloc(sizeof(double) * (size_t)bk * d);
   block_scores(&P, b, h, i, j, fp16, qd, kd, S, bk);

@@ -147,6 +147,10 @@ WORKLOADS = {
     # same distribution and blocking as the 32K prefill at half the length: a profiling size
     "prefill16k": Workload("prefill16k", 5, 1, 32, 8, 16384, 128, True, 128, 64, -1, 500,
                            "heavy_bias"),
+    # the 32K prefill with "inputs as in config 1" read 1-based (the 4K workload's plain N(0,1)
+    # inputs, no heavy tail or key bias) instead of 0-based: an extra, labelled row
+    "prefill32k_plain": Workload("prefill32k_plain", 9, 1, 32, 8, 32768, 128, True, 128, 64, -1, 500,
+                                 "normal"),
     "long131k": Workload("long131k", 3, 1, 32, 8, 131072, 128, True, 128, 128, -1, 200,
                          "student_t"),
     "diffusion": Workload("diffusion", 4, 2, 24, 24, 16384, 64, False, 128, 64, -1, 500,
