@@ -203,7 +203,7 @@ thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, 
 typedef struct {
   int32_t B, Hq, Hkv;  /* batch, query heads, key/value heads (Hq % Hkv == 0) */
   int32_t Nq;          /* query rows per head in this step, 1 <= Nq, (Hq/Hkv) * Nq <= 16 */
-  int32_t Nk;          /* cache length, Nq <= Nk, a multiple of 128 and of block_k */
+  int32_t Nk;          /* cache capacity (the layout's key count), a multiple of 128 and of block_k */
   int32_t d;           /* head dim, 64 or 128 */
   int32_t causal;      /* 0 or 1 (bottom-right aligned, see above) */
   int32_t block_k;     /* key block size, 64 or 128 */
@@ -211,6 +211,12 @@ typedef struct {
   int32_t topk_bp;     /* budget in basis points of the nKb = Nk/block_k key blocks
                           (0 = every block NVFP4, 10000 = every block FP16) */
   float softmax_scale; /* tau; 0 selects 1/sqrt(d) rounded to FP32 */
+  int32_t n_valid;     /* keys held by the cache, Nq <= n_valid <= Nk (any value); 0 means Nk.
+                          Query row r is at position n_valid - Nq + r; keys at or past n_valid
+                          are masked, key blocks starting at or past it are skipped and left
+                          out of the budget (nKb above counts the blocks below n_valid).  The
+                          cache beyond n_valid must hold finite values (thrift_kv_append keeps
+                          it zero). */
 } thrift_decode_cfg;
 
 /* Block means of the cache's keys: kbar [outer, Nk/block_k, d] float64, the exact FP16 sum of
@@ -219,6 +225,38 @@ typedef struct {
  * {64,128}, Nk a multiple of block_k. */
 thrift_status thrift_kv_block_means(const void* k, int64_t outer, int32_t Nk, int32_t d, int32_t block_k,
                                     double* kbar, void* stream);
+
+/* FP32 tensor scale of an FP16 array: tensor_scale (device float[1]) = amax|x| / 2688 (1 for an
+ * all-zero array), the scale thrift_quantize_nvfp4 would use.  x: device FP16, n elements (n a
+ * multiple of 8, 16-byte aligned).  ws: workspace of at least 256 bytes (its header's scratch
+ * word is used).  Sets a double-cached KV cache's fixed scales from its first tokens (the
+ * capacity buffers hold zeros past them, which leaves the amax unchanged). */
+thrift_status thrift_nvfp4_tensor_scale(const void* x, int64_t n, float* tensor_scale, void* ws,
+                                        size_t ws_bytes, void* stream);
+
+/* Appending to the double-cached KV cache (ThriftAttention technical summary, "Betekenis en
+ * Beweringen": the cache held in FP16 and NVFP4; reading R-append for the update rule).
+ * The cache of `outer` = B*Hkv (batch, KV head) pairs has capacity Ncap keys and holds `len`:
+ *   k, v          device FP16 [outer, Ncap, d], zero past the keys held (the caller zero-fills
+ *                 them once; the library writes only positions below len + T);
+ *   k4 / v4       their NVFP4 copies (group_axis 0 / 1, capacity layouts) whose tensor_scale
+ *                 holds the cache's fixed scale;
+ *   kbar          device float64 [outer, Ncap/block_k, d] key block means.
+ * T new keys per pair: k_new, v_new device FP16 [outer, T, d] are copied to positions
+ * [len, len + T) (either may be NULL when the caller already wrote them there).  Then: the new K
+ * rows are encoded with k4's fixed tensor scale (groups along d); every 16-token V group that the
+ * new keys touch is re-encoded from the FP16 cache with v4's fixed scale (groups along tokens;
+ * the group's positions past len + T read zero); the means of the touched key blocks are
+ * recomputed over the keys each holds (exact FP16 sums in float64 divided by the count).  The
+ * result is bit for bit the NVFP4 quantisation, with the fixed scales, of the zero-padded cache
+ * of len + T keys, whatever the sequence of appends.  Values above the build-time amax saturate
+ * (E4M3 448, E2M1 6).  Requirements: d in {64,128}; block_k in {64,128}; Ncap a multiple of 128
+ * and of block_k; 0 <= len, 1 <= T, len + T <= Ncap; 16-byte aligned buffers.  Five launches on
+ * `stream`; decode the grown cache with thrift_decode_cfg.n_valid = len + T. */
+thrift_status thrift_kv_append(const void* k_new, const void* v_new, int64_t outer, int32_t Ncap, int32_t d,
+                               int32_t block_k, int32_t len, int32_t T, void* k, void* v,
+                               const thrift_nvfp4* k4, const thrift_nvfp4* v4, double* kbar,
+                               void* stream);
 
 /* Workspace bytes of thrift_decode_select, thrift_decode_attn and thrift_decode_fwd (the
  * query rows' NVFP4 copy, the selection of thrift_decode_fwd and the splits' partial sums).

@@ -328,6 +328,7 @@ class DecodeConfig:
     topk_abs: int = -1
     topk_bp: int = 500
     softmax_scale: float = 0.0
+    n_valid: int = 0  # keys the cache holds (0: all Nk)
 
     @classmethod
     def from_workload(cls, w) -> "DecodeConfig":
@@ -336,7 +337,11 @@ class DecodeConfig:
 
     def c(self) -> _lib.CDecodeCfg:
         return _lib.CDecodeCfg(self.B, self.Hq, self.Hkv, self.Nq, self.Nk, self.d, int(self.causal),
-                               self.block_k, self.topk_abs, self.topk_bp, self.softmax_scale)
+                               self.block_k, self.topk_abs, self.topk_bp, self.softmax_scale, self.n_valid)
+
+    def for_cache(self, cache: "KVCache") -> "DecodeConfig":
+        """This step against `cache`: its capacity as Nk and the keys it holds as n_valid."""
+        return dataclasses.replace(self, Nk=cache.capacity, n_valid=cache.length)
 
     @property
     def n_kb(self) -> int:
@@ -369,7 +374,8 @@ def kv_block_means(k: torch.Tensor, block_k: int) -> torch.Tensor:
 
 @dataclasses.dataclass
 class KVCache:
-    """A KV cache held twice, FP16 and NVFP4, with the key block means the selection reads."""
+    """A KV cache held twice, FP16 and NVFP4, with the key block means the selection reads.
+    `capacity` keys of storage, of which the first `length` are held (the rest zero)."""
 
     k: torch.Tensor
     v: torch.Tensor
@@ -377,17 +383,65 @@ class KVCache:
     v4: NVFP4Tensor
     kbar: torch.Tensor
     block_k: int
+    length: int = -1
+    capacity: int = -1
+
+    def __post_init__(self):
+        if self.capacity < 0:
+            self.capacity = self.k.shape[-2]
+        if self.length < 0:
+            self.length = self.capacity
 
     @classmethod
-    def build(cls, k: torch.Tensor, v: torch.Tensor, block_k: int, ws: Optional[Workspace] = None) -> "KVCache":
-        return cls(k, v, quantize_nvfp4(k, 0, ws=ws), quantize_nvfp4(v, 1, ws=ws), kv_block_means(k, block_k),
-                   block_k)
+    def build(cls, k: torch.Tensor, v: torch.Tensor, block_k: int, ws: Optional[Workspace] = None,
+              capacity: Optional[int] = None) -> "KVCache":
+        """The cache of the keys and values k, v [B, Hkv, N, d].  Without `capacity` (and N a
+        multiple of 128 and of block_k) the cache is exactly k, v; with it, zero-filled storage of
+        `capacity` keys holds them and appends can follow (thrift_kv_append): the NVFP4 tensor
+        scales are fixed here, from these first N keys."""
+        if capacity is None:
+            return cls(k, v, quantize_nvfp4(k, 0, ws=ws), quantize_nvfp4(v, 1, ws=ws), kv_block_means(k, block_k),
+                       block_k)
+        B, H, N, d = k.shape
+        dev = k.device
+        kc = torch.zeros((B, H, capacity, d), dtype=torch.float16, device=dev)
+        vc = torch.zeros_like(kc)
+        k4 = NVFP4Tensor.empty(B * H, capacity, d, 0, dev)
+        v4 = NVFP4Tensor.empty(B * H, capacity, d, 1, dev)
+        for t in (k4, v4):
+            t.codes.zero_(); t.scales.zero_(); t.scales_mma.zero_()
+        kbar = torch.zeros((B, H, capacity // block_k, d), dtype=torch.float64, device=dev)
+        cache = cls(kc, vc, k4, v4, kbar, block_k, 0, capacity)
+        kc[:, :, :N].copy_(k)
+        vc[:, :, :N].copy_(v)
+        if ws is None:
+            ws = Workspace(256, dev)
+        L = load()
+        for x, t in ((kc, k4), (vc, v4)):
+            check(L.thrift_nvfp4_tensor_scale(_ptr(x), x.numel(), _ptr(t.tensor_scale), ws.ptr, ws.nbytes,
+                                              _stream()), "thrift_nvfp4_tensor_scale")
+        cache.append(None, None, N)
+        return cache
+
+    def append(self, k_new: Optional[torch.Tensor], v_new: Optional[torch.Tensor], T: Optional[int] = None):
+        """Append T keys and values [B, Hkv, T, d] (thrift_kv_append); None: they are already in
+        the FP16 storage at [length, length + T)."""
+        if T is None:
+            T = k_new.shape[-2]
+        B, H, cap, d = self.k.shape
+        check(load().thrift_kv_append(_ptr(k_new), _ptr(v_new), B * H, cap, d, self.block_k, self.length, T,
+                                      _ptr(self.k), _ptr(self.v), ctypes.byref(self.k4.c()),
+                                      ctypes.byref(self.v4.c()), _ptr(self.kbar), _stream()),
+              "thrift_kv_append")
+        self.length += T
+        return self
 
 
 def decode_select(q: torch.Tensor, cache: KVCache, cfg: DecodeConfig, ws: Optional[Workspace] = None,
                   want_scores: bool = False) -> Selection:
     """Per-head top-k key blocks of one decode step (thrift_decode_select); the Selection's
     tensors have a query-block axis of length 1."""
+    cfg = cfg.for_cache(cache)
     dev = q.device
     sel = Selection(
         torch.empty((cfg.B, cfg.Hq, 1, cfg.mask_words), dtype=torch.int32, device=dev),
@@ -414,6 +468,7 @@ def _decode_out(q, cfg, out, lse, want_lse):
 def decode_attn(q: torch.Tensor, cache: KVCache, sel: Optional[Selection], cfg: DecodeConfig,
                 out=None, lse=None, ws: Optional[Workspace] = None, want_lse: bool = True):
     """Decode attention with a given selection (thrift_decode_attn).  Returns (out, lse)."""
+    cfg = cfg.for_cache(cache)
     out, lse = _decode_out(q, cfg, out, lse, want_lse)
     if ws is None:
         ws = cfg.workspace(q.device)
@@ -428,6 +483,7 @@ def decode_attn(q: torch.Tensor, cache: KVCache, sel: Optional[Selection], cfg: 
 def decode_fwd(q: torch.Tensor, cache: KVCache, cfg: DecodeConfig, out=None, lse=None,
                ws: Optional[Workspace] = None, want_lse: bool = True):
     """One decode step, selection and attention (thrift_decode_fwd).  Returns (out, lse)."""
+    cfg = cfg.for_cache(cache)
     out, lse = _decode_out(q, cfg, out, lse, want_lse)
     if ws is None:
         ws = cfg.workspace(q.device)
@@ -443,6 +499,7 @@ def decode_attn_sparse(q: torch.Tensor, cache: KVCache, sel: Selection, cfg: Dec
                        ws: Optional[Workspace] = None, want_lse: bool = True):
     """Compute-matched sparse decode (thrift_decode_attn_sparse): only the selected key blocks, in
     FP16.  Returns (out, lse)."""
+    cfg = cfg.for_cache(cache)
     out, lse = _decode_out(q, cfg, out, lse, want_lse)
     if ws is None:
         ws = cfg.workspace(q.device)

@@ -40,7 +40,7 @@ class CDecodeCfg(ctypes.Structure):
                 ("Nq", ctypes.c_int32), ("Nk", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("causal", ctypes.c_int32), ("block_k", ctypes.c_int32),
                 ("topk_abs", ctypes.c_int32), ("topk_bp", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("n_valid", ctypes.c_int32)]
 
 
 class CNVFP4(ctypes.Structure):
@@ -73,6 +73,9 @@ SIGNATURES = {
     "thrift_attn_fwd_qat": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _nvp, _vp, _vp, _vp, _vp, _cfgp, _vp, _sz,
                                            _vp]),
     "thrift_kv_block_means": (ctypes.c_int, [_vp, _i64, _i32, _i32, _i32, _vp, _vp]),
+    "thrift_nvfp4_tensor_scale": (ctypes.c_int, [_vp, _i64, _vp, _vp, _sz, _vp]),
+    "thrift_kv_append": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _nvp, _nvp, _vp,
+                                        _vp]),
     "thrift_decode_workspace_bytes": (_sz, [_dcfgp]),
     "thrift_decode_select": (ctypes.c_int, [_vp, _vp, _dcfgp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "thrift_decode_attn": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _vp, _vp, _vp, _dcfgp, _vp, _sz, _vp]),

@@ -108,6 +108,7 @@ bool dcfg_ok(const thrift_decode_cfg* c) {
   if (c->topk_abs < -1) return false;
   if (c->topk_abs == -1 && (c->topk_bp < 0 || c->topk_bp > 10000)) return false;
   if (!(c->softmax_scale >= 0.0f) || std::isinf(c->softmax_scale)) return false;
+  if (c->n_valid != 0 && (c->n_valid < c->Nq || c->n_valid > c->Nk)) return false;
   return true;
 }
 
@@ -402,6 +403,32 @@ thrift_status thrift_decode_fwd(const void* q, const void* k, const void* v, con
     if (st != THRIFT_OK) return st;
   }
   return decode_attn_common(q, k, v, k4, v4, mask, out, lse, cfg, ws, ws_bytes, s);
+}
+
+thrift_status thrift_nvfp4_tensor_scale(const void* x, int64_t n, float* tensor_scale, void* ws, size_t ws_bytes,
+                                        void* stream) {
+  if (!x || !tensor_scale || n <= 0 || n % 8 != 0 || reinterpret_cast<uintptr_t>(x) % 16 != 0)
+    return THRIFT_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, kWsHeader)) return THRIFT_ERR_WORKSPACE;
+  return tensor_scale_launch(x, n, tensor_scale,
+                             reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + kWsAmaxOff),
+                             static_cast<cudaStream_t>(stream));
+}
+
+thrift_status thrift_kv_append(const void* k_new, const void* v_new, int64_t outer, int32_t Ncap, int32_t d,
+                               int32_t block_k, int32_t len, int32_t T, void* k, void* v, const thrift_nvfp4* k4,
+                               const thrift_nvfp4* v4, double* kbar, void* stream) {
+  if (!k || !v || !kbar || !nvfp4_ok(k4, 0) || !nvfp4_ok(v4, 1)) return THRIFT_ERR_INVALID_ARG;
+  if (outer <= 0 || Ncap <= 0 || len < 0 || T < 1 || (int64_t)len + T > Ncap) return THRIFT_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (block_k != 64 && block_k != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (Ncap % 128 != 0 || Ncap % block_k != 0) return THRIFT_ERR_UNSUPPORTED;
+  if (outer * (int64_t)Ncap > (int64_t)INT32_MAX / 2) return THRIFT_ERR_UNSUPPORTED;
+  for (const void* ptr : {k_new, v_new, (const void*)k, (const void*)v, (const void*)k4->codes,
+                          (const void*)v4->codes})
+    if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return THRIFT_ERR_INVALID_ARG;
+  return kv_append_launch(k_new, v_new, outer, Ncap, d, block_k, len, T, k, v, k4, v4, kbar,
+                          static_cast<cudaStream_t>(stream));
 }
 
 thrift_status thrift_reset_device_status(void* ws, void* stream) {

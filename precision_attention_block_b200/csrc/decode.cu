@@ -75,6 +75,7 @@ struct DecodeParams {
   float* part_ml;         // [groups, n_split, 16, 2]
   int* status;
   int B, Hq, Hkv, G, Nq, Nk, R, nkb, mask_words, n_split, bps, causal, mode;
+  int n_valid;  // keys the cache holds (keys from n_valid on are masked; nkb covers the blocks below)
   float tau;
   long long wait_limit;
 };
@@ -353,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_kernel(const __grid_c
   const float sv4 = use4 ? __ldg(p.v_ts) * (1.0f / 2688.0f) : 0.0f;
   const float sl4 = use4 ? p.tau * __ldg(p.q_ts) * __ldg(p.k_ts) * kLog2e : 0.0f;  // FP4 score -> log2 units
   const float sl16 = p.tau * kLog2e;
-  const int64_t qpos0 = (int64_t)p.Nk - p.Nq;  // position of query row 0 among the keys
+  const int64_t qpos0 = (int64_t)p.n_valid - p.Nq;  // position of query row 0 among the keys
   const uint4* qa4 = reinterpret_cast<const uint4*>(smem + L::OFF_QA);             // [D/16][32] A fragments
   const uint4* qa16 = qa4 + (D / 16) * 32;
   uint4* pa_w = reinterpret_cast<uint4*>(smem + L::OFF_PA) + warp * (BK / 16) * 32;  // this warp's P fragments
@@ -457,7 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_kernel(const __grid_c
         for (int e = 0; e < 4; ++e) {
           const int rs = e >> 1;
           const int kk = tig * (BK / 4) + 4 * (nt >> 1) + 2 * (nt & 1) + (e & 1);
-          if (g + 8 * rs >= R || (p.causal && (int64_t)j * BK + kk > qpos[rs]) || (p.mode == 3 && !f16r[rs]))
+          const int64_t key = (int64_t)j * BK + kk;
+          if (g + 8 * rs >= R || (p.causal && key > qpos[rs]) || key >= p.n_valid || (p.mode == 3 && !f16r[rs]))
             sc[nt][e] = kNegInf;
         }
     }
@@ -814,8 +816,9 @@ thrift_status decode_attn_launch(const DecodeArgs& a, cudaStream_t stream) {
   prm.Nq = c.Nq;
   prm.Nk = c.Nk;
   prm.R = prm.G * c.Nq;
-  prm.nkb = c.Nk / c.block_k;
-  prm.mask_words = (prm.nkb + 31) / 32;
+  prm.n_valid = decode_valid(c);
+  prm.nkb = (prm.n_valid + c.block_k - 1) / c.block_k;  // the blocks below the valid length
+  prm.mask_words = (c.Nk / c.block_k + 31) / 32;           // the selection's layout (the capacity)
   prm.causal = c.causal;
   prm.mode = a.mode;
   prm.tau = c.softmax_scale > 0.0f ? c.softmax_scale : 1.0f / sqrtf((float)c.d);

@@ -149,7 +149,134 @@ __global__ void __launch_bounds__(256) encode_cols_kernel(const __half* __restri
   }
 }
 
+__global__ void tensor_scale_kernel(const unsigned int* __restrict__ amax_bits, float* __restrict__ tensor_scale) {
+  *tensor_scale = tensor_scale_from(*amax_bits);
+}
+
+// ---- appending to a double-cached KV cache (capacity Ncap, `len` keys held, T new keys)
+
+// The T new rows of every (batch, KV head) into the FP16 cache at [len, len + T).
+__global__ void __launch_bounds__(256) kv_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int T,
+                                                      int Ncap, int len, int d8, int64_t total) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / d8, c = i - row * d8;
+    const int64_t o = row / T, t = row - o * T;
+    dst[(o * Ncap + len + t) * d8 + c] = src[i];
+  }
+}
+
+// NVFP4 codes of the new K rows (groups along d) with the cache's fixed tensor scale.
+__global__ void __launch_bounds__(256) kv_encode_rows_kernel(const __half* __restrict__ k, int Ncap, int len, int T,
+                                                             int d, int64_t n_groups,
+                                                             const float* __restrict__ tensor_scale,
+                                                             uint2* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                             uint8_t* __restrict__ scales_mma) {
+  const float s_t = __ldg(tensor_scale);
+  const int gpr = d >> 4;
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n_groups;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t rn = g / gpr, grp = g - rn * gpr;
+    const int64_t o = rn / T, t = rn - o * T;
+    const int64_t row = o * Ncap + len + t;
+    const uint4* src = reinterpret_cast<const uint4*>(k + row * d + grp * 16);
+    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+    float f[16];
+    const __half2* h0 = reinterpret_cast<const __half2*>(&v0);
+    const __half2* h1 = reinterpret_cast<const __half2*>(&v1);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 a = __half22float2(h0[e]), b = __half22float2(h1[e]);
+      f[2 * e] = a.x; f[2 * e + 1] = a.y; f[8 + 2 * e] = b.x; f[8 + 2 * e + 1] = b.y;
+    }
+    uint2 packed;
+    const uint32_t sb = quant16(f, s_t, packed);
+    codes[row * gpr + grp] = packed;
+    scales[row * gpr + grp] = (uint8_t)sb;
+    scales_mma[sf_mma_offset(row, grp, d >> 6)] = (uint8_t)sb;
+  }
+}
+
+// NVFP4 codes of the 16-token V groups g0 .. g0 + ng - 1 (groups along tokens), from the FP16
+// cache (zero past the keys held) with the cache's fixed tensor scale.
+__global__ void __launch_bounds__(256) kv_encode_cols_kernel(const __half* __restrict__ v, int Ncap, int d, int g0,
+                                                             int ng, int64_t total,
+                                                             const float* __restrict__ tensor_scale,
+                                                             uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                             uint8_t* __restrict__ scales_mma) {
+  const float s_t = __ldg(tensor_scale);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c = i % d, rest = i / d;
+    const int64_t gi = rest % ng, o = rest / ng;
+    const int64_t grp = g0 + gi;
+    float f[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) f[t] = __half2float(v[(o * Ncap + grp * 16 + t) * d + c]);
+    uint2 packed;
+    const uint32_t sb = quant16(f, s_t, packed);
+    const int64_t row = o * d + c;
+    *reinterpret_cast<uint2*>(codes + row * (Ncap / 2) + grp * 8) = packed;
+    scales[row * (Ncap / 16) + grp] = (uint8_t)sb;
+    scales_mma[sf_mma_offset(row, grp, Ncap >> 6)] = (uint8_t)sb;
+  }
+}
+
+// Means of the key blocks j0 .. j0 + nj - 1 over the keys each holds (below n_valid): exact FP16
+// sums in float64 divided by the count.
+__global__ void __launch_bounds__(256) kv_means_kernel(const __half* __restrict__ k, int Ncap, int d, int bk, int j0,
+                                                       int nj, int n_valid, int64_t total, double* __restrict__ kbar) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c = i % d, rest = i / d;
+    const int64_t jj = rest % nj, o = rest / nj;
+    const int64_t j = j0 + jj;
+    const int cnt = (int)min((int64_t)bk, (int64_t)n_valid - j * bk);
+    double s = 0.0;
+    for (int t = 0; t < cnt; ++t) s += (double)__half2float(k[(o * Ncap + j * bk + t) * d + c]);
+    kbar[(o * (Ncap / bk) + j) * d + c] = s / (double)cnt;
+  }
+}
+
 }  // namespace
+
+thrift_status tensor_scale_launch(const void* x, int64_t n, float* tensor_scale, unsigned int* amax_slot,
+                                  cudaStream_t stream) {
+  if (cudaMemsetAsync(amax_slot, 0, sizeof(unsigned int), stream) != cudaSuccess) return THRIFT_ERR_CUDA;
+  int64_t blocks = (n / 8 + 4 * 256 - 1) / (4 * 256);
+  if (blocks > (int64_t)num_sms() * 8) blocks = (int64_t)num_sms() * 8;
+  if (blocks < 1) blocks = 1;
+  amax_kernel<<<(unsigned)blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), n / 8, amax_slot);
+  tensor_scale_kernel<<<1, 1, 0, stream>>>(amax_slot, tensor_scale);
+  return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
+}
+
+thrift_status kv_append_launch(const void* k_new, const void* v_new, int64_t outer, int32_t Ncap, int32_t d,
+                               int32_t block_k, int32_t len, int32_t T, void* k, void* v, const thrift_nvfp4* k4,
+                               const thrift_nvfp4* v4, double* kbar, cudaStream_t stream) {
+  const int sms = num_sms();
+  auto grid_for = [&](int64_t work) {
+    int64_t b = (work + 255) / 256;
+    if (b > (int64_t)sms * 16) b = (int64_t)sms * 16;
+    return (unsigned)(b < 1 ? 1 : b);
+  };
+  const int64_t vecs = outer * (int64_t)T * (d / 8);
+  if (k_new) kv_copy_kernel<<<grid_for(vecs), 256, 0, stream>>>(reinterpret_cast<const uint4*>(k_new),
+                                                                 reinterpret_cast<uint4*>(k), T, Ncap, len, d / 8, vecs);
+  if (v_new) kv_copy_kernel<<<grid_for(vecs), 256, 0, stream>>>(reinterpret_cast<const uint4*>(v_new),
+                                                                 reinterpret_cast<uint4*>(v), T, Ncap, len, d / 8, vecs);
+  const int64_t kgroups = outer * (int64_t)T * (d / 16);
+  kv_encode_rows_kernel<<<grid_for(kgroups), 256, 0, stream>>>(
+      reinterpret_cast<const __half*>(k), Ncap, len, T, d, kgroups, k4->tensor_scale,
+      reinterpret_cast<uint2*>(k4->codes), k4->scales, k4->scales_mma);
+  const int g0 = len / 16, g1 = (len + T - 1) / 16;
+  const int64_t vwork = outer * (int64_t)(g1 - g0 + 1) * d;
+  kv_encode_cols_kernel<<<grid_for(vwork), 256, 0, stream>>>(reinterpret_cast<const __half*>(v), Ncap, d, g0,
+                                                            g1 - g0 + 1, vwork, v4->tensor_scale, v4->codes,
+                                                            v4->scales, v4->scales_mma);
+  const int j0 = len / block_k, j1 = (len + T - 1) / block_k;
+  const int64_t mwork = outer * (int64_t)(j1 - j0 + 1) * d;
+  kv_means_kernel<<<grid_for(mwork), 256, 0, stream>>>(reinterpret_cast<const __half*>(k), Ncap, d, block_k, j0,
+                                                      j1 - j0 + 1, len + T, mwork, kbar);
+  return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
+}
 
 size_t scales_mma_bytes(int64_t outer, int32_t N, int32_t d, int32_t group_axis) {
   int64_t rows = group_axis == 0 ? outer * N : outer * d;

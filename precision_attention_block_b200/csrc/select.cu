@@ -277,10 +277,11 @@ __global__ void __launch_bounds__(32 * kListRowsPerCta) lists_kernel(const uint3
 // query rows of the G heads of one KV head (exact FP16 sums in float64, divided by Nq) and stages
 // kDecScoreBlocks key-block means in shared memory; thread (hl, jj) scores block jj for query head
 // hk*G + hl, the sum in the order c = 0 .. d-1 with no fused multiply-add (the evaluation the
-// prefill scores use).
+// prefill scores use).  Blocks from nkb_valid on (past the cache's valid length) score -inf, which
+// leaves them out of the top-k and its budget.
 constexpr int kDecScoreBlocks = 16;
 __global__ void decode_score_kernel(const __half* __restrict__ q, int Nq, const double* __restrict__ kbar, int Hq,
-                                    int Hkv, int nkb, int d, double* __restrict__ scores) {
+                                    int Hkv, int nkb, int nkb_valid, int d, double* __restrict__ scores) {
   __shared__ double ks[kDecScoreBlocks * 129];
   __shared__ double qs[16 * 128];
   const int G = Hq / Hkv, grp = blockIdx.y;
@@ -304,6 +305,7 @@ __global__ void decode_score_kernel(const __half* __restrict__ q, int Nq, const 
   double acc = 0.0;
 #pragma unroll 8
   for (int c = 0; c < d; ++c) acc = __dadd_rn(acc, __dmul_rn(qr[c], kr[c]));
+  if (j0 + jj >= nkb_valid) acc = -__builtin_huge_val();
   scores[((int64_t)b * Hq + (int64_t)hk * G + hl) * nkb + j0 + jj] = acc;
 }
 
@@ -380,18 +382,20 @@ size_t decode_select_scratch_bytes(const thrift_decode_cfg& c) {
 }
 
 // The decode selection is the prefill selection with one query block of Nq rows per head.
-// Every key block holds a key visible to the newest row, so every pair is valid.
+// Every key block below the valid length holds a key visible to the newest row, so those pairs
+// are valid; the blocks past it are not.
 thrift_status decode_select_launch(const void* q, const double* kbar, const thrift_decode_cfg& c, uint32_t* mask,
                                    int32_t* counts, int16_t* lists, double* scores_out, uint8_t* scratch,
                                    cudaStream_t stream) {
   const int nkb = c.Nk / c.block_k;
+  const int nkb_valid = (decode_valid(c) + c.block_k - 1) / c.block_k;
   const int mask_words = (nkb + 31) / 32;
   const size_t heads = (size_t)c.B * c.Hq;
   double* scores = scores_out ? scores_out
                               : reinterpret_cast<double*>(scratch + align256(heads * c.d * sizeof(double)));
   dim3 g((nkb + kDecScoreBlocks - 1) / kDecScoreBlocks, (unsigned)(c.B * c.Hkv));
   decode_score_kernel<<<g, kDecScoreBlocks * (c.Hq / c.Hkv), 0, stream>>>(
-      reinterpret_cast<const __half*>(q), c.Nq, kbar, c.Hq, c.Hkv, nkb, c.d, scores);
+      reinterpret_cast<const __half*>(q), c.Nq, kbar, c.Hq, c.Hkv, nkb, nkb_valid, c.d, scores);
   if (cudaMemsetAsync(mask, 0, heads * mask_words * sizeof(uint32_t), stream) != cudaSuccess) return THRIFT_ERR_CUDA;
   if (nkb <= kSelSmemKeys)
     topk_kernel<256><<<(unsigned)heads, 256, 0, stream>>>(scores, (int64_t)nkb, nkb, c.topk_abs, c.topk_bp,

@@ -28,6 +28,13 @@ size_t scales_mma_bytes(int64_t outer, int32_t N, int32_t d, int32_t group_axis)
 thrift_status quantize_launch(const void* x, int64_t outer, int32_t N, int32_t d, const thrift_nvfp4* out,
                               unsigned int* amax_slot, cudaStream_t stream);
 
+thrift_status tensor_scale_launch(const void* x, int64_t n, float* tensor_scale, unsigned int* amax_slot,
+                                  cudaStream_t stream);
+
+thrift_status kv_append_launch(const void* k_new, const void* v_new, int64_t outer, int32_t Ncap, int32_t d,
+                               int32_t block_k, int32_t len, int32_t T, void* k, void* v, const thrift_nvfp4* k4,
+                               const thrift_nvfp4* v4, double* kbar, cudaStream_t stream);
+
 thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, uint32_t* mask, int32_t* counts,
                             int16_t* lists, double* scores_out, uint8_t* scratch, cudaStream_t stream);
 
@@ -47,6 +54,9 @@ thrift_status ex2_probe_launch(const float* x, float* y, int64_t n, int which, c
 size_t pipe_rates_ws_bytes();
 
 // ---- decode
+// The cache's valid length (thrift_decode_cfg.n_valid, 0 meaning the whole capacity).
+inline int decode_valid(const thrift_decode_cfg& c) { return c.n_valid > 0 ? c.n_valid : c.Nk; }
+
 struct DecodeArgs {
   const thrift_decode_cfg* cfg;
   const void *q, *k, *v;

@@ -159,3 +159,18 @@ def test_decode_null_and_workspace_errors(L):
     assert L.thrift_kv_block_means(None, 1, 128, 128, 64, p, None) == 1
     assert L.thrift_kv_block_means(p, 1, 100, 128, 64, p, None) == 2
     assert L.thrift_kv_block_means(p, 1, 128, 96, 64, p, None) == 2
+    # appending: the new keys must fit the capacity; unsupported sizes; misaligned buffers
+    n0 = _lib.CNVFP4(0x1000, 0x1000, 0x1000, 0x1000, 0)
+    n1 = _lib.CNVFP4(0x1000, 0x1000, 0x1000, 0x1000, 1)
+    assert L.thrift_kv_append(p, p, 2, 1024, 64, 64, 1000, 25, p, p, ctypes.byref(n0), ctypes.byref(n1), p,
+                              None) == 1
+    assert L.thrift_kv_append(p, p, 2, 1024, 96, 64, 0, 1, p, p, ctypes.byref(n0), ctypes.byref(n1), p, None) == 2
+    assert L.thrift_kv_append(p, p, 2, 1000, 64, 64, 0, 1, p, p, ctypes.byref(n0), ctypes.byref(n1), p, None) == 2
+    assert L.thrift_kv_append(p, p, 2, 1024, 64, 64, 0, 1, p, p, ctypes.byref(n1), ctypes.byref(n1), p, None) == 1
+    assert L.thrift_kv_append(ctypes.c_void_p(0x1008), p, 2, 1024, 64, 64, 0, 1, p, p, ctypes.byref(n0),
+                              ctypes.byref(n1), p, None) == 1
+    assert L.thrift_nvfp4_tensor_scale(p, 12, p, p, 256, None) == 1
+    assert L.thrift_nvfp4_tensor_scale(p, 16, p, None, 256, None) == 5
+    # the decode step's valid length lies between Nq and the capacity
+    assert L.thrift_decode_workspace_bytes(ctypes.byref(dcfg(n_valid=131072 + 1))) == 0
+    assert L.thrift_decode_workspace_bytes(ctypes.byref(dcfg(n_valid=1000))) > 0
