@@ -276,6 +276,33 @@ def attn(q, k, v, q4: NVFP4, k4: NVFP4, v4: NVFP4, sel, w, tau=None, units=None,
     return out.view(np.float16), lse, out64
 
 
+def attn_r2(q, k, v, q4: NVFP4, k4: NVFP4, v4: NVFP4, sel, w, tau=None, units=None, want_f64=False,
+            threads=None):
+    """Attention forward under reading R2 of the two-level P quantisation (the running maximum,
+    in the fused kernel's visiting order -- NVFP4 key blocks ascending, then FP16 ones -- as the
+    first level).  Same arguments and return values as `attn`."""
+    B, Hq, N, d = q.shape
+    if tau is None:
+        tau = softmax_scale(d)
+    if units is None:
+        units = [(b, h, i) for b in range(B) for h in range(Hq) for i in range(N // w.block_q)]
+    u = np.ascontiguousarray(np.array(units, np.int32).reshape(-1))
+    out = np.zeros((B, Hq, N, d), np.uint16)
+    lse = np.zeros((B, Hq, N), np.float32)
+    out64 = np.zeros((B, Hq, N, d), np.float64) if want_f64 else None
+    if threads is None:
+        threads = os.cpu_count() or 1
+    lib().orc_attn(_u16(q).reshape(-1), _u16(k).reshape(-1), _u16(v).reshape(-1),
+                   q4.codes.reshape(-1), q4.scales.reshape(-1), q4.tensor_scale,
+                   k4.codes.reshape(-1), k4.scales.reshape(-1), k4.tensor_scale,
+                   v4.codes.reshape(-1), v4.scales.reshape(-1), v4.tensor_scale,
+                   np.ascontiguousarray(sel, np.uint8).reshape(-1),
+                   B, Hq, k.shape[1], N, d, w.block_q, w.block_k, int(w.causal), np.float32(tau),
+                   u, len(units), 2, None, out.reshape(-1), lse.reshape(-1),
+                   None if out64 is None else out64.ctypes.data, int(threads))
+    return out.view(np.float16), lse, out64
+
+
 def attn_sparse(q, k, v, sel, w, tau=None, units=None, want_f64=False, threads=None):
     """Compute-matched sparse variant (reading R-sparse): only the selected pairs, in FP16; every
     other pair dropped.  A row left with no key gets output 0 and lse -inf.  Same return values as

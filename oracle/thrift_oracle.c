@@ -372,10 +372,20 @@ static void block_scores(const attn_problem* P, int b, int h, int i, int j, int 
  * masked.  Otherwise writes M (row max in the block), sumP (sum of the FP32
  * exp(S - M), unquantised) and Pq (the probabilities the PV product uses, relative
  * to M: FP4 pairs dequantised NVFP4 codes / 2688, FP16 pairs FP16-rounded exp). */
+static void tile_pq_at(const double* S, int bk, int fp16, double M, double* sumP_out, double* Pq);
+
 int orc_tile_pq(const double* S, int bk, int fp16, double* M_out, double* sumP_out, double* Pq) {
   double M = -INFINITY;
   for (int t = 0; t < bk; ++t) if (S[t] > M) M = S[t];
   if (M == -INFINITY) return 0;
+  tile_pq_at(S, bk, fp16, M, sumP_out, Pq);
+  *M_out = M;
+  return 1;
+}
+
+/* The same two-level quantisation with a given first-level reference M >= the tile's maximum:
+ * P^ = exp(S - M) in FP32, P' = 2688 P^ quantised per 16 keys (NVFP4) or P^ rounded to FP16. */
+static void tile_pq_at(const double* S, int bk, int fp16, double M, double* sumP_out, double* Pq) {
   float ph[512];
   double sum = 0.0;
   for (int t = 0; t < bk; ++t) {
@@ -400,9 +410,7 @@ int orc_tile_pq(const double* S, int bk, int fp16, double* M_out, double* sumP_o
       }
     }
   }
-  *M_out = M;
   *sumP_out = sum;
-  return 1;
 }
 
 /* V rows of key block j, [bk, d]: FP16 V, or the token-grouped NVFP4 V dequantised
@@ -488,6 +496,65 @@ static void attn_unit(const attn_problem* P, int b, int h, int i, int online, co
   free(S); free(qd); free(kd); free(vd); free(Pq); free(acc); free(m); free(l);
 }
 
+/* One (b, h, query block i) unit under reading R2 of the two-level P quantisation: the first level
+ * is the row's running maximum m over the key blocks visited so far, in the fused kernel's order
+ * (the NVFP4 blocks in ascending j, then the FP16 blocks in ascending j).  Per row and visited
+ * block: m_new = max(m, M_block); the output and denominator so far are rescaled by
+ * exp(m - m_new); P^ = exp(S - m_new) (so P' = 2688 P^ reaches 2688 only where the block holds
+ * the running maximum); the quantised P^ times V is added to the output and the unquantised sum
+ * of P^ to the denominator.  The result depends on the visiting order, unlike R1's. */
+static void attn_unit_r2(const attn_problem* P, int b, int h, int i, uint16_t* out, float* lse, double* out64) {
+  int nkb = P->Nk / P->bk, d = P->d, bq = P->bq, bk = P->bk;
+  int64_t qoff = qoff_of(P);
+  double* S = (double*)malloc(sizeof(double) * (size_t)bq * bk);
+  double* qd = (double*)malloc(sizeof(double) * (size_t)d);
+  double* kd = (double*)malloc(sizeof(double) * (size_t)bk * d);
+  double* vd = (double*)malloc(sizeof(double) * (size_t)bk * d);
+  double* Pq = (double*)malloc(sizeof(double) * (size_t)bk);
+  double* acc = (double*)calloc((size_t)bq * d, sizeof(double));
+  double* m = (double*)malloc(sizeof(double) * (size_t)bq);
+  double* l = (double*)calloc((size_t)bq, sizeof(double));
+  for (int r = 0; r < bq; ++r) m[r] = -INFINITY;
+  for (int phase = 0; phase < 2; ++phase) {
+    for (int j = 0; j < nkb; ++j) {
+      if (!pair_valid(P->causal, qoff, i, j, bq, bk, P->nvalid)) continue;
+      int fp16 = pair_is_fp16(P, b, h, i, j);
+      if (fp16 != phase) continue;
+      block_scores(P, b, h, i, j, fp16, qd, kd, S, bk);
+      block_values(P, b, h, j, fp16, vd);
+      for (int r = 0; r < bq; ++r) {
+        const double* Sr = S + (int64_t)r * bk;
+        double M = -INFINITY;
+        for (int t = 0; t < bk; ++t) if (Sr[t] > M) M = Sr[t];
+        if (M == -INFINITY) continue;
+        double mn = M > m[r] ? M : m[r];
+        double alpha = m[r] == -INFINITY ? 0.0 : exp(m[r] - mn);
+        double* a = acc + (int64_t)r * d;
+        for (int c = 0; c < d; ++c) a[c] *= alpha;
+        l[r] *= alpha;
+        m[r] = mn;
+        double sumP;
+        tile_pq_at(Sr, bk, fp16, mn, &sumP, Pq);
+        l[r] += sumP;
+        for (int t = 0; t < bk; ++t) {
+          if (Pq[t] == 0.0) continue;
+          for (int c = 0; c < d; ++c) a[c] += Pq[t] * vd[t * d + c];
+        }
+      }
+    }
+  }
+  for (int r = 0; r < bq; ++r) {
+    int64_t orow = ((int64_t)b * P->Hq + h) * P->Nq + (int64_t)i * bq + r;
+    for (int c = 0; c < d; ++c) {
+      double o = l[r] > 0.0 ? acc[(int64_t)r * d + c] / l[r] : 0.0;
+      out[orow * d + c] = orc_double_to_half(o);
+      if (out64) out64[orow * d + c] = o;
+    }
+    lse[orow] = l[r] > 0.0 ? (float)(m[r] + log(l[r])) : -INFINITY;
+  }
+  free(S); free(qd); free(kd); free(vd); free(Pq); free(acc); free(m); free(l);
+}
+
 typedef struct {
   const attn_problem* P;
   const int32_t* units;
@@ -508,13 +575,18 @@ static void* attn_worker(void* arg) {
     int u = J->next++;
     pthread_mutex_unlock(&J->mu);
     if (u >= J->n_units) break;
-    attn_unit(J->P, J->units[3 * u], J->units[3 * u + 1], J->units[3 * u + 2], J->online, J->order, J->out,
-              J->lse, J->out64);
+    if (J->online == 2)
+      attn_unit_r2(J->P, J->units[3 * u], J->units[3 * u + 1], J->units[3 * u + 2], J->out, J->lse, J->out64);
+    else
+      attn_unit(J->P, J->units[3 * u], J->units[3 * u + 1], J->units[3 * u + 2], J->online, J->order, J->out,
+                J->lse, J->out64);
   }
   return NULL;
 }
 
-/* Attention forward over the listed (b, h, i) units.  Inputs: FP16 q [B,Hq,Nq,d], k, v
+/* Attention forward over the listed (b, h, i) units (online = 0: reading R1, two-pass; 1: R1 with
+ * an online merge in the order `order`; 2: reading R2, the kernel's visiting order).
+ * Inputs: FP16 q [B,Hq,Nq,d], k, v
  * [B,Hkv,Nk,d] whose first nvalid keys are valid (query row r at position nvalid - Nq + r;
  * keys at or past nvalid are masked); NVFP4 codes/scales of q, k (grouped
  * along d) and v (grouped along tokens, [B,Hkv,d,Nk/2]) with their tensor scales;
