@@ -160,6 +160,23 @@ thrift_status thrift_attn_fwd_qat(const void* q, const void* k, const void* v,
                                   float* out_hp, float* lse, const thrift_cfg* cfg, void* ws,
                                   size_t ws_bytes, void* stream);
 
+/* thrift_attn_fwd with the other reading of the two-level P requantisation (ThriftAttention
+ * "Twee-niveau P-herkwantisatie", which follows SageAttention3's two-level scheme).
+ * thrift_attn_fwd takes each key block's own row maximum M as the first level: P^ = exp(S - M),
+ * so every block's largest probability requantises at the top of the NVFP4 range.  Here the
+ * first level is the row's running maximum m over the key blocks visited so far, in the kernel's
+ * fixed order -- the NVFP4 blocks in ascending key-block index, then the FP16 blocks ascending:
+ * m = max(m, M), P^ = exp(S - m), the E4M3 group scales of 2688 P^ and the E2M1 codes follow,
+ * and the denominator adds the unquantised sum of P^.  A block below the running maximum thus
+ * requantises with smaller group scales; the output depends on the visiting order and differs
+ * from thrift_attn_fwd's by the requantisation error.  Arguments, requirements and errors as
+ * thrift_attn_fwd (mask only; no counts or lists). */
+thrift_status thrift_attn_fwd_running_max(const void* q, const void* k, const void* v,
+                                          const thrift_nvfp4* q4, const thrift_nvfp4* k4,
+                                          const thrift_nvfp4* v4, const uint32_t* mask, void* out,
+                                          float* lse, const thrift_cfg* cfg, void* ws,
+                                          size_t ws_bytes, void* stream);
+
 /* Compute-matched sparse variant of thrift_attn_fwd (ThriftAttention compares against sparse
  * attention at a matched compute budget): only the selected pairs of `mask` run, in FP16 with the
  * FP16 q, k, v; every other pair is dropped as if masked.  A row left with no key gets output 0

@@ -184,8 +184,11 @@ def block_select(q: torch.Tensor, k: torch.Tensor, cfg: Config, ws: Optional[Wor
 
 def attn_fwd(q, k, v, q4: Optional[NVFP4Tensor], k4: Optional[NVFP4Tensor], v4: Optional[NVFP4Tensor],
              sel: Optional[Selection], cfg: Config, out: Optional[torch.Tensor] = None,
-             lse: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None, want_lse: bool = True):
-    """Selective mixed-precision attention forward (thrift_attn_fwd).  Returns (out, lse)."""
+             lse: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None, want_lse: bool = True,
+             running_max: bool = False):
+    """Selective mixed-precision attention forward (thrift_attn_fwd).  Returns (out, lse).
+    running_max: requantise P against the row's running maximum instead of each key block's own
+    maximum (thrift_attn_fwd_running_max)."""
     ref = q if q is not None else q4.codes
     dev = ref.device
     if out is None:
@@ -197,6 +200,12 @@ def attn_fwd(q, k, v, q4: Optional[NVFP4Tensor], k4: Optional[NVFP4Tensor], v4: 
     c = cfg.c()
     n4 = [None if t is None else t.c() for t in (q4, k4, v4)]
     refs = [None if t is None else ctypes.byref(t) for t in n4]
+    if running_max:
+        check(load().thrift_attn_fwd_running_max(_ptr(q), _ptr(k), _ptr(v), refs[0], refs[1], refs[2],
+                                                 None if sel is None else _ptr(sel.mask), _ptr(out), _ptr(lse),
+                                                 ctypes.byref(c), ws.ptr, ws.nbytes, _stream()),
+              "thrift_attn_fwd_running_max")
+        return out, lse
     check(load().thrift_attn_fwd(_ptr(q), _ptr(k), _ptr(v), refs[0], refs[1], refs[2],
                                  None if sel is None else _ptr(sel.mask),
                                  None if sel is None else _ptr(sel.counts),

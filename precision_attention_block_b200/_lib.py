@@ -72,6 +72,8 @@ SIGNATURES = {
     "thrift_attn_fwd_auto": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _cfgp, _vp, _sz, _vp]),
     "thrift_attn_fwd_qat": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _nvp, _vp, _vp, _vp, _vp, _cfgp, _vp, _sz,
                                            _vp]),
+    "thrift_attn_fwd_running_max": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _nvp, _vp, _vp, _vp, _cfgp, _vp,
+                                                   _sz, _vp]),
     "thrift_kv_block_means": (ctypes.c_int, [_vp, _i64, _i32, _i32, _i32, _vp, _vp]),
     "thrift_nvfp4_tensor_scale": (ctypes.c_int, [_vp, _i64, _vp, _vp, _sz, _vp]),
     "thrift_kv_append": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _nvp, _nvp, _vp,

@@ -13,8 +13,8 @@ namespace thrift {
 
 thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
                               const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
-                              void* out, float* out_hp, float* lse, const thrift_cfg& c, int* status, float* dbg,
-                              int dbg_entry, cudaStream_t stream);
+                              void* out, float* out_hp, float* lse, int running_max, const thrift_cfg& c, int* status,
+                              float* dbg, int dbg_entry, cudaStream_t stream);
 
 int num_sms() {
   static int cache[64] = {0};
@@ -260,8 +260,8 @@ thrift_status thrift_block_select_noalloc(const void* q, const void* k, const th
 
 static thrift_status attn_common(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
                                  const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, void* out,
-                                 float* out_hp, float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes,
-                                 float* dbg, int dbg_entry, void* stream) {
+                                 float* out_hp, float* lse, int running_max, const thrift_cfg* cfg, void* ws,
+                                 size_t ws_bytes, float* dbg, int dbg_entry, void* stream) {
   thrift_status st = cfg_supported(cfg);
   if (st != THRIFT_OK) return st;
   if (!out) return THRIFT_ERR_INVALID_ARG;
@@ -270,8 +270,8 @@ static thrift_status attn_common(const void* q, const void* k, const void* v, co
   if (mode != 1 && (!q || !k || !v)) return THRIFT_ERR_INVALID_ARG;
   if (mode == 0 && !mask) return THRIFT_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, kWsHeader)) return THRIFT_ERR_WORKSPACE;
-  return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, out_hp, lse, *cfg, status_ptr(ws), dbg, dbg_entry,
-                         static_cast<cudaStream_t>(stream));
+  return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, out_hp, lse, running_max, *cfg, status_ptr(ws), dbg,
+                         dbg_entry, static_cast<cudaStream_t>(stream));
 }
 
 thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
@@ -280,7 +280,14 @@ thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, const
                               const thrift_cfg* cfg, void* ws, size_t ws_bytes, void* stream) {
   (void)counts;
   (void)lists;
-  return attn_common(q, k, v, q4, k4, v4, mask, out, nullptr, lse, cfg, ws, ws_bytes, nullptr, -1, stream);
+  return attn_common(q, k, v, q4, k4, v4, mask, out, nullptr, lse, 0, cfg, ws, ws_bytes, nullptr, -1, stream);
+}
+
+thrift_status thrift_attn_fwd_running_max(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
+                                          const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask,
+                                          void* out, float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes,
+                                          void* stream) {
+  return attn_common(q, k, v, q4, k4, v4, mask, out, nullptr, lse, 1, cfg, ws, ws_bytes, nullptr, -1, stream);
 }
 
 thrift_status thrift_attn_fwd_qat(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
@@ -288,7 +295,7 @@ thrift_status thrift_attn_fwd_qat(const void* q, const void* k, const void* v, c
                                   float* out_hp, float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes,
                                   void* stream) {
   if (!out_hp) return THRIFT_ERR_INVALID_ARG;
-  return attn_common(q, k, v, q4, k4, v4, mask, out, out_hp, lse, cfg, ws, ws_bytes, nullptr, -1, stream);
+  return attn_common(q, k, v, q4, k4, v4, mask, out, out_hp, lse, 0, cfg, ws, ws_bytes, nullptr, -1, stream);
 }
 
 thrift_status thrift_debug_attn_dump(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
@@ -296,7 +303,7 @@ thrift_status thrift_debug_attn_dump(const void* q, const void* k, const void* v
                                      void* out, float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes,
                                      float* dbg, int32_t dbg_entry, void* stream) {
   if (!dbg) return THRIFT_ERR_INVALID_ARG;
-  return attn_common(q, k, v, q4, k4, v4, mask, out, nullptr, lse, cfg, ws, ws_bytes, dbg, dbg_entry, stream);
+  return attn_common(q, k, v, q4, k4, v4, mask, out, nullptr, lse, 0, cfg, ws, ws_bytes, dbg, dbg_entry, stream);
 }
 
 thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, void* out, float* lse,
@@ -326,7 +333,7 @@ thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, 
                        nullptr, w + L.select, s);
     if (st != THRIFT_OK) return st;
   }
-  return attn_launch_dbg(q, k, v, &q4, &k4, &v4, mode == 0 ? mask : nullptr, mode, out, nullptr, lse, c,
+  return attn_launch_dbg(q, k, v, &q4, &k4, &v4, mode == 0 ? mask : nullptr, mode, out, nullptr, lse, 0, c,
                          status_ptr(ws), nullptr, -1, s);
 }
 
@@ -382,7 +389,7 @@ thrift_status thrift_attn_fwd_sparse(const void* q, const void* k, const void* v
   if (st != THRIFT_OK) return st;
   if (!q || !k || !v || !mask || !out) return THRIFT_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, kWsHeader)) return THRIFT_ERR_WORKSPACE;
-  return attn_launch_dbg(q, k, v, nullptr, nullptr, nullptr, mask, 3, out, nullptr, lse, *cfg, status_ptr(ws), nullptr, -1,
+  return attn_launch_dbg(q, k, v, nullptr, nullptr, nullptr, mask, 3, out, nullptr, lse, 0, *cfg, status_ptr(ws), nullptr, -1,
                          static_cast<cudaStream_t>(stream));
 }
 

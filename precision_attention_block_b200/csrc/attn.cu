@@ -132,6 +132,7 @@ struct AttnParams {
   float* dbg;  // optional dump of one entry (S, P bytes, PV) of tile 0 of the first unit of CTA 0
   int dbg_entry;
   int B, Hq, Hkv, N, bq, causal, mode, nqb, nkb, mask_words, n_units;  // mode as attn_launch
+  int running_max;  // first level of the P requantisation: 0 = the block maximum, 1 = the running maximum
   int npage, maxe, off_bar, off_list;
   float tau;
   long long wait_limit;
@@ -738,6 +739,9 @@ __global__ void __launch_bounds__(384, 1)
       // maximum exceeds it by more than 2^kRescale (the final O / l does not depend on m_ref).
       // Both warpgroups see the same block maxima, so they take the same decisions.
       float m_ref = kNegInf, l_run = 0.0f;
+      // running maximum of the row over the entries visited so far (log2 units), the first level
+      // of the P requantisation when p.running_max is set
+      float m_run = kNegInf;
       // block maximum (log2 units; -inf: the row took no part), unquantised sum and precision of
       // the entries whose PV products are still to be merged: entry e - 1 (p1) and e - 2 (p2)
       float p1_M = kNegInf, p1_sum = 0.0f, p2_M = kNegInf, p2_sum = 0.0f;
@@ -845,7 +849,11 @@ __global__ void __launch_bounds__(384, 1)
             for (int q = 0; q < KH / 16; ++q) gm[q] = kNegInf;
           }
           const bool valid = M != kNegInf;  // false when every key of the block is masked for this row
-          const float Ms = valid ? M * sl2 : __builtin_huge_valf();  // +inf zeroes every probability
+          float Ms = valid ? M * sl2 : __builtin_huge_valf();  // +inf zeroes every probability
+          if (p.running_max && valid) {
+            Ms = fmaxf(Ms, m_run);
+            m_run = Ms;
+          }
 
           // this warpgroup's probabilities, 32 keys at a time, into PV operand buffer `buf`; its
           // previous reader, the PV product of entry e - 2, has completed (ready(v) covers it)
@@ -1047,8 +1055,8 @@ __global__ void wait_timeout_kernel(int* status, long long limit) {
 
 thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
                               const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
-                              void* out, float* out_hp, float* lse, const thrift_cfg& c, int* status, float* dbg,
-                              int dbg_entry, cudaStream_t stream) {
+                              void* out, float* out_hp, float* lse, int running_max, const thrift_cfg& c, int* status,
+                              float* dbg, int dbg_entry, cudaStream_t stream) {
   AttnParams prm;
   memset(&prm, 0, sizeof(prm));
   prm.mask = mask;
@@ -1073,6 +1081,7 @@ thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const
   prm.bq = c.block_q;
   prm.causal = c.causal;
   prm.mode = mode;
+  prm.running_max = running_max;
   prm.nqb = c.N / c.block_q;
   prm.nkb = c.N / c.block_k;
   prm.mask_words = (prm.nkb + 31) / 32;
@@ -1089,7 +1098,7 @@ thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const
 thrift_status attn_launch(const void* q, const void* k, const void* v, const thrift_nvfp4* q4, const thrift_nvfp4* k4,
                           const thrift_nvfp4* v4, const uint32_t* mask, int mode, void* out, float* lse,
                           const thrift_cfg& c, int* status, cudaStream_t stream) {
-  return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, nullptr, lse, c, status, nullptr, -1, stream);
+  return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, nullptr, lse, 0, c, status, nullptr, -1, stream);
 }
 
 thrift_status ex2_probe_launch(const float* x, float* y, int64_t n, int which, cudaStream_t stream) {

@@ -98,6 +98,14 @@ def test_null_and_workspace_errors(L):
     # the Attn-QAT variant needs its FP32 output
     assert L.thrift_attn_fwd_qat(p, p, p, ctypes.byref(nv), ctypes.byref(nv), ctypes.byref(nv), p, p, None, None,
                                  ctypes.byref(c), p, 256, None) == 1
+    # the running-maximum variant checks its arguments as thrift_attn_fwd does
+    assert L.thrift_attn_fwd_running_max(p, p, p, None, None, None, p, p, None, ctypes.byref(cfg(topk_bp=0)),
+                                         p, 256, None) == 1
+    assert L.thrift_attn_fwd_running_max(p, p, p, ctypes.byref(nv), ctypes.byref(nv), ctypes.byref(nv), None, p,
+                                         None, ctypes.byref(c), p, 256, None) == 1
+    nv1 = _lib.CNVFP4(0x1000, 0x1000, 0x1000, 0x1000, 1)
+    assert L.thrift_attn_fwd_running_max(p, p, p, ctypes.byref(nv), ctypes.byref(nv), ctypes.byref(nv1), p, p,
+                                         None, ctypes.byref(c), None, 0, None) == 5
 
 
 def dcfg(**kw):

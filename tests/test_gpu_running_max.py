@@ -1,0 +1,74 @@
+"""The running-maximum reading of the two-level P requantisation (thrift_attn_fwd_running_max;
+ThriftAttention "Twee-niveau P-herkwantisatie" after SageAttention3's scheme): the CUDA path against
+the oracle's reading R2 (first level = the row's running maximum in the kernel's visiting order,
+NVFP4 key blocks ascending then FP16 ones), to the same bar as thrift_attn_fwd against R1: rel-L2
+<= 1e-3, max-abs <= 1e-2 (one FP16 step where that is larger), LSE within 1e-3."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from test_gpu_parity import compare_attention, gpu_qkv, oracle_quant
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pab(cuda_device):
+    from precision_attention_block_b200 import build
+    build.build()
+    import precision_attention_block_b200 as pab
+    pab.load()
+    return pab
+
+
+def run_r2(pab, name, bp=None, n_units=None):
+    d = oracle_quant(name)
+    w = d["w"] if bp is None else d["w"].with_budget(bp)
+    gq, gk, gv = gpu_qkv(name)
+    cfg = pab.Config.from_workload(w)
+    q4, k4, v4 = pab.quantize_qkv(gq, gk, gv)
+    sel = pab.block_select(gq, gk, cfg)
+    out_g, lse_g = pab.attn_fwd(gq, gk, gv, q4, k4, v4, sel, cfg, running_max=True)
+    out_r1, _ = pab.attn_fwd(gq, gk, gv, q4, k4, v4, sel, cfg)
+    torch.cuda.synchronize()
+    scores = d["scores"] if bp is None else oracle.block_scores(d["q"], d["k"], w)
+    sel_o, _, _ = oracle.select(scores, w)
+    if n_units is None:
+        units = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.n_qb)]
+    else:
+        units = workloads.sample_units(w, n_units)
+    out_o, lse_o, _ = oracle.attn_r2(d["q"], d["k"], d["v"], d["q4"], d["k4"], d["v4"], sel_o, w, units=units)
+    compare_attention(out_g, lse_g, out_o, lse_o, w, units)
+    return out_g, out_r1
+
+
+@pytest.mark.parametrize("bp", [None, 0, 10000])
+def test_running_max_tiny(pab, bp):
+    run_r2(pab, "tiny", bp)
+
+
+@pytest.mark.parametrize("bp", [None, 0])
+def test_running_max_n4k(pab, bp):
+    out_g, out_r1 = run_r2(pab, "n4k", bp)
+    # the reading changes the result: NVFP4 blocks below the running maximum requantise differently
+    assert not torch.equal(out_g, out_r1)
+
+
+def test_running_max_all_fp16_equals_r1(pab):
+    """With every pair in FP16 the first level only shifts exp(S - m) before its FP16 rounding:
+    both readings stay within the output bar of each other (and of the same SDPA)."""
+    out_g, out_r1 = run_r2(pab, "n4k", 10000)
+    a, b = out_g.float().cpu().numpy(), out_r1.float().cpu().numpy()
+    assert np.linalg.norm(a - b) / np.linalg.norm(b) <= 1e-3
+
+
+@pytest.mark.parametrize("bp", [500, 2000])
+def test_running_max_diffusion_sampled(pab, bp):
+    run_r2(pab, "diffusion", bp, n_units=8)
+
+
+def test_running_max_prefill32k_sampled(pab):
+    run_r2(pab, "prefill32k", None, n_units=24)
