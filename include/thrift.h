@@ -23,6 +23,8 @@
  *     Errors that only the device can see (a bounded wait that ran out) are recorded in a
  *     status word inside the workspace and read with thrift_get_device_status.
  *   - Tensors are dense and row-major.  FP16 means IEEE binary16.
+ *   - Every tensor pointer (FP16 inputs and outputs, NVFP4 buffers) must be 16-byte aligned;
+ *     a misaligned one is rejected with THRIFT_ERR_INVALID_ARG.
  */
 #ifndef THRIFT_H
 #define THRIFT_H

@@ -1,9 +1,11 @@
 // The C ABI of libthrift (include/thrift.h): argument checks, workspace layout, launches on the
 // caller's stream.  The library allocates nothing; every buffer belongs to the caller.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/thrift.h"
 #include "../../include/thrift_debug.h"
@@ -16,19 +18,52 @@ thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const
                               void* out, float* out_hp, float* lse, int running_max, const thrift_cfg& c, int* status,
                               float* dbg, int dbg_entry, cudaStream_t stream);
 
+unsigned long long current_context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(ptr);
+    ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(ptr);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 int num_sms() {
+  // SM count of the current device, cached per device and context: a context created after
+  // cudaDeviceReset (or a green context with fewer SMs) is looked up afresh.
+  static std::mutex mu;
   static int cache[64] = {0};
+  static unsigned long long cache_ctx[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cache[dev] == 0) {
+  const unsigned long long ctx = current_context_id();
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0 || cache_ctx[dev] != ctx || ctx == 0) {
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
     cache[dev] = n;
+    cache_ctx[dev] = ctx;
   }
   return cache[dev];
 }
 
 namespace {
+
+bool al16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
 
 bool cfg_ok(const thrift_cfg* c) {
   if (!c) return false;
@@ -158,8 +193,6 @@ DecodeLayout decode_layout(const thrift_decode_cfg& c) {
   return L;
 }
 
-bool al16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
-
 thrift_status decode_attn_common(const void* q, const void* k, const void* v, const thrift_nvfp4* k4,
                                  const thrift_nvfp4* v4, const uint32_t* mask, void* out, float* lse,
                                  const thrift_decode_cfg* cfg, void* ws, size_t ws_bytes, cudaStream_t s,
@@ -242,6 +275,7 @@ thrift_status thrift_block_select(const void* q, const void* k, const thrift_cfg
   thrift_status st = cfg_supported(cfg);
   if (st != THRIFT_OK) return st;
   if (!q || !k || !mask || !counts || !lists) return THRIFT_ERR_INVALID_ARG;
+  if (!al16(q) || !al16(k)) return THRIFT_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, thrift_workspace_bytes(cfg))) return THRIFT_ERR_WORKSPACE;
   return select_launch(q, k, *cfg, mask, counts, lists, scores, static_cast<uint8_t*>(ws) + kWsHeader,
                        static_cast<cudaStream_t>(stream));
@@ -252,6 +286,7 @@ thrift_status thrift_block_select_noalloc(const void* q, const void* k, const th
   thrift_status st = cfg_supported(cfg);
   if (st != THRIFT_OK) return st;
   if (!q || !k || !mask || !counts || !lists) return THRIFT_ERR_INVALID_ARG;
+  if (!al16(q) || !al16(k)) return THRIFT_ERR_INVALID_ARG;
   if (select_layout(*cfg).bytes > noalloc_select_scratch_bytes()) return THRIFT_ERR_WORKSPACE;
   uint8_t* scratch = nullptr;
   if ((st = noalloc_select_scratch(&scratch)) != THRIFT_OK) return st;
@@ -268,6 +303,8 @@ static thrift_status attn_common(const void* q, const void* k, const void* v, co
   int mode = attn_mode(cfg);
   if (mode != 2 && (!nvfp4_ok(q4, 0) || !nvfp4_ok(k4, 0) || !nvfp4_ok(v4, 1))) return THRIFT_ERR_INVALID_ARG;
   if (mode != 1 && (!q || !k || !v)) return THRIFT_ERR_INVALID_ARG;
+  if (mode != 1 && (!al16(q) || !al16(k) || !al16(v))) return THRIFT_ERR_INVALID_ARG;
+  if (!al16(out) || (out_hp && !al16(out_hp))) return THRIFT_ERR_INVALID_ARG;
   if (mode == 0 && !mask) return THRIFT_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, kWsHeader)) return THRIFT_ERR_WORKSPACE;
   return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, out_hp, lse, running_max, *cfg, status_ptr(ws), dbg,
@@ -311,6 +348,7 @@ thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, 
   thrift_status st = cfg_supported(cfg);
   if (st != THRIFT_OK) return st;
   if (!q || !k || !v || !out) return THRIFT_ERR_INVALID_ARG;
+  if (!al16(q) || !al16(k) || !al16(v) || !al16(out)) return THRIFT_ERR_INVALID_ARG;
   AutoLayout L = auto_layout(*cfg);
   if (!ws_ok(ws, ws_bytes, L.bytes)) return THRIFT_ERR_WORKSPACE;
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -339,7 +377,7 @@ thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, 
 
 thrift_status thrift_kv_block_means(const void* k, int64_t outer, int32_t Nk, int32_t d, int32_t block_k,
                                     double* kbar, void* stream) {
-  if (!k || !kbar || outer <= 0 || Nk <= 0) return THRIFT_ERR_INVALID_ARG;
+  if (!k || !kbar || outer <= 0 || Nk <= 0 || !al16(k)) return THRIFT_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return THRIFT_ERR_UNSUPPORTED;
   if (block_k != 64 && block_k != 128) return THRIFT_ERR_UNSUPPORTED;
   if (Nk % block_k != 0 || outer > 65535) return THRIFT_ERR_UNSUPPORTED;

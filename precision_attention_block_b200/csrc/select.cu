@@ -6,10 +6,14 @@
 //           the block size (a power of two, exact).
 //   scores  float64 products and sums in the order c = 0 .. d-1 with no fused multiply-add, so
 //           every score is the correctly rounded result of one fixed evaluation order.
-//   top-k   one CTA per (batch, query head): a most-significant-digit-first radix select over
+//   top-k   per (batch, query head) a most-significant-digit-first radix select over
 //           order-preserving 64-bit keys finds the k-th largest score; keys above it are taken,
 //           ties at it are taken in index order (smaller i * nKb + j first) through a block scan.
+//           Long rows run on a cluster of CTAs that split the row into contiguous index ranges,
+//           hold their keys in shared memory and add up their digit histograms through
+//           distributed shared memory; short rows run on one CTA.
 //   lists   one thread per query block walks its mask words in ascending order.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -27,56 +31,113 @@ static __device__ __align__(256) uint8_t g_select_scratch[kNoAllocSelectScratchB
 
 namespace {
 
-// Block sums: one CTA per (batch*head, block); thread c sums column c over the block's tokens.
-__global__ void block_mean_kernel(const __half* __restrict__ x, int N, int d, int bs, double* __restrict__ mean) {
-  int64_t bh = blockIdx.y;
-  int blk = blockIdx.x;
+// Block sums: one CTA of 256 threads per (batch*head, block).  Sixteen lanes cover a token row
+// of d <= 128 halves with 16-byte loads (8 columns each) and the 16 row groups of the CTA stride
+// over the block's tokens; the partial sums meet in shared memory.  Every partial and total sum of
+// FP16 values here is exact in float64 (the block's |sum| stays below 2^23 on the 2^-24 grid of
+// FP16), so the order of the additions does not change the result.
+constexpr int kMeanThreads = 256;
+__global__ void __launch_bounds__(kMeanThreads) block_mean_kernel(const __half* __restrict__ x, int N, int d, int bs,
+                                                                  double* __restrict__ mean) {
+  __shared__ double part[kMeanThreads / 16][128];
+  const int64_t bh = blockIdx.y;
+  const int blk = blockIdx.x;
   const __half* base = x + (bh * N + (int64_t)blk * bs) * d;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+  const int lane16 = threadIdx.x & 15, grp = threadIdx.x >> 4;
+  const int c0 = lane16 * 8;  // first of this thread's 8 columns
+  double acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+  if (c0 < d) {
+    for (int t = grp; t < bs; t += kMeanThreads / 16) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)t * d + c0));
+      const __half2* h = reinterpret_cast<const __half2*>(&w);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(h[e]);
+        acc[2 * e] += (double)f.x;
+        acc[2 * e + 1] += (double)f.y;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[grp][c0 + e] = acc[e];
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < d; c += kMeanThreads) {
     double s = 0.0;
-    for (int t = 0; t < bs; ++t) s = __dadd_rn(s, (double)__half2float(base[(int64_t)t * d + c]));
+#pragma unroll
+    for (int g = 0; g < kMeanThreads / 16; ++g) s += part[g][c];
     mean[(bh * (N / bs) + blk) * d + c] = s / (double)bs;
   }
 }
 
-constexpr int kTileQ = 16, kTileK = 16;
-
-// Scores for a 16 x 16 tile of (query block, key block) pairs of one (batch, query head).
+// Scores of a 64 x 64 tile of (query block, key block) pairs of one (batch, query head): thread
+// (ty, tx) of 16 x 16 owns the 4 x 4 pairs (i0 + ty + 16a, j0 + tx + 16b), so each column step
+// reads 8 means from shared memory for 16 products.  Every score is the float64 sum in the order
+// c = 0 .. d-1 of the separately rounded products (no fused multiply-add); the columns are staged
+// 32 at a time and the sums carried across the chunks in registers, which keeps that order.
+// Tiles that lie entirely past the causal diagonal only write -inf.
+constexpr int kTileQ = 64, kTileK = 64, kScoreChunk = 32;
 __global__ void __launch_bounds__(256) block_score_kernel(const double* __restrict__ qbar,
                                                           const double* __restrict__ kbar, int Hq, int Hkv,
                                                           int nqb, int nkb, int d, int bq, int bk, int causal,
                                                           double* __restrict__ scores) {
-  extern __shared__ double sm[];
-  double* qs = sm;                          // [kTileQ][d+1]
-  double* ks = sm + kTileQ * (d + 1);       // [kTileK][d+1]
-  int bh = blockIdx.z;
-  int b = bh / Hq, h = bh % Hq, hk = h / (Hq / Hkv);
-  int i0 = blockIdx.y * kTileQ, j0 = blockIdx.x * kTileK;
+  __shared__ double qs[kTileQ][kScoreChunk + 1];
+  __shared__ double ks[kTileK][kScoreChunk + 1];
+  const int bh = blockIdx.z;
+  const int b = bh / Hq, h = bh % Hq, hk = h / (Hq / Hkv);
+  const int i0 = blockIdx.y * kTileQ, j0 = blockIdx.x * kTileK;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const double ninf = -__longlong_as_double(0x7ff0000000000000LL);
+  double* out = scores + ((int64_t)bh * nqb) * nkb;
+  const int i_last = min(nqb, i0 + kTileQ) - 1;
+  if (causal && (int64_t)j0 * bk > (int64_t)(i_last + 1) * bq - 1) {
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) {
+        const int i = i0 + ty + 16 * a, j = j0 + tx + 16 * bb;
+        if (i < nqb && j < nkb) out[(int64_t)i * nkb + j] = ninf;
+      }
+    return;
+  }
   const double* qb = qbar + ((int64_t)bh * nqb) * d;
   const double* kb = kbar + ((int64_t)(b * Hkv + hk) * nkb) * d;
-  for (int e = threadIdx.x; e < kTileQ * d; e += blockDim.x) {
-    int r = e / d, c = e % d;
-    qs[r * (d + 1) + c] = (i0 + r < nqb) ? qb[(int64_t)(i0 + r) * d + c] : 0.0;
+  double acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int bb = 0; bb < 4; ++bb) acc[a][bb] = 0.0;
+  for (int cc = 0; cc < d; cc += kScoreChunk) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < kTileQ * kScoreChunk; e += 256) {
+      const int r = e / kScoreChunk, c = e % kScoreChunk;
+      qs[r][c] = (i0 + r < nqb) ? __ldg(qb + (int64_t)(i0 + r) * d + cc + c) : 0.0;
+      ks[r][c] = (j0 + r < nkb) ? __ldg(kb + (int64_t)(j0 + r) * d + cc + c) : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int c = 0; c < kScoreChunk; ++c) {
+      double qv[4], kv[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) qv[a] = qs[ty + 16 * a][c];
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) kv[bb] = ks[tx + 16 * bb][c];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) acc[a][bb] = __dadd_rn(acc[a][bb], __dmul_rn(qv[a], kv[bb]));
+    }
   }
-  for (int e = threadIdx.x; e < kTileK * d; e += blockDim.x) {
-    int r = e / d, c = e % d;
-    ks[r * (d + 1) + c] = (j0 + r < nkb) ? kb[(int64_t)(j0 + r) * d + c] : 0.0;
-  }
-  __syncthreads();
-  int ii = threadIdx.x / kTileK, jj = threadIdx.x % kTileK;
-  int i = i0 + ii, j = j0 + jj;
-  if (i >= nqb || j >= nkb) return;
-  double out;
-  if (causal && (int64_t)j * bk > (int64_t)(i + 1) * bq - 1) {
-    out = -__longlong_as_double(0x7ff0000000000000LL);
-  } else {
-    double s = 0.0;
-    const double* qr = qs + ii * (d + 1);
-    const double* kr = ks + jj * (d + 1);
-    for (int c = 0; c < d; ++c) s = __dadd_rn(s, __dmul_rn(qr[c], kr[c]));
-    out = s;
-  }
-  scores[((int64_t)bh * nqb + i) * nkb + j] = out;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int bb = 0; bb < 4; ++bb) {
+      const int i = i0 + ty + 16 * a, j = j0 + tx + 16 * bb;
+      if (i >= nqb || j >= nkb) continue;
+      const bool valid = !causal || (int64_t)j * bk <= (int64_t)(i + 1) * bq - 1;
+      out[(int64_t)i * nkb + j] = valid ? acc[a][bb] : ninf;
+    }
 }
 
 // Order-preserving key of a score: larger score -> larger key; invalid (-inf) -> 0.
@@ -116,6 +177,14 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int& total
   return before;
 }
 
+// Adds a per-thread count into a shared 64-bit counter: a warp sum first, then one atomic per warp
+// (1024 same-address 64-bit shared atomics per block are slow).
+__device__ __forceinline__ void warp_add_u64(unsigned long long* ctr, unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0 && v) atomicAdd(ctr, v);
+}
+
 struct TopkShared {
   unsigned int hist[256];
   int warp_sums[32];
@@ -136,7 +205,7 @@ __device__ void topk_row(KeyAt key_at, int64_t n, int nkb, int topk_abs, int top
   __syncthreads();
   unsigned long long cnt = 0;
   for (int64_t t = threadIdx.x; t < n; t += THREADS) cnt += key_at(t) != 0ull;
-  atomicAdd(&sh.nvalid, cnt);
+  warp_add_u64(&sh.nvalid, cnt);
   __syncthreads();
   long long nvalid = (long long)sh.nvalid;
   long long k = topk_abs >= 0 ? (long long)topk_abs : ((long long)topk_bp * nvalid + 9999) / 10000;
@@ -150,23 +219,17 @@ __device__ void topk_row(KeyAt key_at, int64_t n, int nkb, int topk_abs, int top
     for (int b = threadIdx.x; b < 256; b += THREADS) sh.hist[b] = 0;
     __syncthreads();
     unsigned long long hi_mask = shift == 56 ? 0ull : (~0ull << (shift + 8));
-    if (shift >= 48) {
-      // the leading bytes (sign, exponent, top of the mantissa) are shared by most scores of a
-      // head, so most keys fall in the same few bins: one shared-memory atomic per distinct bin of
-      // a warp instead of one per key
-      for (int64_t base = 0; base < n; base += THREADS) {
-        const int64_t t = base + threadIdx.x;
-        const uint64_t key = t < n ? key_at(t) : 0ull;
-        const bool in = key != 0ull && (key & hi_mask) == prefix;
-        const int bin = in ? (int)((key >> shift) & 255) : -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, bin);
-        if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], (unsigned)__popc(peers));
-      }
-    } else {
-      for (int64_t t = threadIdx.x; t < n; t += THREADS) {
-        const uint64_t key = key_at(t);
-        if (key != 0ull && (key & hi_mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & 255], 1u);
-      }
+    // Neighbouring keys of a row are often close (the scores of one query block share most of
+    // their leading bytes), so a warp's keys tend to fall in the same bins: one shared-memory
+    // atomic per distinct bin of a warp instead of one per key (same-address atomics of a warp
+    // serialise).
+    for (int64_t base = 0; base < n; base += THREADS) {
+      const int64_t t = base + threadIdx.x;
+      const uint64_t key = t < n ? key_at(t) : 0ull;
+      const bool in = key != 0ull && (key & hi_mask) == prefix;
+      const int bin = in ? (int)((key >> shift) & 255) : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], (unsigned)__popc(peers));
     }
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -234,6 +297,257 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const double* __restrict_
     for (int64_t t = threadIdx.x; t < n; t += THREADS) keys_sm[t] = score_key(sc[t]);
   auto key_at = [&](int64_t t) -> uint64_t { return in_smem ? keys_sm[t] : score_key(sc[t]); };
   topk_row<THREADS>(key_at, n, nkb, topk_abs, topk_bp, mask_words, mk, sh);
+}
+
+// Top-k of long rows on a cluster of kTopkCluster CTAs per (batch, query head).  CTA r owns the
+// contiguous index range [r * chunk, (r + 1) * chunk) of the row and reads its scores from global
+// memory (L2) for every digit, four coalesced loads in flight per thread; with little shared memory
+// several clusters share an SM, so all heads run at once.  The radix select takes digits of 12, 12,
+// 12, 12, 12 and 4 bits from the top of the key.  For each digit a CTA counts its keys into a
+// shared-memory histogram, one atomic per distinct bin of a warp (neighbouring keys, one query
+// block's scores, mostly share their leading digits, and same-address atomics serialise), adds the
+// non-zero bins into the head's histogram of that digit in global memory (zeroed before the
+// launch), and after a cluster barrier every CTA reads the head's totals and takes the same
+// decision.  Keys above the k-th key are taken; its ties are taken in index order, CTA r taking the
+// first (need - ties held by the CTAs before it) of its own.
+constexpr int kTopkCluster = 8;
+constexpr int kTopkClusterThreads = 512;
+constexpr int kTopkBins = 4096;
+constexpr int kTopkDigits = 6;
+
+struct TopkClusterShared {
+  unsigned int hist[kTopkBins];
+  long long scan_part[32];
+  int warp_sums[32];
+  unsigned long long nvalid, nties;
+  unsigned long long prefix;
+  long long need;
+  long long bcast;
+};
+
+// Inclusive prefix sum of v over the block (thread order), 64-bit.
+template <int THREADS>
+__device__ __forceinline__ long long block_incl_scan_ll(long long v, long long* part) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) part[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = lane < THREADS / 32 ? part[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    part[lane] = w;
+  }
+  __syncthreads();
+  const long long r = x + (warp > 0 ? part[warp - 1] : 0);
+  __syncthreads();
+  return r;
+}
+
+__global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkClusterThreads, 3)
+    topk_cluster_kernel(const double* __restrict__ scores, int64_t n, int nkb, int topk_abs, int topk_bp,
+                        int mask_words, uint32_t* __restrict__ mask, unsigned int* __restrict__ ghist) {
+  namespace cg = cooperative_groups;
+  constexpr int THREADS = kTopkClusterThreads;
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = (int)cl.block_rank();
+  const int head = blockIdx.x / kTopkCluster;
+  __shared__ TopkClusterShared sh;
+  const double* sc = scores + (int64_t)head * n;
+  const int64_t chunk = (n + kTopkCluster - 1) / kTopkCluster;
+  const int64_t t0 = min(n, (int64_t)rank * chunk);
+  const int64_t m = min(n, t0 + chunk) - t0;
+  const int nqb = (int)(n / nkb);
+  uint32_t* mk = mask + (int64_t)head * nqb * mask_words;
+  unsigned int* gh = ghist + (int64_t)head * kTopkDigits * kTopkBins;
+  const int lane = threadIdx.x & 31;
+  auto key_at = [&](int64_t t) -> uint64_t { return score_key(__ldg(sc + t0 + t)); };
+  // sum of one 64-bit counter over the CTAs of ranks [0, upto): warp 0 reads one rank per lane
+  auto cluster_sum = [&](unsigned long long* local, int upto) -> long long {
+    if (threadIdx.x < 32) {
+      long long v = threadIdx.x < upto ? (long long)*cl.map_shared_rank(local, (int)threadIdx.x) : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (threadIdx.x == 0) sh.bcast = v;
+    }
+    __syncthreads();
+    const long long r = sh.bcast;
+    __syncthreads();
+    return r;
+  };
+
+  if (threadIdx.x == 0) {
+    sh.nvalid = 0;
+    sh.nties = 0;
+  }
+  __syncthreads();
+  unsigned long long prefix = 0ull;
+  long long need = 0;
+#pragma unroll 1
+  for (int p = 0; p < kTopkDigits; ++p) {
+    const int shift = p < 5 ? 52 - 12 * p : 0, width = p < 5 ? 12 : 4;
+    const unsigned int dmask = (1u << width) - 1u;
+    unsigned int* hist = sh.hist;
+    for (int b = threadIdx.x; b < kTopkBins; b += THREADS) hist[b] = 0;
+    __syncthreads();
+    const unsigned long long hi_mask = p == 0 ? 0ull : (~0ull << (shift + width));
+    unsigned long long valid = 0;
+    for (int64_t base = 0; base < m; base += 4 * THREADS) {
+      uint64_t kb[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int64_t t = base + e * THREADS + threadIdx.x;
+        kb[e] = t < m ? key_at(t) : 0ull;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint64_t key = kb[e];
+        valid += key != 0ull;
+        const bool in = key != 0ull && (key & hi_mask) == prefix;
+        const int bin = in ? (int)((key >> shift) & dmask) : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (unsigned)__popc(peers));
+      }
+    }
+    if (p == 0) warp_add_u64(&sh.nvalid, valid);
+    __syncthreads();
+    unsigned int* gp = gh + p * kTopkBins;
+    for (int b = threadIdx.x; b < kTopkBins; b += THREADS)
+      if (hist[b]) atomicAdd(&gp[b], hist[b]);
+    __threadfence();
+    cl.sync();
+    if (p == 0) {
+      const long long nvalid = cluster_sum(&sh.nvalid, kTopkCluster);
+      long long k = topk_abs >= 0 ? (long long)topk_abs : ((long long)topk_bp * nvalid + 9999) / 10000;
+      if (k > nvalid) k = nvalid;
+      if (k <= 0) {
+        cl.sync();  // no CTA leaves while another may still read its count
+        return;
+      }
+      need = k;
+    }
+    // the head's totals into the shared histogram, then thread t holds bins nb-1-8t .. nb-8-8t
+    // (descending); the thread whose inclusive count first reaches `need` finds the bin of the
+    // k-th key among its eight
+    constexpr int BPT = kTopkBins / THREADS;
+    const int nb = 1 << width;
+    for (int b = threadIdx.x; b < nb; b += THREADS) hist[b] = __ldcg(gp + b);
+    __syncthreads();
+    unsigned int tot[BPT];
+    const int b0 = nb - 1 - BPT * (int)threadIdx.x;
+    long long mine = 0;
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) {
+      tot[i] = b0 - i >= 0 ? hist[b0 - i] : 0u;
+      mine += tot[i];
+    }
+    const long long incl = block_incl_scan_ll<THREADS>(mine, sh.scan_part);
+    if (incl >= need && incl - mine < need) {
+      long long acc = incl - mine;
+      int i = 0;
+      for (; i < BPT - 1; ++i) {
+        if (acc + (long long)tot[i] >= need) break;
+        acc += tot[i];
+      }
+      sh.prefix = prefix | ((unsigned long long)(b0 - i) << shift);
+      sh.need = need - acc;
+    }
+    __syncthreads();
+    prefix = sh.prefix;
+    need = sh.need;
+  }
+  // every key of the CTA's range, four coalesced loads in flight per thread
+  auto for_keys = [&](auto&& f) {
+    for (int64_t base = 0; base < m; base += 4 * THREADS) {
+      uint64_t kb[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int64_t t = base + e * THREADS + threadIdx.x;
+        kb[e] = t < m ? key_at(t) : 0ull;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int64_t t = base + e * THREADS + threadIdx.x;
+        if (t < m) f(t, kb[e]);
+      }
+    }
+  };
+  // prefix is the k-th largest key; need = how many of its ties to take, in index order
+  unsigned long long ties = 0;
+  for_keys([&](int64_t, uint64_t key) { ties += key == prefix; });
+  warp_add_u64(&sh.nties, ties);
+  cl.sync();
+  const long long before_me = cluster_sum(&sh.nties, rank);
+  const long long my_ties = (long long)sh.nties;
+  const long long need_here = need - before_me;
+  auto take_at = [&](int64_t t) {
+    const int64_t g = t0 + t;
+    const int i = (int)(g / nkb), j = (int)(g % nkb);
+    atomicOr(&mk[(int64_t)i * mask_words + (j >> 5)], 1u << (j & 31));
+  };
+  if (need_here <= 0 || need_here >= my_ties) {
+    // none or all of this CTA's ties
+    const bool all_ties = need_here > 0;
+    for_keys([&](int64_t t, uint64_t key) {
+      if (key > prefix || (all_ties && key == prefix)) take_at(t);
+    });
+  } else {
+    long long taken_ties = 0;
+    for (int64_t base = 0; base < m; base += THREADS) {
+      const int64_t t = base + threadIdx.x;
+      const uint64_t key = t < m ? key_at(t) : 0ull;
+      const int tie = (key != 0ull && key == prefix) ? 1 : 0;
+      int total;
+      const int before = block_excl_scan<THREADS>(tie, sh.warp_sums, total);
+      if ((key > prefix) || (tie && (taken_ties + before) < need_here)) take_at(t);
+      taken_ties += total;
+    }
+  }
+  cl.sync();  // no CTA leaves while another may still read its counts
+}
+
+// Whether the cluster top-k can run on the current device: clusters of kTopkCluster CTAs with
+// `smem` bytes of dynamic shared memory each must fit (checked once per device and context).
+bool topk_cluster_ok(size_t smem) {
+  static std::mutex mu;
+  static unsigned long long ctx_seen[64] = {0};
+  static int ok_at[64] = {0};
+  static size_t smem_at[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const unsigned long long ctx = current_context_id();
+  std::lock_guard<std::mutex> lock(mu);
+  if (ctx != 0 && ctx_seen[dev] == ctx && smem_at[dev] == smem) return ok_at[dev] != 0;
+  int ok = 0;
+  if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+      cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kTopkCluster);
+    cfg.blockDim = dim3(kTopkClusterThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = kTopkCluster;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, topk_cluster_kernel, &cfg) == cudaSuccess && nclusters > 0) ok = 1;
+  }
+  (void)cudaGetLastError();  // a refused query leaves no error behind for the next launch check
+  ctx_seen[dev] = ctx;
+  ok_at[dev] = ok;
+  smem_at[dev] = smem;
+  return ok != 0;
 }
 
 constexpr int kListRowsPerCta = 8;
@@ -317,25 +631,31 @@ SelectLayout select_layout(const thrift_cfg& c) {
   L.qbar_off = 0;
   L.kbar_off = align256(L.qbar_off + (size_t)c.B * c.Hq * nqb * c.d * sizeof(double));
   L.scores_off = align256(L.kbar_off + (size_t)c.B * c.Hkv * nkb * c.d * sizeof(double));
-  L.bytes = align256(L.scores_off + (size_t)c.B * c.Hq * nqb * nkb * sizeof(double));
+  L.topk_hist_off = align256(L.scores_off + (size_t)c.B * c.Hq * nqb * nkb * sizeof(double));
+  // per (batch, query head): one histogram per radix digit of the cluster top-k
+  L.bytes = align256(L.topk_hist_off + (size_t)c.B * c.Hq * kTopkDigits * kTopkBins * sizeof(unsigned int));
   return L;
 }
 
 size_t noalloc_select_scratch_bytes() { return kNoAllocSelectScratchBytes; }
 
 // Device address of g_select_scratch on the current device.  In host code the array's name is
-// only a host-side stand-in, so the address comes from cudaGetSymbolAddress, looked up once per
-// device (with that device current) and cached.
+// only a host-side stand-in, so the address comes from cudaGetSymbolAddress, looked up with that
+// device current and cached per device and context: after cudaDeviceReset the module is loaded
+// into a new context, possibly at another address, and the lookup runs again.
 thrift_status noalloc_select_scratch(uint8_t** out) {
   static std::mutex mu;
   static void* cache[64] = {nullptr};
+  static unsigned long long cache_ctx[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return THRIFT_ERR_CUDA;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(mu);
-  if (!cache[dev]) {
+  if (!cache[dev] || ctx == 0 || cache_ctx[dev] != ctx) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_select_scratch) != cudaSuccess || !ptr) return THRIFT_ERR_CUDA;
     cache[dev] = ptr;
+    cache_ctx[dev] = current_context_id();  // the lookup made the primary context current if none was
   }
   *out = static_cast<uint8_t*>(cache[dev]);
   return THRIFT_OK;
@@ -349,19 +669,25 @@ thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, u
   double* qbar = reinterpret_cast<double*>(scratch + L.qbar_off);
   double* kbar = reinterpret_cast<double*>(scratch + L.kbar_off);
   double* scores = scores_out ? scores_out : reinterpret_cast<double*>(scratch + L.scores_off);
-  int tpb = c.d >= 128 ? 128 : c.d;
-  block_mean_kernel<<<dim3(nqb, c.B * c.Hq), tpb, 0, stream>>>(reinterpret_cast<const __half*>(q), c.N, c.d,
-                                                               c.block_q, qbar);
-  block_mean_kernel<<<dim3(nkb, c.B * c.Hkv), tpb, 0, stream>>>(reinterpret_cast<const __half*>(k), c.N, c.d,
-                                                                c.block_k, kbar);
-  size_t smem = (size_t)(kTileQ + kTileK) * (c.d + 1) * sizeof(double);
+  block_mean_kernel<<<dim3(nqb, c.B * c.Hq), kMeanThreads, 0, stream>>>(reinterpret_cast<const __half*>(q), c.N,
+                                                                         c.d, c.block_q, qbar);
+  block_mean_kernel<<<dim3(nkb, c.B * c.Hkv), kMeanThreads, 0, stream>>>(reinterpret_cast<const __half*>(k), c.N,
+                                                                          c.d, c.block_k, kbar);
   dim3 g((nkb + kTileK - 1) / kTileK, (nqb + kTileQ - 1) / kTileQ, c.B * c.Hq);
-  block_score_kernel<<<g, kTileQ * kTileK, smem, stream>>>(qbar, kbar, c.Hq, c.Hkv, nqb, nkb, c.d, c.block_q,
-                                                           c.block_k, c.causal, scores);
+  block_score_kernel<<<g, 256, 0, stream>>>(qbar, kbar, c.Hq, c.Hkv, nqb, nkb, c.d, c.block_q, c.block_k, c.causal,
+                                            scores);
   size_t mask_bytes = (size_t)c.B * c.Hq * nqb * mask_words * sizeof(uint32_t);
   if (cudaMemsetAsync(mask, 0, mask_bytes, stream) != cudaSuccess) return THRIFT_ERR_CUDA;
-  topk_kernel<kSelThreads><<<c.B * c.Hq, kSelThreads, 0, stream>>>(scores, (int64_t)nqb * nkb, nkb, c.topk_abs,
-                                                                    c.topk_bp, mask_words, mask);
+  const int64_t n = (int64_t)nqb * nkb;
+  if (n > kSelSmemKeys && topk_cluster_ok(0)) {
+    unsigned int* ghist = reinterpret_cast<unsigned int*>(scratch + L.topk_hist_off);
+    if (cudaMemsetAsync(ghist, 0, L.bytes - L.topk_hist_off, stream) != cudaSuccess) return THRIFT_ERR_CUDA;
+    topk_cluster_kernel<<<(unsigned)(c.B * c.Hq * kTopkCluster), kTopkClusterThreads, 0, stream>>>(
+        scores, n, nkb, c.topk_abs, c.topk_bp, mask_words, mask, ghist);
+  } else {
+    topk_kernel<kSelThreads><<<c.B * c.Hq, kSelThreads, 0, stream>>>(scores, n, nkb, c.topk_abs, c.topk_bp,
+                                                                      mask_words, mask);
+  }
   int64_t rows = (int64_t)c.B * c.Hq * nqb;
   lists_kernel<<<(unsigned)((rows + kListRowsPerCta - 1) / kListRowsPerCta), 32 * kListRowsPerCta, 0, stream>>>(
       mask, rows, nkb, mask_words, counts, lists);
@@ -370,9 +696,8 @@ thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, u
 
 thrift_status kv_means_launch(const void* k, int64_t outer, int32_t Nk, int32_t d, int32_t block_k, double* kbar,
                               cudaStream_t stream) {
-  int tpb = d >= 128 ? 128 : d;
-  block_mean_kernel<<<dim3(Nk / block_k, (unsigned)outer), tpb, 0, stream>>>(reinterpret_cast<const __half*>(k), Nk,
-                                                                             d, block_k, kbar);
+  block_mean_kernel<<<dim3(Nk / block_k, (unsigned)outer), kMeanThreads, 0, stream>>>(
+      reinterpret_cast<const __half*>(k), Nk, d, block_k, kbar);
   return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 

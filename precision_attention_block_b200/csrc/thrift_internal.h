@@ -13,13 +13,17 @@ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 int num_sms();
 
+// Unique id of the calling thread's current CUDA context (cuCtxGetId), 0 when none is current or
+// the driver cannot tell; per-device caches of context-bound values are keyed by it.
+unsigned long long current_context_id();
+
 // Workspace: [0, 256) status word and small scalars; then per-call scratch.
 constexpr size_t kWsHeader = 256;
 constexpr size_t kWsStatusOff = 0;    // int32 device status
 constexpr size_t kWsAmaxOff = 16;     // uint32 amax bits for the quantiser
 
 struct SelectLayout {
-  size_t qbar_off, kbar_off, scores_off, bytes;
+  size_t qbar_off, kbar_off, scores_off, topk_hist_off, bytes;
 };
 SelectLayout select_layout(const thrift_cfg& c);
 

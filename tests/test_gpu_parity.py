@@ -126,6 +126,51 @@ def test_select_exact(pab, name, bp):
     check_selection(d, w, sel, sel.scores)
 
 
+def _select_bits(sel_g, nkb):
+    mask = sel_g.mask.cpu().numpy().view(np.uint32)
+    return ((mask[..., :, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(*mask.shape[:-1], -1)[..., :nkb]
+
+
+@pytest.mark.parametrize("causal,bp", [(True, 500), (False, 500), (True, 5000)])
+def test_select_ties_in_index_order(pab, causal, bp):
+    """Every valid pair ties (constant Q and K): the k pairs taken are the first k valid ones in
+    index order i * nKb + j.  With 128 x 128 pairs per head the row is split over the CTAs of a
+    cluster, so the CTAs after the first must count the ties taken before them."""
+    w = workloads.Workload("ties", 95, 1, 2, 1, 8192, 64, causal, 64, 64, -1, bp, "normal")
+    q = np.full((1, 2, w.N, w.d), 0.25, np.float16)
+    k = np.full((1, 1, w.N, w.d), 0.5, np.float16)
+    s_o = oracle.block_scores(q, k, w)
+    sel_o, _, kc = oracle.select(s_o, w)
+    cfg = pab.Config.from_workload(w)
+    sel = pab.block_select(torch.from_numpy(q).cuda(), torch.from_numpy(k).cuda(), cfg, want_scores=True)
+    torch.cuda.synchronize()
+    bits = _select_bits(sel, w.n_kb)
+    assert np.array_equal(bits.astype(bool), sel_o.astype(bool))
+    flat = bits.reshape(2, -1)
+    valid = np.isfinite(s_o).reshape(2, -1)
+    for h in range(2):  # the first k valid indices, none after
+        idx = np.nonzero(valid[h])[0]
+        kk = int(flat[h].sum())
+        assert flat[h][idx[:kk]].all() and not flat[h][idx[kk:]].any()
+
+
+def test_select_exact_long131k(pab):
+    """Block scores and selection of the 131K prefill (1,048,576 pairs per head: the top-k CTAs
+    re-read their keys every radix pass instead of holding them in shared memory)."""
+    w = workloads.WORKLOADS["long131k"]
+    q, k, _ = workloads.make_qkv(w)
+    s_o = oracle.block_scores(q, k, w)
+    sel_o, _, _ = oracle.select(s_o, w)
+    cfg = pab.Config.from_workload(w)
+    sel = pab.block_select(torch.from_numpy(q).cuda(), torch.from_numpy(k).cuda(), cfg, want_scores=True)
+    torch.cuda.synchronize()
+    s_g = sel.scores.cpu().numpy()
+    fin = np.isfinite(s_o)
+    assert np.array_equal(np.isfinite(s_g), fin)
+    assert np.array_equal(s_g[fin], s_o[fin])
+    assert np.array_equal(_select_bits(sel, w.n_kb).astype(bool), sel_o.astype(bool))
+
+
 def compare_attention(out_g, lse_g, out_o, lse_o, w, units):
     og = out_g.cpu().numpy().astype(np.float64)
     lg = lse_g.cpu().numpy().astype(np.float64)
