@@ -100,7 +100,8 @@ bool ws_ok(const void* ws, size_t have, size_t need) {
 int* status_ptr(void* ws) { return reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + kWsStatusOff); }
 
 bool nvfp4_ok(const thrift_nvfp4* t, int axis) {
-  return t && t->codes && t->scales && t->scales_mma && t->tensor_scale && t->group_axis == axis;
+  return t && t->codes && t->scales && t->scales_mma && t->tensor_scale && t->group_axis == axis &&
+         al16(t->codes) && al16(t->scales) && al16(t->scales_mma) && reinterpret_cast<uintptr_t>(t->tensor_scale) % 4 == 0;
 }
 
 struct AutoLayout {

@@ -115,37 +115,58 @@ __global__ void __launch_bounds__(256) encode_rows_kernel(const uint4* __restric
   }
 }
 
-// Groups along tokens: one CTA per (outer index, 64-token tile); 256 threads.
+// Groups along tokens: one CTA per (outer index, 128-token tile); 256 threads.  The tile is staged
+// in shared memory; thread (c, part) quantises channel c's GPT consecutive 16-token groups, so
+// its codes (8 bytes per group), scales and tensor-core scales (one byte per group, consecutive
+// in both layouts) leave as one contiguous store each instead of one per group.
 template <int D>
 __global__ void __launch_bounds__(256) encode_cols_kernel(const __half* __restrict__ x, int N,
                                                           const unsigned int* __restrict__ amax_bits,
                                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                                                           uint8_t* __restrict__ scales_mma,
                                                           float* __restrict__ tensor_scale) {
-  __shared__ __align__(16) __half tile[64 * D];
-  float s_t = tensor_scale_from(*amax_bits);
+  constexpr int TOK = 128;
+  constexpr int PARTS = 256 / D;           // token parts per channel
+  constexpr int GPT = TOK / 16 / PARTS;    // groups per thread: 4 (D = 128) or 2 (D = 64)
+  __shared__ __align__(16) __half tile[TOK * D];
+  const float s_t = tensor_scale_from(*amax_bits);
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *tensor_scale = s_t;
-  int64_t o = blockIdx.y;
-  int t0 = blockIdx.x * 64;
+  const int64_t o = blockIdx.y;
+  const int t0 = blockIdx.x * TOK;
   const uint4* src = reinterpret_cast<const uint4*>(x + ((int64_t)o * N + t0) * D);
   uint4* dst = reinterpret_cast<uint4*>(tile);
-  constexpr int VECS = 64 * D / 8;
+  constexpr int VECS = TOK * D / 8;
 #pragma unroll
   for (int v = threadIdx.x; v < VECS; v += 256) dst[v] = __ldg(src + v);
   __syncthreads();
-  int64_t n_kblocks = N >> 6;
-  for (int p = threadIdx.x; p < 4 * D; p += 256) {
-    int c = p % D, g = p / D;
+  const int c = threadIdx.x % D, part = threadIdx.x / D;
+  const int g_first = part * GPT;  // first group of the thread within the tile
+  uint32_t cw[2 * GPT];
+  uint32_t sbs = 0;
+#pragma unroll
+  for (int gi = 0; gi < GPT; ++gi) {
+    const int g = g_first + gi;
     float f[16];
 #pragma unroll
     for (int t = 0; t < 16; ++t) f[t] = __half2float(tile[(g * 16 + t) * D + c]);
     uint2 packed;
-    uint32_t sb = quant16(f, s_t, packed);
-    int64_t row = o * D + c;
-    *reinterpret_cast<uint2*>(codes + row * (N / 2) + (t0 + g * 16) / 2) = packed;
-    int64_t grp = (t0 >> 4) + g;
-    scales[row * (N / 16) + grp] = (uint8_t)sb;
-    scales_mma[sf_mma_offset(row, grp, n_kblocks)] = (uint8_t)sb;
+    const uint32_t sb = quant16(f, s_t, packed);
+    cw[2 * gi] = packed.x;
+    cw[2 * gi + 1] = packed.y;
+    sbs |= sb << (8 * gi);
+  }
+  const int64_t row = o * D + c;
+  const int64_t grp0 = (t0 >> 4) + g_first;  // a multiple of GPT
+  uint8_t* cdst = codes + row * (N / 2) + grp0 * 8;
+  if constexpr (GPT == 4) {
+    reinterpret_cast<uint4*>(cdst)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    reinterpret_cast<uint4*>(cdst)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+    *reinterpret_cast<uint32_t*>(scales + row * (N / 16) + grp0) = sbs;
+    *reinterpret_cast<uint32_t*>(scales_mma + sf_mma_offset(row, grp0, N >> 6)) = sbs;
+  } else {
+    reinterpret_cast<uint4*>(cdst)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    *reinterpret_cast<uint16_t*>(scales + row * (N / 16) + grp0) = (uint16_t)sbs;
+    *reinterpret_cast<uint16_t*>(scales_mma + sf_mma_offset(row, grp0, N >> 6)) = (uint16_t)sbs;
   }
 }
 
@@ -302,7 +323,7 @@ thrift_status quantize_launch(const void* x, int64_t outer, int32_t N, int32_t d
         reinterpret_cast<const uint4*>(x), groups, d, amax_slot, reinterpret_cast<uint2*>(out->codes),
         out->scales, out->scales_mma, out->tensor_scale);
   } else {
-    dim3 grid(N / 64, (unsigned)outer);
+    dim3 grid(N / 128, (unsigned)outer);
     if (d == 128)
       encode_cols_kernel<128><<<grid, 256, 0, stream>>>(reinterpret_cast<const __half*>(x), N, amax_slot,
                                                          out->codes, out->scales, out->scales_mma,
