@@ -59,6 +59,17 @@ typedef struct {
   float softmax_scale;       /* tau; 0 selects 1/sqrt(d) rounded to FP32 */
 } thrift_cfg;
 
+/* Strides of an FP16 tensor viewed as [B, H, N, d] (batch, head, token, channel), in elements;
+ * the d channels of a token row are contiguous.  The dense layout is {H*N*d, N*d, d}; a tensor
+ * stored token-major as [B, N, H, d] (the usual output of a fused QKV projection) has
+ * {N*H*d, d, H*d}.  Every stride must be a non-negative multiple of 8 (16 bytes: the rows are
+ * moved by tensor copies) and n >= d; an output's rows must not overlap.  Entry points that take
+ * strides accept NULL for the dense layout.  NVFP4 copies, masks, lists, scores and lse are
+ * always dense. */
+typedef struct {
+  int64_t b, h, n;
+} thrift_strides;
+
 /* NVFP4 tensor view.  All pointers are device pointers owned by the caller.
  * For an FP16 tensor viewed as [outer, N, d]:
  *   group_axis 0 (Q, K): 16-element groups along d.
@@ -99,6 +110,14 @@ thrift_status thrift_quantize_nvfp4(const void* x, int64_t outer, int32_t N, int
                                     const thrift_nvfp4* out, void* ws, size_t ws_bytes,
                                     void* stream);
 
+/* thrift_quantize_nvfp4 of a strided [B, H, N, d] tensor (outer = B * H); the codes and scales
+ * are written in the dense layouts above.  Errors as thrift_quantize_nvfp4, plus
+ * THRIFT_ERR_INVALID_ARG for bad strides and THRIFT_ERR_UNSUPPORTED for B * H > 65535. */
+thrift_status thrift_quantize_nvfp4_strided(const void* x, const thrift_strides* xs, int32_t B,
+                                            int32_t H, int32_t N, int32_t d,
+                                            const thrift_nvfp4* out, void* ws, size_t ws_bytes,
+                                            void* stream);
+
 /* Block selection (ThriftAttention "Heuristische Blokkenselectie").
  * q: device FP16 [B,Hq,N,d]; k: device FP16 [B,Hkv,N,d].
  * Outputs (device):
@@ -129,6 +148,12 @@ thrift_status thrift_block_select(const void* q, const void* k, const thrift_cfg
 thrift_status thrift_block_select_noalloc(const void* q, const void* k, const thrift_cfg* cfg,
                                           uint32_t* mask, int32_t* counts, int16_t* lists,
                                           double* scores, void* stream);
+
+/* thrift_block_select with strided q [B,Hq,N,d] and k [B,Hkv,N,d] views (qs, ks; NULL = dense). */
+thrift_status thrift_block_select_strided(const void* q, const thrift_strides* qs, const void* k,
+                                          const thrift_strides* ks, const thrift_cfg* cfg,
+                                          uint32_t* mask, int32_t* counts, int16_t* lists,
+                                          double* scores, void* ws, size_t ws_bytes, void* stream);
 
 /* Attention forward (ThriftAttention "Gemengd-Precisie Berekening & Samenvoeging").
  * q, k, v: device FP16 [B,Hq,N,d], [B,Hkv,N,d], [B,Hkv,N,d] (used for the FP16 pairs);
@@ -161,6 +186,18 @@ thrift_status thrift_attn_fwd_qat(const void* q, const void* k, const void* v,
                                   const thrift_nvfp4* v4, const uint32_t* mask, void* out,
                                   float* out_hp, float* lse, const thrift_cfg* cfg, void* ws,
                                   size_t ws_bytes, void* stream);
+
+/* thrift_attn_fwd with strided FP16 operands and output: q, k, v and out are [B,H,N,d] views
+ * with strides qs, ks, vs, os (NULL = dense); the FP16 tiles are fetched through 4-D tensor maps,
+ * so the layout costs nothing in the kernel.  q4, k4, v4, mask and lse are dense.  Arguments and
+ * errors otherwise as thrift_attn_fwd (mask only). */
+thrift_status thrift_attn_fwd_strided(const void* q, const thrift_strides* qs, const void* k,
+                                      const thrift_strides* ks, const void* v,
+                                      const thrift_strides* vs, const thrift_nvfp4* q4,
+                                      const thrift_nvfp4* k4, const thrift_nvfp4* v4,
+                                      const uint32_t* mask, void* out, const thrift_strides* os,
+                                      float* lse, const thrift_cfg* cfg, void* ws, size_t ws_bytes,
+                                      void* stream);
 
 /* thrift_attn_fwd with the other reading of the two-level P requantisation (ThriftAttention
  * "Twee-niveau P-herkwantisatie", which follows SageAttention3's two-level scheme).
@@ -195,6 +232,16 @@ size_t thrift_auto_workspace_bytes(const thrift_cfg* cfg);
 thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, void* out,
                                    float* lse, const thrift_cfg* cfg, void* ws,
                                    size_t ws_bytes, void* stream);
+
+/* thrift_attn_fwd_auto with strided q, k, v and out ([B,H,N,d] views, NULL = dense): the whole
+ * path reads the inputs and writes the output in their own layouts; the NVFP4 copies and the
+ * selection in the workspace stay dense. */
+thrift_status thrift_attn_fwd_auto_strided(const void* q, const thrift_strides* qs, const void* k,
+                                           const thrift_strides* ks, const void* v,
+                                           const thrift_strides* vs, void* out,
+                                           const thrift_strides* os, float* lse,
+                                           const thrift_cfg* cfg, void* ws, size_t ws_bytes,
+                                           void* stream);
 
 /* ------------------------------------------------------------------ decode
  *

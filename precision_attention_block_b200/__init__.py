@@ -137,10 +137,25 @@ class Workspace:
         return cls(n, device)
 
 
+def _strides(t: Optional[torch.Tensor]):
+    """thrift_strides of a [B, H, N, d] view (None when dense): a token-major [B, N, H, d] tensor
+    passed as t.transpose(1, 2) reaches the kernels without a copy."""
+    if t is None or t.is_contiguous():
+        return None
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError("strided tensors must be [B, H, N, d] views with contiguous d")
+    return _lib.CStrides(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _sref(st):
+    return None if st is None else ctypes.byref(st)
+
+
 def quantize_nvfp4(x: torch.Tensor, group_axis: int, out: Optional[NVFP4Tensor] = None,
                    ws: Optional[Workspace] = None) -> NVFP4Tensor:
-    """NVFP4 quantisation of a contiguous FP16 [.., N, d] CUDA tensor (thrift_quantize_nvfp4)."""
-    assert x.is_cuda and x.dtype == torch.float16 and x.is_contiguous()
+    """NVFP4 quantisation of an FP16 [.., N, d] CUDA tensor (thrift_quantize_nvfp4), or of a
+    strided [B, H, N, d] view (thrift_quantize_nvfp4_strided)."""
+    assert x.is_cuda and x.dtype == torch.float16
     *lead, N, d = x.shape
     outer = 1
     for s in lead:
@@ -150,6 +165,12 @@ def quantize_nvfp4(x: torch.Tensor, group_axis: int, out: Optional[NVFP4Tensor] 
     if ws is None:
         ws = Workspace(256, x.device)
     c = out.c()
+    st = _strides(x)
+    if st is not None:
+        check(load().thrift_quantize_nvfp4_strided(_ptr(x), ctypes.byref(st), x.shape[0], x.shape[1], N, d,
+                                                   ctypes.byref(c), ws.ptr, ws.nbytes, _stream()),
+              "thrift_quantize_nvfp4_strided")
+        return out
     check(load().thrift_quantize_nvfp4(_ptr(x), outer, N, d, ctypes.byref(c), ws.ptr, ws.nbytes, _stream()),
           "thrift_quantize_nvfp4")
     return out
@@ -176,6 +197,13 @@ def block_select(q: torch.Tensor, k: torch.Tensor, cfg: Config, ws: Optional[Wor
     if ws is None:
         ws = Workspace.for_config(cfg, dev)
     c = cfg.c()
+    qs, ks = _strides(q), _strides(k)
+    if qs is not None or ks is not None:
+        check(load().thrift_block_select_strided(_ptr(q), _sref(qs), _ptr(k), _sref(ks), ctypes.byref(c),
+                                                 _ptr(out.mask), _ptr(out.counts), _ptr(out.lists),
+                                                 _ptr(out.scores), ws.ptr, ws.nbytes, _stream()),
+              "thrift_block_select_strided")
+        return out
     check(load().thrift_block_select(_ptr(q), _ptr(k), ctypes.byref(c), _ptr(out.mask), _ptr(out.counts),
                                      _ptr(out.lists), _ptr(out.scores), ws.ptr, ws.nbytes, _stream()),
           "thrift_block_select")
@@ -200,6 +228,16 @@ def attn_fwd(q, k, v, q4: Optional[NVFP4Tensor], k4: Optional[NVFP4Tensor], v4: 
     c = cfg.c()
     n4 = [None if t is None else t.c() for t in (q4, k4, v4)]
     refs = [None if t is None else ctypes.byref(t) for t in n4]
+    strided = [_strides(t) for t in (q, k, v, out)]
+    if any(st is not None for st in strided):
+        if running_max:
+            raise ValueError("the running-maximum variant takes dense tensors")
+        qs, ks, vs, os_ = strided
+        check(load().thrift_attn_fwd_strided(_ptr(q), _sref(qs), _ptr(k), _sref(ks), _ptr(v), _sref(vs),
+                                             refs[0], refs[1], refs[2], None if sel is None else _ptr(sel.mask),
+                                             _ptr(out), _sref(os_), _ptr(lse), ctypes.byref(c), ws.ptr, ws.nbytes,
+                                             _stream()), "thrift_attn_fwd_strided")
+        return out, lse
     if running_max:
         check(load().thrift_attn_fwd_running_max(_ptr(q), _ptr(k), _ptr(v), refs[0], refs[1], refs[2],
                                                  None if sel is None else _ptr(sel.mask), _ptr(out), _ptr(lse),
@@ -271,6 +309,13 @@ def attn_fwd_auto(q, k, v, cfg: Config, out=None, lse=None, ws: Optional[Workspa
     if ws is None:
         ws = Workspace.for_config(cfg, dev, auto=True)
     c = cfg.c()
+    strided = [_strides(t) for t in (q, k, v, out)]
+    if any(st is not None for st in strided):
+        qs, ks, vs, os_ = strided
+        check(load().thrift_attn_fwd_auto_strided(_ptr(q), _sref(qs), _ptr(k), _sref(ks), _ptr(v), _sref(vs),
+                                                  _ptr(out), _sref(os_), _ptr(lse), ctypes.byref(c), ws.ptr,
+                                                  ws.nbytes, _stream()), "thrift_attn_fwd_auto_strided")
+        return out, lse
     check(load().thrift_attn_fwd_auto(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), ctypes.byref(c),
                                       ws.ptr, ws.nbytes, _stream()), "thrift_attn_fwd_auto")
     return out, lse

@@ -43,6 +43,10 @@ class CDecodeCfg(ctypes.Structure):
                 ("softmax_scale", ctypes.c_float), ("n_valid", ctypes.c_int32)]
 
 
+class CStrides(ctypes.Structure):
+    _fields_ = [("b", ctypes.c_int64), ("h", ctypes.c_int64), ("n", ctypes.c_int64)]
+
+
 class CNVFP4(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("scales_mma", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p),
@@ -59,6 +63,7 @@ _i64 = ctypes.c_int64
 _cfgp = ctypes.POINTER(CCfg)
 _nvp = ctypes.POINTER(CNVFP4)
 _dcfgp = ctypes.POINTER(CDecodeCfg)
+_stp = ctypes.POINTER(CStrides)
 
 SIGNATURES = {
     "thrift_nvfp4_scales_mma_bytes": (_sz, [_i64, _i32, _i32, _i32]),
@@ -74,6 +79,12 @@ SIGNATURES = {
                                            _vp]),
     "thrift_attn_fwd_running_max": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _nvp, _vp, _vp, _vp, _cfgp, _vp,
                                                    _sz, _vp]),
+    "thrift_quantize_nvfp4_strided": (ctypes.c_int, [_vp, _stp, _i32, _i32, _i32, _i32, _nvp, _vp, _sz, _vp]),
+    "thrift_block_select_strided": (ctypes.c_int, [_vp, _stp, _vp, _stp, _cfgp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "thrift_attn_fwd_strided": (ctypes.c_int, [_vp, _stp, _vp, _stp, _vp, _stp, _nvp, _nvp, _nvp, _vp, _vp, _stp,
+                                               _vp, _cfgp, _vp, _sz, _vp]),
+    "thrift_attn_fwd_auto_strided": (ctypes.c_int, [_vp, _stp, _vp, _stp, _vp, _stp, _vp, _stp, _vp, _cfgp, _vp,
+                                                    _sz, _vp]),
     "thrift_kv_block_means": (ctypes.c_int, [_vp, _i64, _i32, _i32, _i32, _vp, _vp]),
     "thrift_nvfp4_tensor_scale": (ctypes.c_int, [_vp, _i64, _vp, _vp, _sz, _vp]),
     "thrift_kv_append": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _nvp, _nvp, _vp,

@@ -16,7 +16,7 @@ namespace thrift {
 thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
                               const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
                               void* out, float* out_hp, float* lse, int running_max, const thrift_cfg& c, int* status,
-                              float* dbg, int dbg_entry, cudaStream_t stream);
+                              float* dbg, int dbg_entry, cudaStream_t stream, const AttnRows* rows = nullptr);
 
 unsigned long long current_context_id() {
   typedef CUresult (*GetCurrentFn)(CUcontext*);
@@ -64,6 +64,18 @@ int num_sms() {
 namespace {
 
 bool al16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
+
+// Strides of a [B, H, N, d] view: non-negative multiples of 8 elements (16 bytes, what the tensor
+// copies need), token rows at least d apart; NULL is the dense layout.
+bool strides_ok(const thrift_strides* s, int d) {
+  if (!s) return true;
+  if (s->b < 0 || s->h < 0 || s->n < d) return false;
+  return s->b % 8 == 0 && s->h % 8 == 0 && s->n % 8 == 0;
+}
+
+RowMap rows_of(const thrift_strides* s, int H, int N, int d) {
+  return s ? RowMap{s->b, s->h, s->n, H} : dense_rows(H, N, d);
+}
 
 bool cfg_ok(const thrift_cfg* c) {
   if (!c) return false;
@@ -214,7 +226,7 @@ thrift_status decode_attn_common(const void* q, const void* k, const void* v, co
   const thrift_decode_cfg& c = *cfg;
   if (mode <= 1) {
     unsigned int* amax = reinterpret_cast<unsigned int*>(w + kWsAmaxOff);
-    thrift_status st = quantize_launch(q, (int64_t)c.B * c.Hq, c.Nq, c.d, &q4, amax, s);
+    thrift_status st = quantize_launch(q, dense_rows(c.Hq, c.Nq, c.d), (int64_t)c.B * c.Hq, c.Nq, c.d, &q4, amax, s);
     if (st != THRIFT_OK) return st;
   }
   DecodeArgs a;
@@ -257,29 +269,49 @@ size_t thrift_auto_workspace_bytes(const thrift_cfg* cfg) {
   return auto_layout(*cfg).bytes;
 }
 
-thrift_status thrift_quantize_nvfp4(const void* x, int64_t outer, int32_t N, int32_t d, const thrift_nvfp4* out,
-                                    void* ws, size_t ws_bytes, void* stream) {
-  if (!x || outer <= 0 || N <= 0 || !out) return THRIFT_ERR_INVALID_ARG;
+static thrift_status quantize_common(const void* x, const thrift_strides* xs, int64_t outer, int32_t H, int32_t N,
+                                     int32_t d, const thrift_nvfp4* out, void* ws, size_t ws_bytes, void* stream) {
+  if (!x || outer <= 0 || N <= 0 || !out || H <= 0 || outer % H != 0) return THRIFT_ERR_INVALID_ARG;
   if (out->group_axis != 0 && out->group_axis != 1) return THRIFT_ERR_INVALID_ARG;
   if (!nvfp4_ok(out, out->group_axis)) return THRIFT_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return THRIFT_ERR_UNSUPPORTED;
   if (N % 128 != 0) return THRIFT_ERR_UNSUPPORTED;
-  if (reinterpret_cast<uintptr_t>(x) % 16 != 0) return THRIFT_ERR_INVALID_ARG;
+  if ((xs || out->group_axis == 1) && outer > 65535) return THRIFT_ERR_UNSUPPORTED;  // grid rows per slice
+  if (!al16(x) || !strides_ok(xs, d)) return THRIFT_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, kWsHeader)) return THRIFT_ERR_WORKSPACE;
   unsigned int* amax = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + kWsAmaxOff);
-  return quantize_launch(x, outer, N, d, out, amax, static_cast<cudaStream_t>(stream));
+  return quantize_launch(x, rows_of(xs, H, N, d), outer, N, d, out, amax, static_cast<cudaStream_t>(stream));
+}
+
+thrift_status thrift_quantize_nvfp4(const void* x, int64_t outer, int32_t N, int32_t d, const thrift_nvfp4* out,
+                                    void* ws, size_t ws_bytes, void* stream) {
+  return quantize_common(x, nullptr, outer, 1, N, d, out, ws, ws_bytes, stream);
+}
+
+thrift_status thrift_quantize_nvfp4_strided(const void* x, const thrift_strides* xs, int32_t B, int32_t H, int32_t N,
+                                            int32_t d, const thrift_nvfp4* out, void* ws, size_t ws_bytes,
+                                            void* stream) {
+  if (B <= 0 || H <= 0) return THRIFT_ERR_INVALID_ARG;
+  return quantize_common(x, xs, (int64_t)B * H, H, N, d, out, ws, ws_bytes, stream);
+}
+
+thrift_status thrift_block_select_strided(const void* q, const thrift_strides* qs, const void* k,
+                                          const thrift_strides* ks, const thrift_cfg* cfg, uint32_t* mask,
+                                          int32_t* counts, int16_t* lists, double* scores, void* ws, size_t ws_bytes,
+                                          void* stream) {
+  thrift_status st = cfg_supported(cfg);
+  if (st != THRIFT_OK) return st;
+  if (!q || !k || !mask || !counts || !lists) return THRIFT_ERR_INVALID_ARG;
+  if (!al16(q) || !al16(k) || !strides_ok(qs, cfg->d) || !strides_ok(ks, cfg->d)) return THRIFT_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, thrift_workspace_bytes(cfg))) return THRIFT_ERR_WORKSPACE;
+  return select_launch(q, rows_of(qs, cfg->Hq, cfg->N, cfg->d), k, rows_of(ks, cfg->Hkv, cfg->N, cfg->d), *cfg, mask,
+                       counts, lists, scores, static_cast<uint8_t*>(ws) + kWsHeader, static_cast<cudaStream_t>(stream));
 }
 
 thrift_status thrift_block_select(const void* q, const void* k, const thrift_cfg* cfg, uint32_t* mask,
                                   int32_t* counts, int16_t* lists, double* scores, void* ws, size_t ws_bytes,
                                   void* stream) {
-  thrift_status st = cfg_supported(cfg);
-  if (st != THRIFT_OK) return st;
-  if (!q || !k || !mask || !counts || !lists) return THRIFT_ERR_INVALID_ARG;
-  if (!al16(q) || !al16(k)) return THRIFT_ERR_INVALID_ARG;
-  if (!ws_ok(ws, ws_bytes, thrift_workspace_bytes(cfg))) return THRIFT_ERR_WORKSPACE;
-  return select_launch(q, k, *cfg, mask, counts, lists, scores, static_cast<uint8_t*>(ws) + kWsHeader,
-                       static_cast<cudaStream_t>(stream));
+  return thrift_block_select_strided(q, nullptr, k, nullptr, cfg, mask, counts, lists, scores, ws, ws_bytes, stream);
 }
 
 thrift_status thrift_block_select_noalloc(const void* q, const void* k, const thrift_cfg* cfg, uint32_t* mask,
@@ -291,15 +323,27 @@ thrift_status thrift_block_select_noalloc(const void* q, const void* k, const th
   if (select_layout(*cfg).bytes > noalloc_select_scratch_bytes()) return THRIFT_ERR_WORKSPACE;
   uint8_t* scratch = nullptr;
   if ((st = noalloc_select_scratch(&scratch)) != THRIFT_OK) return st;
-  return select_launch(q, k, *cfg, mask, counts, lists, scores, scratch, static_cast<cudaStream_t>(stream));
+  const thrift_cfg& c = *cfg;
+  return select_launch(q, dense_rows(c.Hq, c.N, c.d), k, dense_rows(c.Hkv, c.N, c.d), c, mask, counts, lists, scores,
+                       scratch, static_cast<cudaStream_t>(stream));
 }
 
 static thrift_status attn_common(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
                                  const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, void* out,
                                  float* out_hp, float* lse, int running_max, const thrift_cfg* cfg, void* ws,
-                                 size_t ws_bytes, float* dbg, int dbg_entry, void* stream) {
+                                 size_t ws_bytes, float* dbg, int dbg_entry, void* stream,
+                                 const thrift_strides* qs = nullptr, const thrift_strides* ks = nullptr,
+                                 const thrift_strides* vs = nullptr, const thrift_strides* os = nullptr) {
   thrift_status st = cfg_supported(cfg);
   if (st != THRIFT_OK) return st;
+  const int d = cfg->d;
+  if (!strides_ok(qs, d) || !strides_ok(ks, d) || !strides_ok(vs, d) || !strides_ok(os, d))
+    return THRIFT_ERR_INVALID_ARG;
+  AttnRows rows;
+  rows.q = rows_of(qs, cfg->Hq, cfg->N, d);
+  rows.k = rows_of(ks, cfg->Hkv, cfg->N, d);
+  rows.v = rows_of(vs, cfg->Hkv, cfg->N, d);
+  rows.out = rows_of(os, cfg->Hq, cfg->N, d);
   if (!out) return THRIFT_ERR_INVALID_ARG;
   int mode = attn_mode(cfg);
   if (mode != 2 && (!nvfp4_ok(q4, 0) || !nvfp4_ok(k4, 0) || !nvfp4_ok(v4, 1))) return THRIFT_ERR_INVALID_ARG;
@@ -309,7 +353,7 @@ static thrift_status attn_common(const void* q, const void* k, const void* v, co
   if (mode == 0 && !mask) return THRIFT_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, kWsHeader)) return THRIFT_ERR_WORKSPACE;
   return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, out_hp, lse, running_max, *cfg, status_ptr(ws), dbg,
-                         dbg_entry, static_cast<cudaStream_t>(stream));
+                         dbg_entry, static_cast<cudaStream_t>(stream), &rows);
 }
 
 thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
@@ -319,6 +363,15 @@ thrift_status thrift_attn_fwd(const void* q, const void* k, const void* v, const
   (void)counts;
   (void)lists;
   return attn_common(q, k, v, q4, k4, v4, mask, out, nullptr, lse, 0, cfg, ws, ws_bytes, nullptr, -1, stream);
+}
+
+thrift_status thrift_attn_fwd_strided(const void* q, const thrift_strides* qs, const void* k, const thrift_strides* ks,
+                                      const void* v, const thrift_strides* vs, const thrift_nvfp4* q4,
+                                      const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, void* out,
+                                      const thrift_strides* os, float* lse, const thrift_cfg* cfg, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  return attn_common(q, k, v, q4, k4, v4, mask, out, nullptr, lse, 0, cfg, ws, ws_bytes, nullptr, -1, stream, qs, ks,
+                     vs, os);
 }
 
 thrift_status thrift_attn_fwd_running_max(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
@@ -346,10 +399,20 @@ thrift_status thrift_debug_attn_dump(const void* q, const void* k, const void* v
 
 thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, void* out, float* lse,
                                    const thrift_cfg* cfg, void* ws, size_t ws_bytes, void* stream) {
+  return thrift_attn_fwd_auto_strided(q, nullptr, k, nullptr, v, nullptr, out, nullptr, lse, cfg, ws, ws_bytes,
+                                      stream);
+}
+
+thrift_status thrift_attn_fwd_auto_strided(const void* q, const thrift_strides* qs, const void* k,
+                                           const thrift_strides* ks, const void* v, const thrift_strides* vs,
+                                           void* out, const thrift_strides* os, float* lse, const thrift_cfg* cfg,
+                                           void* ws, size_t ws_bytes, void* stream) {
   thrift_status st = cfg_supported(cfg);
   if (st != THRIFT_OK) return st;
   if (!q || !k || !v || !out) return THRIFT_ERR_INVALID_ARG;
   if (!al16(q) || !al16(k) || !al16(v) || !al16(out)) return THRIFT_ERR_INVALID_ARG;
+  if (!strides_ok(qs, cfg->d) || !strides_ok(ks, cfg->d) || !strides_ok(vs, cfg->d) || !strides_ok(os, cfg->d))
+    return THRIFT_ERR_INVALID_ARG;
   AutoLayout L = auto_layout(*cfg);
   if (!ws_ok(ws, ws_bytes, L.bytes)) return THRIFT_ERR_WORKSPACE;
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -361,19 +424,24 @@ thrift_status thrift_attn_fwd_auto(const void* q, const void* k, const void* v, 
   unsigned int* amax = reinterpret_cast<unsigned int*>(w + kWsAmaxOff);
   int mode = attn_mode(cfg);
   const thrift_cfg& c = *cfg;
+  AttnRows rows;
+  rows.q = rows_of(qs, c.Hq, c.N, c.d);
+  rows.k = rows_of(ks, c.Hkv, c.N, c.d);
+  rows.v = rows_of(vs, c.Hkv, c.N, c.d);
+  rows.out = rows_of(os, c.Hq, c.N, c.d);
   if (mode != 2) {
-    if ((st = quantize_launch(q, (int64_t)c.B * c.Hq, c.N, c.d, &q4, amax, s)) != THRIFT_OK) return st;
-    if ((st = quantize_launch(k, (int64_t)c.B * c.Hkv, c.N, c.d, &k4, amax, s)) != THRIFT_OK) return st;
-    if ((st = quantize_launch(v, (int64_t)c.B * c.Hkv, c.N, c.d, &v4, amax, s)) != THRIFT_OK) return st;
+    if ((st = quantize_launch(q, rows.q, (int64_t)c.B * c.Hq, c.N, c.d, &q4, amax, s)) != THRIFT_OK) return st;
+    if ((st = quantize_launch(k, rows.k, (int64_t)c.B * c.Hkv, c.N, c.d, &k4, amax, s)) != THRIFT_OK) return st;
+    if ((st = quantize_launch(v, rows.v, (int64_t)c.B * c.Hkv, c.N, c.d, &v4, amax, s)) != THRIFT_OK) return st;
   }
   uint32_t* mask = reinterpret_cast<uint32_t*>(w + L.mask);
   if (mode == 0) {
-    st = select_launch(q, k, c, mask, reinterpret_cast<int32_t*>(w + L.counts), reinterpret_cast<int16_t*>(w + L.lists),
-                       nullptr, w + L.select, s);
+    st = select_launch(q, rows.q, k, rows.k, c, mask, reinterpret_cast<int32_t*>(w + L.counts),
+                       reinterpret_cast<int16_t*>(w + L.lists), nullptr, w + L.select, s);
     if (st != THRIFT_OK) return st;
   }
   return attn_launch_dbg(q, k, v, &q4, &k4, &v4, mode == 0 ? mask : nullptr, mode, out, nullptr, lse, 0, c,
-                         status_ptr(ws), nullptr, -1, s);
+                         status_ptr(ws), nullptr, -1, s, &rows);
 }
 
 thrift_status thrift_kv_block_means(const void* k, int64_t outer, int32_t Nk, int32_t d, int32_t block_k,

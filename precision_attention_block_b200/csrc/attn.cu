@@ -126,6 +126,7 @@ struct AttnParams {
   const float* k_ts;
   const float* v_ts;
   __half* out;
+  long long osb, osh, osn;  // output strides in elements ([B, Hq, N, d] view, d contiguous)
   float* out_hp;  // optional FP32 copy of the output before its FP16 rounding (Attn-QAT's O')
   float* lse;
   int* status;
@@ -503,7 +504,8 @@ __global__ void __launch_bounds__(384, 1)
               uint8_t* sq = smem + L::OFF_Q16;
               mbar_arrive_expect_tx(&bars->q16_full, L::Q16_BYTES);
 #pragma unroll
-              for (int cb = 0; cb < D / 64; ++cb) tma_load_2d(sq + cb * kBQ * 128, &tm_q16, &bars->q16_full, cb * 64, qrow0);
+              for (int cb = 0; cb < D / 64; ++cb)
+                tma_load_4d(sq + cb * kBQ * 128, &tm_q16, &bars->q16_full, cb * 64, ui.t * kBQ, ui.h, ui.b);
               q16_loaded = true;
             }
             int pg, ph;
@@ -515,7 +517,8 @@ __global__ void __launch_bounds__(384, 1)
                 mbar_arrive_expect_tx(&bars->page_full[pg], L::K16_BYTES);
 #pragma unroll
                 for (int cb = 0; cb < D / 64; ++cb)
-                  tma_load_2d(dst + cb * BK * 128, kv ? &tm_v16 : &tm_k16, &bars->page_full[pg], cb * 64, krow0);
+                  tma_load_4d(dst + cb * BK * 128, kv ? &tm_v16 : &tm_k16, &bars->page_full[pg], cb * 64, j * BK,
+                              ui.hk, ui.b);
               }
             } else {
               ring.next(pg, ph);
@@ -918,7 +921,7 @@ __global__ void __launch_bounds__(384, 1)
       const float l_tot = bars->lx[lb][0][rr] + bars->lx[lb][1][rr];
       const float inv_l = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
       const int64_t orow = (int64_t)(ui.b * p.Hq + ui.h) * p.N + row;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D + wg * DH);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + ui.b * p.osb + ui.h * p.osh + row * p.osn + wg * DH);
 #pragma unroll
       for (int c = 0; c < DH / 8; ++c) {
         uint4 v;
@@ -964,6 +967,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// 4D map over an FP16 [B, H, N, D] tensor with row strides `rows` (D contiguous), boxes of 64
+// channels x box_rows tokens of one (batch, head).
+bool make_map4(CUtensorMap* m, const void* base, const RowMap& rows, int B, int H, int N, int D, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)rows.sn * 2, (cuuint64_t)rows.sh * 2, (cuuint64_t)rows.sb * 2};
+  cuuint32_t box[4] = {64, box_rows, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2D map over a row-major [rows, inner] array (inner contiguous).
 bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t inner, uint64_t rows,
               uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
@@ -984,7 +1001,7 @@ CUtensorMapSwizzle swz_enum(int row_bytes) {
 
 template <int D, int BK>
 thrift_status launch_t(const void* q, const void* k, const void* v, const thrift_nvfp4* q4, const thrift_nvfp4* k4,
-                       const thrift_nvfp4* v4, AttnParams& prm, cudaStream_t stream) {
+                       const thrift_nvfp4* v4, const AttnRows& rows, AttnParams& prm, cudaStream_t stream) {
   using L = Layout<D, BK>;
   // entry lists: [unit parity][maxe] u16 after the barrier block; the rest goes to pages
   prm.maxe = (prm.bq == 64 ? 2 : 1) * prm.nkb;
@@ -1011,9 +1028,9 @@ thrift_status launch_t(const void* q, const void* k, const void* v, const thrift
                    (uint64_t)prm.B * prm.Hkv * D, BK / 2, D, swz_enum(BK / 2));
   }
   if (prm.mode != 1) {
-    ok &= make_map(&maps[3], q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, D, qrows, 64, kBQ, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_map(&maps[4], k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, D, krows, 64, BK, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_map(&maps[5], v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, D, krows, 64, BK, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map4(&maps[3], q, rows.q, prm.B, prm.Hq, prm.N, D, kBQ);
+    ok &= make_map4(&maps[4], k, rows.k, prm.B, prm.Hkv, prm.N, D, BK);
+    ok &= make_map4(&maps[5], v, rows.v, prm.B, prm.Hkv, prm.N, D, BK);
   }
   if (!ok) return THRIFT_ERR_CUDA;
   auto kern = prm.dbg ? attn_kernel<D, BK, true> : attn_kernel<D, BK, false>;
@@ -1056,7 +1073,8 @@ __global__ void wait_timeout_kernel(int* status, long long limit) {
 thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
                               const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
                               void* out, float* out_hp, float* lse, int running_max, const thrift_cfg& c, int* status,
-                              float* dbg, int dbg_entry, cudaStream_t stream) {
+                              float* dbg, int dbg_entry, cudaStream_t stream, const AttnRows* rows_in) {
+  const AttnRows rows = rows_in ? *rows_in : dense_attn_rows(c);
   AttnParams prm;
   memset(&prm, 0, sizeof(prm));
   prm.mask = mask;
@@ -1069,6 +1087,9 @@ thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const
     prm.v_ts = v4->tensor_scale;
   }
   prm.out = reinterpret_cast<__half*>(out);
+  prm.osb = rows.out.sb;
+  prm.osh = rows.out.sh;
+  prm.osn = rows.out.sn;
   prm.out_hp = out_hp;
   prm.lse = lse;
   prm.status = status;
@@ -1088,17 +1109,27 @@ thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const
   prm.tau = c.softmax_scale > 0.0f ? c.softmax_scale : 1.0f / sqrtf((float)c.d);
   if (prm.nkb > 8191) return THRIFT_ERR_UNSUPPORTED;  // key-block index field of an entry
   prm.wait_limit = kWaitLimit;
-  if (c.d == 128 && c.block_k == 64) return launch_t<128, 64>(q, k, v, q4, k4, v4, prm, stream);
-  if (c.d == 128 && c.block_k == 128) return launch_t<128, 128>(q, k, v, q4, k4, v4, prm, stream);
-  if (c.d == 64 && c.block_k == 64) return launch_t<64, 64>(q, k, v, q4, k4, v4, prm, stream);
-  if (c.d == 64 && c.block_k == 128) return launch_t<64, 128>(q, k, v, q4, k4, v4, prm, stream);
+  if (c.d == 128 && c.block_k == 64) return launch_t<128, 64>(q, k, v, q4, k4, v4, rows, prm, stream);
+  if (c.d == 128 && c.block_k == 128) return launch_t<128, 128>(q, k, v, q4, k4, v4, rows, prm, stream);
+  if (c.d == 64 && c.block_k == 64) return launch_t<64, 64>(q, k, v, q4, k4, v4, rows, prm, stream);
+  if (c.d == 64 && c.block_k == 128) return launch_t<64, 128>(q, k, v, q4, k4, v4, rows, prm, stream);
   return THRIFT_ERR_UNSUPPORTED;
 }
 
 thrift_status attn_launch(const void* q, const void* k, const void* v, const thrift_nvfp4* q4, const thrift_nvfp4* k4,
                           const thrift_nvfp4* v4, const uint32_t* mask, int mode, void* out, float* lse,
                           const thrift_cfg& c, int* status, cudaStream_t stream) {
-  return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, nullptr, lse, 0, c, status, nullptr, -1, stream);
+  return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, nullptr, lse, 0, c, status, nullptr, -1, stream,
+                         nullptr);
+}
+
+AttnRows dense_attn_rows(const thrift_cfg& c) {
+  AttnRows r;
+  r.q = dense_rows(c.Hq, c.N, c.d);
+  r.k = dense_rows(c.Hkv, c.N, c.d);
+  r.v = dense_rows(c.Hkv, c.N, c.d);
+  r.out = dense_rows(c.Hq, c.N, c.d);
+  return r;
 }
 
 thrift_status ex2_probe_launch(const float* x, float* y, int64_t n, int which, cudaStream_t stream) {

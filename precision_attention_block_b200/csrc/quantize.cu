@@ -8,7 +8,9 @@
 //      with IEEE divisions (round to nearest) so that codes and scales are bit-identical to any
 //      other correctly rounded implementation of the same steps.
 //      Groups along d (Q, K): one thread per group, 32-byte loads, 8-byte code stores.
-//      Groups along tokens (V): a 64-token x d tile is staged in shared memory and transposed.
+//      Groups along tokens (V): a 128-token x d tile is staged in shared memory and transposed.
+// Inputs may be strided ([B, H, N, d] with any row strides, e.g. a token-major [B, N, H, d]
+// tensor); the codes and scales are always written in the dense layouts.
 #include <cuda_runtime.h>
 
 #include "sm100.cuh"
@@ -54,6 +56,35 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint4* __restrict__ x, 
   }
 }
 
+// amax of a strided tensor: CTA (tile, o) reads rows [64 tile, 64 tile + 64) of slice o.
+__global__ void __launch_bounds__(256) amax_rows_kernel(const __half* __restrict__ x, RowMap rows, int N, int d,
+                                                        unsigned int* __restrict__ amax_bits) {
+  const int o = blockIdx.y, n0 = blockIdx.x * 64;
+  const int d8 = d >> 3;
+  const __half* base = x + rows.base(o);
+  __half2 m2 = __float2half2_rn(0.0f);
+  for (int v = threadIdx.x; v < 64 * d8; v += 256) {
+    const int n = n0 + v / d8, c8 = v % d8;
+    if (n >= N) break;
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)n * rows.sn + c8 * 8));
+    const __half2* h = reinterpret_cast<const __half2*>(&w);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) m2 = __hmax2(m2, __habs2(h[t]));
+  }
+  float m = fmaxf(__low2float(m2), __high2float(m2));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  __shared__ float red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < 8 ? red[threadIdx.x] : 0.0f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (threadIdx.x == 0) atomicMax(amax_bits, __float_as_uint(m));
+  }
+}
+
 __device__ __forceinline__ float tensor_scale_from(unsigned int amax_bits) {
   float amax = __uint_as_float(amax_bits);
   return amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
@@ -84,8 +115,11 @@ __device__ __forceinline__ int64_t sf_mma_offset(int64_t row, int64_t group, int
   return (rb * n_kblocks + kb) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (group & 3);
 }
 
-// Groups along d: one thread per group of 16 consecutive elements of a row.
-__global__ void __launch_bounds__(256) encode_rows_kernel(const uint4* __restrict__ x, int64_t n_groups, int d,
+// Groups along d: one thread per group of 16 consecutive elements of a row (group g of the dense
+// order: row g / (d/16) = o * N + n; DENSE reads it at 16 g, otherwise through the row map).
+template <bool DENSE>
+__global__ void __launch_bounds__(256) encode_rows_kernel(const __half* __restrict__ xh, RowMap rows, int N,
+                                                          int64_t n_groups, int d,
                                                           const unsigned int* __restrict__ amax_bits,
                                                           uint2* __restrict__ codes, uint8_t* __restrict__ scales,
                                                           uint8_t* __restrict__ scales_mma,
@@ -96,7 +130,15 @@ __global__ void __launch_bounds__(256) encode_rows_kernel(const uint4* __restric
   int64_t n_kblocks = d >> 6;
   for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n_groups;
        g += (int64_t)gridDim.x * blockDim.x) {
-    uint4 v0 = __ldg(x + 2 * g), v1 = __ldg(x + 2 * g + 1);
+    const uint4* src;
+    if constexpr (DENSE) {
+      src = reinterpret_cast<const uint4*>(xh) + 2 * g;
+    } else {
+      const int64_t r = g / gpr;
+      const int o = (int)(r / N), n = (int)(r - (int64_t)o * N);
+      src = reinterpret_cast<const uint4*>(xh + rows.off(o, n) + (g - r * gpr) * 16);
+    }
+    uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
     float f[16];
     const __half2* h0 = reinterpret_cast<const __half2*>(&v0);
     const __half2* h1 = reinterpret_cast<const __half2*>(&v1);
@@ -120,7 +162,7 @@ __global__ void __launch_bounds__(256) encode_rows_kernel(const uint4* __restric
 // its codes (8 bytes per group), scales and tensor-core scales (one byte per group, consecutive
 // in both layouts) leave as one contiguous store each instead of one per group.
 template <int D>
-__global__ void __launch_bounds__(256) encode_cols_kernel(const __half* __restrict__ x, int N,
+__global__ void __launch_bounds__(256) encode_cols_kernel(const __half* __restrict__ x, RowMap rows, int N,
                                                           const unsigned int* __restrict__ amax_bits,
                                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                                                           uint8_t* __restrict__ scales_mma,
@@ -133,11 +175,12 @@ __global__ void __launch_bounds__(256) encode_cols_kernel(const __half* __restri
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *tensor_scale = s_t;
   const int64_t o = blockIdx.y;
   const int t0 = blockIdx.x * TOK;
-  const uint4* src = reinterpret_cast<const uint4*>(x + ((int64_t)o * N + t0) * D);
+  const __half* src = x + rows.off((int)o, t0);
   uint4* dst = reinterpret_cast<uint4*>(tile);
   constexpr int VECS = TOK * D / 8;
 #pragma unroll
-  for (int v = threadIdx.x; v < VECS; v += 256) dst[v] = __ldg(src + v);
+  for (int v = threadIdx.x; v < VECS; v += 256)
+    dst[v] = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)(v / (D / 8)) * rows.sn + (v % (D / 8)) * 8));
   __syncthreads();
   const int c = threadIdx.x % D, part = threadIdx.x / D;
   const int g_first = part * GPT;  // first group of the thread within the tile
@@ -306,32 +349,37 @@ size_t scales_mma_bytes(int64_t outer, int32_t N, int32_t d, int32_t group_axis)
   return (size_t)(nrb * (len / 64) * 512);
 }
 
-thrift_status quantize_launch(const void* x, int64_t outer, int32_t N, int32_t d, const thrift_nvfp4* out,
-                              unsigned int* amax_slot, cudaStream_t stream) {
+thrift_status quantize_launch(const void* x, const RowMap& rows, int64_t outer, int32_t N, int32_t d,
+                              const thrift_nvfp4* out, unsigned int* amax_slot, cudaStream_t stream) {
   int64_t total = outer * (int64_t)N * d;
+  const bool dense = rows.dense((int)(outer / rows.H), N, d);
+  const __half* xh = reinterpret_cast<const __half*>(x);
   if (cudaMemsetAsync(amax_slot, 0, sizeof(unsigned int), stream) != cudaSuccess) return THRIFT_ERR_CUDA;
   int sms = num_sms();
-  int64_t amax_blocks = (total / 8 + 4 * 256 - 1) / (4 * 256);  // about four vectors per thread
-  if (amax_blocks > (int64_t)sms * 8) amax_blocks = (int64_t)sms * 8;
-  if (amax_blocks < 1) amax_blocks = 1;
-  amax_kernel<<<(unsigned)amax_blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), total / 8, amax_slot);
+  if (dense) {
+    int64_t amax_blocks = (total / 8 + 4 * 256 - 1) / (4 * 256);  // about four vectors per thread
+    if (amax_blocks > (int64_t)sms * 8) amax_blocks = (int64_t)sms * 8;
+    if (amax_blocks < 1) amax_blocks = 1;
+    amax_kernel<<<(unsigned)amax_blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), total / 8, amax_slot);
+  } else {
+    amax_rows_kernel<<<dim3((N + 63) / 64, (unsigned)outer), 256, 0, stream>>>(xh, rows, N, d, amax_slot);
+  }
   if (out->group_axis == 0) {
     int64_t groups = total / 16;
     int64_t blocks = (groups + 255) / 256;
     if (blocks > (int64_t)sms * 32) blocks = (int64_t)sms * 32;
-    encode_rows_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
-        reinterpret_cast<const uint4*>(x), groups, d, amax_slot, reinterpret_cast<uint2*>(out->codes),
-        out->scales, out->scales_mma, out->tensor_scale);
+    auto kern = dense ? encode_rows_kernel<true> : encode_rows_kernel<false>;
+    kern<<<(unsigned)blocks, 256, 0, stream>>>(xh, rows, N, groups, d, amax_slot,
+                                               reinterpret_cast<uint2*>(out->codes), out->scales, out->scales_mma,
+                                               out->tensor_scale);
   } else {
     dim3 grid(N / 128, (unsigned)outer);
     if (d == 128)
-      encode_cols_kernel<128><<<grid, 256, 0, stream>>>(reinterpret_cast<const __half*>(x), N, amax_slot,
-                                                         out->codes, out->scales, out->scales_mma,
-                                                         out->tensor_scale);
+      encode_cols_kernel<128><<<grid, 256, 0, stream>>>(xh, rows, N, amax_slot, out->codes, out->scales,
+                                                         out->scales_mma, out->tensor_scale);
     else
-      encode_cols_kernel<64><<<grid, 256, 0, stream>>>(reinterpret_cast<const __half*>(x), N, amax_slot,
-                                                        out->codes, out->scales, out->scales_mma,
-                                                        out->tensor_scale);
+      encode_cols_kernel<64><<<grid, 256, 0, stream>>>(xh, rows, N, amax_slot, out->codes, out->scales,
+                                                        out->scales_mma, out->tensor_scale);
   }
   return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }

@@ -37,12 +37,12 @@ namespace {
 // FP16 values here is exact in float64 (the block's |sum| stays below 2^23 on the 2^-24 grid of
 // FP16), so the order of the additions does not change the result.
 constexpr int kMeanThreads = 256;
-__global__ void __launch_bounds__(kMeanThreads) block_mean_kernel(const __half* __restrict__ x, int N, int d, int bs,
-                                                                  double* __restrict__ mean) {
+__global__ void __launch_bounds__(kMeanThreads) block_mean_kernel(const __half* __restrict__ x, RowMap rows, int N,
+                                                                  int d, int bs, double* __restrict__ mean) {
   __shared__ double part[kMeanThreads / 16][128];
   const int64_t bh = blockIdx.y;
   const int blk = blockIdx.x;
-  const __half* base = x + (bh * N + (int64_t)blk * bs) * d;
+  const __half* base = x + rows.off((int)bh, blk * bs);
   const int lane16 = threadIdx.x & 15, grp = threadIdx.x >> 4;
   const int c0 = lane16 * 8;  // first of this thread's 8 columns
   double acc[8];
@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kMeanThreads) block_mean_kernel(const __half* 
   for (int e = 0; e < 8; ++e) acc[e] = 0.0;
   if (c0 < d) {
     for (int t = grp; t < bs; t += kMeanThreads / 16) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)t * d + c0));
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)t * rows.sn + c0));
       const __half2* h = reinterpret_cast<const __half2*>(&w);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -661,18 +661,19 @@ thrift_status noalloc_select_scratch(uint8_t** out) {
   return THRIFT_OK;
 }
 
-thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, uint32_t* mask, int32_t* counts,
-                            int16_t* lists, double* scores_out, uint8_t* scratch, cudaStream_t stream) {
+thrift_status select_launch(const void* q, const RowMap& qrows, const void* k, const RowMap& krows,
+                            const thrift_cfg& c, uint32_t* mask, int32_t* counts, int16_t* lists, double* scores_out,
+                            uint8_t* scratch, cudaStream_t stream) {
   SelectLayout L = select_layout(c);
   int nqb = c.N / c.block_q, nkb = c.N / c.block_k;
   int mask_words = (nkb + 31) / 32;
   double* qbar = reinterpret_cast<double*>(scratch + L.qbar_off);
   double* kbar = reinterpret_cast<double*>(scratch + L.kbar_off);
   double* scores = scores_out ? scores_out : reinterpret_cast<double*>(scratch + L.scores_off);
-  block_mean_kernel<<<dim3(nqb, c.B * c.Hq), kMeanThreads, 0, stream>>>(reinterpret_cast<const __half*>(q), c.N,
-                                                                         c.d, c.block_q, qbar);
-  block_mean_kernel<<<dim3(nkb, c.B * c.Hkv), kMeanThreads, 0, stream>>>(reinterpret_cast<const __half*>(k), c.N,
-                                                                          c.d, c.block_k, kbar);
+  block_mean_kernel<<<dim3(nqb, c.B * c.Hq), kMeanThreads, 0, stream>>>(reinterpret_cast<const __half*>(q), qrows,
+                                                                         c.N, c.d, c.block_q, qbar);
+  block_mean_kernel<<<dim3(nkb, c.B * c.Hkv), kMeanThreads, 0, stream>>>(reinterpret_cast<const __half*>(k), krows,
+                                                                          c.N, c.d, c.block_k, kbar);
   dim3 g((nkb + kTileK - 1) / kTileK, (nqb + kTileQ - 1) / kTileQ, c.B * c.Hq);
   block_score_kernel<<<g, 256, 0, stream>>>(qbar, kbar, c.Hq, c.Hkv, nqb, nkb, c.d, c.block_q, c.block_k, c.causal,
                                             scores);
@@ -697,7 +698,7 @@ thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, u
 thrift_status kv_means_launch(const void* k, int64_t outer, int32_t Nk, int32_t d, int32_t block_k, double* kbar,
                               cudaStream_t stream) {
   block_mean_kernel<<<dim3(Nk / block_k, (unsigned)outer), kMeanThreads, 0, stream>>>(
-      reinterpret_cast<const __half*>(k), Nk, d, block_k, kbar);
+      reinterpret_cast<const __half*>(k), dense_rows(1, Nk, d), Nk, d, block_k, kbar);
   return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 

@@ -11,6 +11,24 @@ namespace thrift {
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Element offsets in an FP16 tensor viewed as [B, H, N, d] with strides (sb, sh, sn) in elements
+// (the d elements of a token row contiguous): row n of slice o = b * H + h starts at off(o, n).
+struct RowMap {
+  int64_t sb, sh, sn;
+  int H;
+  __host__ __device__ __forceinline__ int64_t base(int o) const {
+    return (int64_t)(o / H) * sb + (int64_t)(o % H) * sh;
+  }
+  __host__ __device__ __forceinline__ int64_t off(int o, int n) const { return base(o) + (int64_t)n * sn; }
+  // the dense layout (sb only matters with more than one batch)
+  bool dense(int B, int N, int d) const {
+    return sn == d && sh == (int64_t)N * d && (B == 1 || sb == (int64_t)H * N * d);
+  }
+};
+inline RowMap dense_rows(int H, int N, int d) {
+  return RowMap{(int64_t)H * N * d, (int64_t)N * d, (int64_t)d, H};
+}
+
 int num_sms();
 
 // Unique id of the calling thread's current CUDA context (cuCtxGetId), 0 when none is current or
@@ -29,8 +47,9 @@ SelectLayout select_layout(const thrift_cfg& c);
 
 size_t scales_mma_bytes(int64_t outer, int32_t N, int32_t d, int32_t group_axis);
 
-thrift_status quantize_launch(const void* x, int64_t outer, int32_t N, int32_t d, const thrift_nvfp4* out,
-                              unsigned int* amax_slot, cudaStream_t stream);
+// x: [outer, N, d] rows addressed through `rows` (rows.H divides outer into batch and head).
+thrift_status quantize_launch(const void* x, const RowMap& rows, int64_t outer, int32_t N, int32_t d,
+                              const thrift_nvfp4* out, unsigned int* amax_slot, cudaStream_t stream);
 
 thrift_status tensor_scale_launch(const void* x, int64_t n, float* tensor_scale, unsigned int* amax_slot,
                                   cudaStream_t stream);
@@ -39,8 +58,9 @@ thrift_status kv_append_launch(const void* k_new, const void* v_new, int64_t out
                                int32_t block_k, int32_t len, int32_t T, void* k, void* v, const thrift_nvfp4* k4,
                                const thrift_nvfp4* v4, double* kbar, cudaStream_t stream);
 
-thrift_status select_launch(const void* q, const void* k, const thrift_cfg& c, uint32_t* mask, int32_t* counts,
-                            int16_t* lists, double* scores_out, uint8_t* scratch, cudaStream_t stream);
+thrift_status select_launch(const void* q, const RowMap& qrows, const void* k, const RowMap& krows,
+                            const thrift_cfg& c, uint32_t* mask, int32_t* counts, int16_t* lists, double* scores_out,
+                            uint8_t* scratch, cudaStream_t stream);
 
 size_t noalloc_select_scratch_bytes();
 thrift_status noalloc_select_scratch(uint8_t** out);
@@ -50,6 +70,12 @@ thrift_status noalloc_select_scratch(uint8_t** out);
 thrift_status attn_launch(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
                           const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
                           void* out, float* lse, const thrift_cfg& c, int* status, cudaStream_t stream);
+
+// Row maps of the FP16 operands and of the output of one attention launch (dense unless given).
+struct AttnRows {
+  RowMap q, k, v, out;
+};
+AttnRows dense_attn_rows(const thrift_cfg& c);
 
 thrift_status wait_timeout_launch(int* status, long long limit, cudaStream_t stream);
 

@@ -106,6 +106,24 @@ def test_null_and_workspace_errors(L):
     nv1 = _lib.CNVFP4(0x1000, 0x1000, 0x1000, 0x1000, 1)
     assert L.thrift_attn_fwd_running_max(p, p, p, ctypes.byref(nv), ctypes.byref(nv), ctypes.byref(nv1), p, p,
                                          None, ctypes.byref(c), None, 0, None) == 5
+    # strides: multiples of 8 elements, token rows at least d apart; NULL is dense
+    bad = [_lib.CStrides(8 * 512 * 128, 512 * 128, 100), _lib.CStrides(8 * 512 * 128, 512 * 128, 64),
+           _lib.CStrides(-8, 512 * 128, 128), _lib.CStrides(4, 512 * 128, 128)]
+    for st in bad:
+        assert L.thrift_attn_fwd_auto_strided(p, ctypes.byref(st), p, None, p, None, p, None, None,
+                                              ctypes.byref(c), p, 1 << 40, None) == 1
+        assert L.thrift_block_select_strided(p, None, p, ctypes.byref(st), ctypes.byref(c), p, p, p, None, p,
+                                             1 << 40, None) == 1
+        assert L.thrift_quantize_nvfp4_strided(p, ctypes.byref(st), 1, 8, 512, 128, ctypes.byref(nv), p, 256,
+                                               None) == 1
+        assert L.thrift_attn_fwd_strided(p, None, p, None, p, None, ctypes.byref(nv), ctypes.byref(nv),
+                                         ctypes.byref(nv1), p, p, ctypes.byref(st), None, ctypes.byref(c), p, 256,
+                                         None) == 1
+    good = _lib.CStrides(512 * 8 * 128, 128, 8 * 128)  # token-major [B, N, H, d]
+    assert L.thrift_quantize_nvfp4_strided(p, ctypes.byref(good), 1, 8, 512, 128, ctypes.byref(nv), None, 0,
+                                           None) == 5
+    assert L.thrift_quantize_nvfp4_strided(p, ctypes.byref(good), 0, 8, 512, 128, ctypes.byref(nv), p, 256,
+                                           None) == 1
 
 
 def dcfg(**kw):
