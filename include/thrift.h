@@ -42,7 +42,11 @@ typedef enum {
   THRIFT_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels implement */
   THRIFT_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
   THRIFT_ERR_TIMEOUT = 4,      /* device status only: a bounded wait inside a kernel ran out */
-  THRIFT_ERR_WORKSPACE = 5     /* workspace pointer null, misaligned or too small */
+  THRIFT_ERR_WORKSPACE = 5,    /* workspace pointer null, misaligned or too small */
+  THRIFT_ERR_CHECK = 8         /* device status only, checked build (libthrift_checked): an in-kernel
+                                  bounds check failed; the access was skipped and the kernel unwound.
+                                  The device status word is the bitwise OR of the device-side errors
+                                  seen (THRIFT_ERR_TIMEOUT, THRIFT_ERR_CHECK). */
 } thrift_status;
 
 /* Problem description, passed by value-pointer; the library keeps no copy. */

@@ -40,6 +40,15 @@ thrift_status thrift_debug_ex2(const float* x, float* y, int64_t n, int32_t whic
 size_t thrift_debug_pipe_rates_ws_bytes(void);
 thrift_status thrift_debug_pipe_rates(void* ws, size_t ws_bytes, double* out, void* stream);
 
+/* 1 when the library was built with in-kernel bounds checks (libthrift_checked.so: every index
+ * that selects a tile, list entry or mask word is checked before use), else 0. */
+int32_t thrift_debug_checks_enabled(void);
+
+/* Runs one in-kernel check that fails when `fail` is non-zero.  In the checked build a failing
+ * check records THRIFT_ERR_CHECK in the workspace status word (and skips nothing else); in the
+ * regular build checks are compiled out and the status stays 0. */
+thrift_status thrift_debug_check(void* ws, int32_t fail, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -11,7 +11,8 @@ import os
 import threading
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libthrift.so")
+# THRIFT_LIB selects another build of the same ABI (e.g. libthrift_checked.so, the checked build)
+LIB_PATH = os.environ.get("THRIFT_LIB") or os.path.join(HERE, "libthrift.so")
 
 THRIFT_OK = 0
 THRIFT_ERR_INVALID_ARG = 1
@@ -19,6 +20,7 @@ THRIFT_ERR_UNSUPPORTED = 2
 THRIFT_ERR_CUDA = 3
 THRIFT_ERR_TIMEOUT = 4
 THRIFT_ERR_WORKSPACE = 5
+THRIFT_ERR_CHECK = 8
 
 
 class ThriftError(RuntimeError):
@@ -101,6 +103,8 @@ SIGNATURES = {
     "thrift_debug_ex2": (ctypes.c_int, [_vp, _vp, _i64, _i32, _vp]),
     "thrift_debug_pipe_rates_ws_bytes": (_sz, []),
     "thrift_debug_pipe_rates": (ctypes.c_int, [_vp, _sz, _vp, _vp]),
+    "thrift_debug_checks_enabled": (ctypes.c_int32, []),
+    "thrift_debug_check": (ctypes.c_int, [_vp, _i32, _vp]),
     "thrift_status_str": (ctypes.c_char_p, [ctypes.c_int]),
     "thrift_debug_attn_dump": (ctypes.c_int, [_vp, _vp, _vp, _nvp, _nvp, _nvp, _vp, _vp, _vp, _cfgp, _vp,
                                               _sz, _vp, _i32, _vp]),

@@ -1,6 +1,8 @@
-"""Build libthrift.so in-tree with nvcc for sm_100a (no JIT cache, no torch extension).
+"""Build libthrift.so in-tree with nvcc for sm_100a (no JIT cache, no torch extension), and the
+checked variant libthrift_checked.so (THRIFT_CHECKS: in-kernel bounds checks that record
+THRIFT_ERR_CHECK in the device status word and skip the access).
 
-    python -m precision_attention_block_b200.build [--force]
+    python -m precision_attention_block_b200.build [--force] [--checked]
 """
 
 from __future__ import annotations
@@ -15,6 +17,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libthrift.so")
 BUILD = os.path.join(HERE, "_build")
+LIB_CHECKED = os.path.join(HERE, "libthrift_checked.so")
+BUILD_CHECKED = os.path.join(HERE, "_build_checked")
 SOURCES = ["quantize.cu", "select.cu", "attn.cu", "decode.cu", "probe.cu", "api.cu"]
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
@@ -27,14 +31,16 @@ def _deps():
     return max(os.path.getmtime(f) for f in files)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    lib, bdir = (LIB_CHECKED, BUILD_CHECKED) if checked else (LIB, BUILD)
+    if not force and os.path.exists(lib) and os.path.getmtime(lib) >= _deps():
+        return lib
+    os.makedirs(bdir, exist_ok=True)
+    flags = FLAGS + (["-DTHRIFT_CHECKS=1"] if checked else [])
 
     def compile_one(src):
-        obj = os.path.join(BUILD, src.replace(".cu", ".o"))
-        cmd = [NVCC, *FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
+        obj = os.path.join(bdir, src.replace(".cu", ".o"))
+        cmd = [NVCC, *flags, "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -46,14 +52,20 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
     with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
         objs = list(ex.map(compile_one, SOURCES))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     r = subprocess.run([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", tmp],
                        capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build_all(force: bool = False) -> None:
+    """Both libraries (the regular one and the checked one), built side by side."""
+    with ThreadPoolExecutor(max_workers=2) as ex:
+        list(ex.map(lambda c: build(force=force, checked=c), (False, True)))
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, checked="--checked" in sys.argv))

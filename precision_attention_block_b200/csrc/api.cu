@@ -583,6 +583,19 @@ thrift_status thrift_debug_pipe_rates(void* ws, size_t ws_bytes, double* out, vo
   return pipe_rates_launch(ws, out, static_cast<cudaStream_t>(stream));
 }
 
+int32_t thrift_debug_checks_enabled(void) {
+#ifdef THRIFT_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+thrift_status thrift_debug_check(void* ws, int32_t fail, void* stream) {
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 != 0) return THRIFT_ERR_WORKSPACE;
+  return check_probe_launch(status_ptr(ws), fail, static_cast<cudaStream_t>(stream));
+}
+
 const char* thrift_status_str(thrift_status s) {
   switch (s) {
     case THRIFT_OK: return "ok";
@@ -591,6 +604,7 @@ const char* thrift_status_str(thrift_status s) {
     case THRIFT_ERR_CUDA: return "CUDA error";
     case THRIFT_ERR_TIMEOUT: return "device wait timed out";
     case THRIFT_ERR_WORKSPACE: return "workspace null, misaligned or too small";
+    case THRIFT_ERR_CHECK: return "in-kernel bounds check failed";
   }
   return "unknown status";
 }

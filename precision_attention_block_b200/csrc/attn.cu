@@ -196,7 +196,8 @@ __device__ int build_list(const AttnParams& p, int b, int h, int t, uint16_t* li
       if (two && jj < jmax1 && sel(m1, jj) == phase) rm |= 2;
       if (!two && rm) rm = 3;
       const unsigned bal = __ballot_sync(0xffffffffu, rm != 0);
-      if (rm) list[n + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)(jj | (phase << 13) | (rm << 14));
+      if (rm && THRIFT_CHECK(n + __popc(bal) <= p.maxe, p.status))
+        list[n + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)(jj | (phase << 13) | (rm << 14));
       n += __popc(bal);
     }
   }
@@ -498,6 +499,12 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t xe = list[e];
             const int j = xe & 0x1fff, f16 = (xe >> 13) & 1;
             const int krow0 = kvh * p.N + j * BK;
+            // the tiles of this entry lie inside the tensors
+            if (!THRIFT_CHECK(j < p.nkb && (ui.t + 1) * kBQ <= p.N && ui.hk < p.Hkv && ui.b < p.B, p.status)) {
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
             if (f16 && !q16_loaded) {
               if (!(ok = mbar_wait(&bars->q16_empty, (u16c & 1) ^ 1, abort_flag, p.status, lim))) break;
               ++u16c;
@@ -733,6 +740,11 @@ __global__ void __launch_bounds__(384, 1)
       if (!(ok = mbar_wait(&bars->list_full[lb], lph, abort_flag, p.status, lim))) break;
       const int n_entries = bars->list_count[lb];
       const uint16_t* list = lists + lb * p.maxe;
+      if (!THRIFT_CHECK(n_entries <= p.maxe, p.status)) {
+        *abort_flag = 1;
+        ok = false;
+        break;
+      }
       const int row = ui.t * kBQ + rr;
       const int half = (p.bq == 64) ? (rr >> 6) : 0;
       float O[DH];

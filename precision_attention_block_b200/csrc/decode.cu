@@ -310,6 +310,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_kernel(const __grid_c
         const int j = j0 + i;
         const uint32_t bits = bits_of(i);
         const int64_t kr = krow0 + (int64_t)j * BK;
+        // the key block lies inside the cache
+        if (!THRIFT_CHECK((int64_t)(j + 1) * BK <= p.Nk, p.status)) {
+          *abort_flag = 1;
+          break;
+        }
         if (use4) {
           const int s = i % NST;
           ok = mbar_wait(&empty4[s], ((i / NST) & 1) ^ 1, abort_flag, p.status, p.wait_limit);

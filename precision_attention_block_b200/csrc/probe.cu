@@ -3,6 +3,7 @@
 // threads per SM running eight independent chains per thread.
 #include <cuda_runtime.h>
 
+#include "sm100.cuh"
 #include "thrift_internal.h"
 
 namespace thrift {
@@ -57,5 +58,14 @@ thrift_status pipe_rates_launch(void* ws, double* out, cudaStream_t stream) {
 }
 
 size_t pipe_rates_ws_bytes() { return kWsHeader + 64 + kProbeThreads * sizeof(float); }
+
+__global__ void check_probe_kernel(int* status, int fail) {
+  if (!THRIFT_CHECK(fail == 0, status)) return;
+}
+
+thrift_status check_probe_launch(int* status, int fail, cudaStream_t stream) {
+  check_probe_kernel<<<1, 1, 0, stream>>>(status, fail);
+  return cudaPeekAtLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
+}
 
 }  // namespace thrift

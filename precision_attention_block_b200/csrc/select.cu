@@ -491,7 +491,8 @@ __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkClus
   auto take_at = [&](int64_t t) {
     const int64_t g = t0 + t;
     const int i = (int)(g / nkb), j = (int)(g % nkb);
-    atomicOr(&mk[(int64_t)i * mask_words + (j >> 5)], 1u << (j & 31));
+    if (THRIFT_CHECK(g < n && (j >> 5) < mask_words, nullptr))
+      atomicOr(&mk[(int64_t)i * mask_words + (j >> 5)], 1u << (j & 31));
   };
   if (need_here <= 0 || need_here >= my_ties) {
     // none or all of this CTA's ties

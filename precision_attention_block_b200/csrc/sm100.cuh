@@ -9,6 +9,25 @@ namespace thrift {
 
 // Device status bits recorded in the workspace status word.
 constexpr int kStatusTimeout = 4;  // same value as THRIFT_ERR_TIMEOUT
+constexpr int kStatusCheck = 8;    // same value as THRIFT_ERR_CHECK
+
+// In-kernel checks of the checked build (THRIFT_CHECKS defined): THRIFT_CHECK(cond, status)
+// evaluates cond; when it is false it records kStatusCheck in the status word and the source line
+// in the word two after it (first failure only), and yields false so that the caller skips the
+// access (and, in the warp-specialised kernels, raises the abort flag that unwinds every wait).
+// In the regular build it is the constant true and the checks compile away.
+__device__ __forceinline__ bool check_ok(bool ok, int* status, int line) {
+  if (!ok && status) {
+    atomicOr(status, kStatusCheck);
+    atomicCAS(status + 2, 0, line);
+  }
+  return ok;
+}
+#ifdef THRIFT_CHECKS
+#define THRIFT_CHECK(cond, status) (::thrift::check_ok((cond), (status), __LINE__))
+#else
+#define THRIFT_CHECK(cond, status) true
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

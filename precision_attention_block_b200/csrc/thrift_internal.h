@@ -82,6 +82,7 @@ thrift_status wait_timeout_launch(int* status, long long limit, cudaStream_t str
 thrift_status pipe_rates_launch(void* ws, double* out, cudaStream_t stream);
 thrift_status ex2_probe_launch(const float* x, float* y, int64_t n, int which, cudaStream_t stream);
 size_t pipe_rates_ws_bytes();
+thrift_status check_probe_launch(int* status, int fail, cudaStream_t stream);
 
 // ---- decode
 // The cache's valid length (thrift_decode_cfg.n_valid, 0 meaning the whole capacity).

@@ -23,7 +23,8 @@ def declared_functions():
     for fn in os.listdir(os.path.join(ROOT, "include")):
         if fn.endswith(".h"):
             src = open(os.path.join(ROOT, "include", fn)).read()
-            names |= set(re.findall(r"^\s*(?:const\s+char\s*\*|size_t|thrift_status)\s+(thrift_\w+)\s*\(", src, re.M))
+            names |= set(re.findall(r"^\s*(?:const\s+char\s*\*|size_t|int32_t|thrift_status)\s+(thrift_\w+)\s*\(",
+                                    src, re.M))
     return names
 
 
@@ -32,6 +33,20 @@ def test_every_declared_symbol_is_exported(L):
     assert {"thrift_quantize_nvfp4", "thrift_block_select", "thrift_attn_fwd"} <= names
     for n in names:
         assert hasattr(L, n), n
+
+
+def test_checked_build_exports_the_same_abi(L):
+    """libthrift_checked.so (in-kernel bounds checks) is a drop-in build of the same ABI; only it
+    reports the checks as enabled."""
+    from precision_attention_block_b200 import build
+    path = build.build(checked=True)
+    C = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(C, n), n
+    C.thrift_debug_checks_enabled.restype = ctypes.c_int32
+    assert C.thrift_debug_checks_enabled() == 1
+    assert L.thrift_debug_checks_enabled() == 0
+    assert L.thrift_status_str(8) == b"in-kernel bounds check failed"
 
 
 def test_binding_covers_every_declared_symbol():
