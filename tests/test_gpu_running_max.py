@@ -65,6 +65,33 @@ def test_running_max_all_fp16_equals_r1(pab):
     assert np.linalg.norm(a - b) / np.linalg.norm(b) <= 1e-3
 
 
+SHAPES = {
+    # 128-key blocks, causal, GQA 4:1
+    "bk128": workloads.Workload("r2_bk128", 97, 1, 8, 2, 1024, 128, True, 128, 128, -1, 1500, "heavy_bias"),
+    # 64-row query blocks (two per tile, each with its own entry order), causal, d = 64
+    "bq64": workloads.Workload("r2_bq64", 98, 2, 4, 4, 1024, 64, True, 64, 64, -1, 2500, "normal"),
+    # 128-key blocks with d = 64 (the shortest entry lists)
+    "d64_bk128": workloads.Workload("r2_d64", 99, 1, 4, 1, 512, 64, True, 128, 128, -1, 3000, "student_t"),
+}
+
+
+@pytest.mark.parametrize("shape", list(SHAPES))
+def test_running_max_shapes(pab, shape):
+    w = SHAPES[shape]
+    q, k, v = workloads.make_qkv(w)
+    gq, gk, gv = (torch.from_numpy(x).cuda() for x in (q, k, v))
+    cfg = pab.Config.from_workload(w)
+    q4, k4, v4 = pab.quantize_qkv(gq, gk, gv)
+    sel = pab.block_select(gq, gk, cfg)
+    out_g, lse_g = pab.attn_fwd(gq, gk, gv, q4, k4, v4, sel, cfg, running_max=True)
+    torch.cuda.synchronize()
+    q4o, k4o, v4o = oracle.quantize_nvfp4(q, 0), oracle.quantize_nvfp4(k, 0), oracle.quantize_nvfp4(v, 1)
+    sel_o, _, _ = oracle.select(oracle.block_scores(q, k, w), w)
+    units = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.n_qb)]
+    out_o, lse_o, _ = oracle.attn_r2(q, k, v, q4o, k4o, v4o, sel_o, w, units=units)
+    compare_attention(out_g, lse_g, out_o, lse_o, w, units)
+
+
 @pytest.mark.parametrize("bp", [500, 2000])
 def test_running_max_diffusion_sampled(pab, bp):
     run_r2(pab, "diffusion", bp, n_units=8)
