@@ -10,9 +10,10 @@
 //           order-preserving 64-bit keys finds the k-th largest score; keys above it are taken,
 //           ties at it are taken in index order (smaller i * nKb + j first) through a block scan.
 //           Long rows run on a cluster of CTAs that split the row into contiguous index ranges,
-//           hold their keys in shared memory and add up their digit histograms through
-//           distributed shared memory; short rows run on one CTA.
-//   lists   one thread per query block walks its mask words in ascending order.
+//           stream their keys from L2 for every digit and add up their digit histograms in a
+//           per-head histogram in global memory behind a cluster barrier; short rows (at most
+//           4096 keys) run on one CTA with the keys in shared memory.
+//   lists   one warp per row of mask words; lanes own runs of words, a warp scan places them.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
