@@ -171,8 +171,13 @@ def peaks():
 
 
 def attn_src_hash() -> str:
-    with open(ATTN_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of the attention kernel's sources (the kernel file and the inline-PTX header it
+    includes): stored DRAM counters count only for the kernel they were taken on."""
+    h = hashlib.sha256()
+    for path in (ATTN_SRC, os.path.join(os.path.dirname(ATTN_SRC), "sm100.cuh")):
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def stored_traffic(workload: str):

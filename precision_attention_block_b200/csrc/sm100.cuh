@@ -77,8 +77,9 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity (polls with a short sleep between tries).
-// Gives up after `limit` clock cycles,
+// Bounded wait for the phase with the given parity.  try_wait itself may suspend the thread for a
+// while when the phase is not complete; no extra sleep is added between tries (a 60 ns back-off
+// cost 1 % of the prefill attention kernel's time).  Gives up after `limit` clock cycles,
 // records the timeout in the global status word (and, in the word after it, which wait gave up
 // first) and raises the CTA's abort flag (a shared flag:
 // once any wait of the CTA gives up, every later wait returns at once, so that all warps reach
@@ -89,9 +90,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   long long t0 = clock64();
   while (true) {
     if (*abort_flag) return false;
-    // back off between polls: a waiting warp that polls continuously takes issue slots from the
-    // warps on its SM sub-partition that do the work it waits for
-    __nanosleep(60);
     if (mbar_try_wait(bar, parity)) return true;
     if (clock64() - t0 > limit) {
       *abort_flag = 1;
