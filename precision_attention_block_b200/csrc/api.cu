@@ -13,11 +13,6 @@
 
 namespace thrift {
 
-thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
-                              const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
-                              void* out, float* out_hp, float* lse, int running_max, const thrift_cfg& c, int* status,
-                              float* dbg, int dbg_entry, cudaStream_t stream, const AttnRows* rows = nullptr);
-
 unsigned long long current_context_id() {
   typedef CUresult (*GetCurrentFn)(CUcontext*);
   typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);

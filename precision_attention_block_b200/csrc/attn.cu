@@ -1128,13 +1128,6 @@ thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const
   return THRIFT_ERR_UNSUPPORTED;
 }
 
-thrift_status attn_launch(const void* q, const void* k, const void* v, const thrift_nvfp4* q4, const thrift_nvfp4* k4,
-                          const thrift_nvfp4* v4, const uint32_t* mask, int mode, void* out, float* lse,
-                          const thrift_cfg& c, int* status, cudaStream_t stream) {
-  return attn_launch_dbg(q, k, v, q4, k4, v4, mask, mode, out, nullptr, lse, 0, c, status, nullptr, -1, stream,
-                         nullptr);
-}
-
 AttnRows dense_attn_rows(const thrift_cfg& c) {
   AttnRows r;
   r.q = dense_rows(c.Hq, c.N, c.d);

@@ -65,17 +65,21 @@ thrift_status select_launch(const void* q, const RowMap& qrows, const void* k, c
 size_t noalloc_select_scratch_bytes();
 thrift_status noalloc_select_scratch(uint8_t** out);
 
-// mode: 0 = FP16 pairs from the mask, 1 = every pair NVFP4, 2 = every pair FP16, 3 = only the
-// FP16 pairs of the mask (the compute-matched sparse variant; no NVFP4 operand is read).
-thrift_status attn_launch(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
-                          const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
-                          void* out, float* lse, const thrift_cfg& c, int* status, cudaStream_t stream);
-
 // Row maps of the FP16 operands and of the output of one attention launch (dense unless given).
 struct AttnRows {
   RowMap q, k, v, out;
 };
 AttnRows dense_attn_rows(const thrift_cfg& c);
+
+// The fused attention launch.  mode: 0 = FP16 pairs from the mask, 1 = every pair NVFP4,
+// 2 = every pair FP16, 3 = only the FP16 pairs of the mask (the compute-matched sparse variant; no
+// NVFP4 operand is read).  out_hp: the FP32 copy of the output (may be null); running_max: the
+// running maximum as the P requantisation's first level (reading R2); dbg, dbg_entry: the debug
+// dump of one entry (null and -1 normally); rows: null for dense operands and output.
+thrift_status attn_launch_dbg(const void* q, const void* k, const void* v, const thrift_nvfp4* q4,
+                              const thrift_nvfp4* k4, const thrift_nvfp4* v4, const uint32_t* mask, int mode,
+                              void* out, float* out_hp, float* lse, int running_max, const thrift_cfg& c, int* status,
+                              float* dbg, int dbg_entry, cudaStream_t stream, const AttnRows* rows = nullptr);
 
 thrift_status wait_timeout_launch(int* status, long long limit, cudaStream_t stream);
 
