@@ -3,7 +3,7 @@
  * forward on NVIDIA B200 (sm_100a).
  *
  * The method (ThriftAttention technical summary, gist.science 2605.23081, section
- * "Methodologie"; the same text in the French version, "Methodologie : ThriftAttention"):
+ * "Methodologie"; the same text in the French version, "Méthodologie : ThriftAttention"):
  *   1. Q, K and V are split into blocks; every (query block i, key block j) pair gets the
  *      importance score S^_ij = qbar_i . kbar_j, the dot product of the blocks' token means.
  *   2. The k highest-scoring pairs (per batch and query head here) run in FP16; all other
@@ -204,7 +204,8 @@ thrift_status thrift_attn_fwd_strided(const void* q, const thrift_strides* qs, c
                                       void* stream);
 
 /* thrift_attn_fwd with the other reading of the two-level P requantisation (ThriftAttention
- * "Twee-niveau P-herkwantisatie", which follows SageAttention3's two-level scheme).
+ * "Methodologie", "Online Samenvoeging": the probability blocks get a two-level quantisation
+ * adapted from SageAttention3, inside an online softmax).
  * thrift_attn_fwd takes each key block's own row maximum M as the first level: P^ = exp(S - M),
  * so every block's largest probability requantises at the top of the NVFP4 range.  Here the
  * first level is the row's running maximum m over the key blocks visited so far, in the kernel's

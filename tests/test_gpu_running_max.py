@@ -1,5 +1,6 @@
 """The running-maximum reading of the two-level P requantisation (thrift_attn_fwd_running_max;
-ThriftAttention "Twee-niveau P-herkwantisatie" after SageAttention3's scheme): the CUDA path against
+ThriftAttention summary, "Methodologie", "Online Samenvoeging": a two-level scheme for the
+probability blocks adapted from SageAttention3): the CUDA path against
 the oracle's reading R2 (first level = the row's running maximum in the kernel's visiting order,
 NVFP4 key blocks ascending then FP16 ones), to the same bar as thrift_attn_fwd against R1: rel-L2
 <= 1e-3, max-abs <= 1e-2 (one FP16 step where that is larger), LSE within 1e-3."""

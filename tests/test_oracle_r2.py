@@ -1,8 +1,9 @@
 """Pins for the oracle's reading R2 of the two-level P quantisation: the first level is the row's
 running maximum in the fused kernel's visiting order (NVFP4 key blocks in ascending order, then
 the FP16 ones), so a block whose maximum lies below the running maximum re-quantises exp(S - m)
-with a group scale below 448 (ThriftAttention "Twee-niveau P-herkwantisatie"; the running-maximum
-first level follows SageAttention3's two-level P quantisation).
+with a group scale below 448 (ThriftAttention summary, "Methodologie", "Online Samenvoeging": a
+two-level quantisation of the probability blocks adapted from SageAttention3, inside an online
+softmax; the running maximum of that online softmax is taken as the first level).
 
 Each test checks the oracle against a closed form built from library casts (ml_dtypes E4M3/E2M1,
 numpy float16), torch SDPA in float64, or the R1 oracle where the two readings coincide."""
