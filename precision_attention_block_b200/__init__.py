@@ -144,7 +144,12 @@ def _strides(t: Optional[torch.Tensor]):
         return None
     if t.dim() != 4 or t.stride(3) != 1:
         raise ValueError("strided tensors must be [B, H, N, d] views with contiguous d")
-    return _lib.CStrides(t.stride(0), t.stride(1), t.stride(2))
+    # the stride of a dimension of size 1 is never used, and torch may report any value for it:
+    # pass the dense layout's stride there (a valid multiple of 16 bytes for the tensor maps)
+    B, H, N, d = t.shape
+    dense = (H * N * d, N * d, d)
+    sb, sh, sn = (dense[i] if t.shape[i] == 1 else t.stride(i) for i in range(3))
+    return _lib.CStrides(sb, sh, sn)
 
 
 def _sref(st):

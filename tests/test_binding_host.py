@@ -21,7 +21,7 @@ def test_token_major_view():
 
 
 def test_padded_rows_view():
-    x = torch.zeros(1, 2, 16, 72, dtype=torch.float16)[..., :64]
+    x = torch.zeros(2, 2, 16, 72, dtype=torch.float16)[..., :64]
     st = _strides(x)
     assert (st.b, st.h, st.n) == (2 * 16 * 72, 16 * 72, 72)
 
@@ -32,3 +32,13 @@ def test_non_unit_channel_stride_is_refused():
         _strides(x)
     with pytest.raises(ValueError):
         _strides(torch.zeros(4, 8, 16, dtype=torch.float16)[:, ::2])
+
+
+def test_strides_of_size_one_dimensions_are_the_dense_ones():
+    """torch may report any stride for a dimension of size 1; it is never used, so the dense
+    layout's stride (a valid multiple of 16 bytes) is passed instead."""
+    x = torch.zeros(1, 16, 4, 8, dtype=torch.float16).transpose(1, 2)
+    assert _strides(x).b == 4 * 16 * 8
+    y = torch.zeros(3, 16, 1, 8, dtype=torch.float16).transpose(1, 2)[:, :, ::2]
+    st = _strides(y)
+    assert (st.b, st.h, st.n) == (16 * 8, 8 * 8, 16)
